@@ -1,0 +1,225 @@
+"""Pins of the oracle's layer forward / backward.
+
+* brute force: a per-token, per-slot loop written from the definitions matches the
+  vectorised, expert-streaming oracle;
+* dense equivalence: with every expert holding the same weights the layer equals a dense
+  SwiGLU FFN of the quantised tokens times the routing-weight sum (= 1), computed with a
+  plain np.matmul chain;
+* special cases: k = 1, E = 1, T = 1;
+* backward: the exact-arithmetic gradients agree with central finite differences and
+  with torch fp64 autograd; the quantised backward with every quantiser switched to the
+  identity equals them.
+"""
+import numpy as np
+import pytest
+
+import synth
+from oracle import layer as L
+from oracle import mxfp8 as mx
+from oracle import routing as rt
+
+
+def _case(T=40, d=64, f=96, E=5, k=2, score=0, bias="none", seed=11):
+    return synth.MoeCase("t", T, d, f, E, k, score, bias, seed)
+
+
+def _inputs(case):
+    x = synth.make_x(case)
+    lg = synth.make_logits(case)
+    wcache = {}
+
+    def wfn(e):
+        if e not in wcache:
+            wcache[e] = synth.expert_weights_f64(case, e)
+        return wcache[e]
+    return x, lg, wfn
+
+
+def _brute_forward(x_bits, logits, k, score_fn, wfn):
+    """Per-token, per-slot loop straight from the definitions."""
+    x = L.bf16_bits_to_f64(x_bits)
+    T, d = x.shape
+    out = np.zeros((T, d))
+    for t in range(T):
+        xh = mx.fake_quantize_mx(x[t])
+        order = sorted(range(logits.shape[1]), key=lambda e: (-float(logits[t, e]), e))[:k]
+        sel = np.array([float(logits[t, e]) for e in order])
+        if score_fn == 0:
+            w = np.exp(sel - sel.max()); w /= w.sum()
+        else:
+            s = 1 / (1 + np.exp(-sel)); w = s / s.sum()
+        for j, e in enumerate(order):
+            Wg, Wu, Wd = wfn(e)
+            g = xh @ mx.fake_quantize_mx(Wg.T).T
+            u = xh @ mx.fake_quantize_mx(Wu.T).T
+            h = mx.fake_quantize_mx(g / (1 + np.exp(-g)) * u)
+            out[t] += w[j] * (h @ mx.fake_quantize_mx(Wd.T).T)
+    return out
+
+
+@pytest.mark.parametrize("score,bias", [(0, "none"), (1, "normal0.5"), (0, "skew1.5")])
+def test_forward_matches_bruteforce(score, bias):
+    case = _case(score=score, bias=bias)
+    x, lg, wfn = _inputs(case)
+    res = L.forward(x, lg, case.k, score, case.E, wfn)
+    ref = _brute_forward(x, lg, case.k, score, wfn)
+    assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_forward_token_sampling_matches_full():
+    case = _case(T=30)
+    x, lg, wfn = _inputs(case)
+    full = L.forward(x, lg, case.k, 0, case.E, wfn)
+    toks = np.array([0, 7, 29])
+    part = L.forward(x, lg, case.k, 0, case.E, wfn, tokens=toks)
+    assert np.array_equal(part["out"][toks], full["out"][toks])
+
+
+def test_dense_equivalence():
+    case = _case(T=48, E=6, k=3)
+    x, lg, wfn0 = _inputs(case)
+    same = wfn0(2)
+    res = L.forward(x, lg, case.k, 0, case.E, lambda e: same)
+    Wg, Wu, Wd = same
+    xh = mx.fake_quantize_mx(L.bf16_bits_to_f64(x))
+    g = np.matmul(xh, mx.fake_quantize_mx(Wg.T).T)
+    u = np.matmul(xh, mx.fake_quantize_mx(Wu.T).T)
+    h = mx.fake_quantize_mx(g * (1 / (1 + np.exp(-g))) * u)
+    dense = np.matmul(h, mx.fake_quantize_mx(Wd.T).T)
+    wsum = res["w"].sum(1, keepdims=True)
+    assert np.allclose(wsum, 1.0, atol=1e-12)
+    assert np.allclose(res["out"], wsum * dense, rtol=1e-11, atol=1e-11)
+
+
+def test_k1_is_unpermute_and_E1_is_dense():
+    case = _case(T=25, E=4, k=1)
+    x, lg, wfn = _inputs(case)
+    res = L.forward(x, lg, 1, 0, case.E, wfn, keep=True)
+    assert np.all(res["w"] == 1.0)
+    assert np.allclose(res["out"], res["y"][res["inv"]], rtol=0, atol=0)
+    case1 = _case(T=17, E=1, k=1, seed=3)
+    x1, lg1, wfn1 = _inputs(case1)
+    r1 = L.forward(x1, lg1, 1, 1, 1, wfn1, keep=True)
+    assert r1["perm"].tolist() == list(range(17))
+    assert np.allclose(r1["out"], r1["y"], rtol=0, atol=0)
+
+
+def test_T1():
+    case = _case(T=1, E=8, k=3)
+    x, lg, wfn = _inputs(case)
+    res = L.forward(x, lg, 3, 0, 8, wfn)
+    ref = _brute_forward(x, lg, 3, 0, wfn)
+    assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_exact_forward_matches_unquantised_reference():
+    case = _case(T=20, E=4, k=2)
+    x, lg, wfn = _inputs(case)
+    res = L.forward(x, lg, 2, 0, 4, wfn, exact=True)
+    ref = L.forward_exact(L.bf16_bits_to_f64(x), res["idx"], res["w"],
+                          [wfn(e) for e in range(4)])
+    assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def _tiny_problem(seed=0, T=4, d=6, f=5, E=3, k=2):
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(T, d))
+    W = [(rng.normal(size=(d, f)), rng.normal(size=(d, f)), rng.normal(size=(f, d)))
+         for _ in range(E)]
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)])
+    w = rng.uniform(0.1, 1.0, (T, k))
+    dout = rng.normal(size=(T, d))
+    return x, W, idx, w, dout
+
+
+def test_exact_backward_central_differences():
+    x, W, idx, w, dout = _tiny_problem()
+    dx, dw, dW = L.backward_exact(x, idx, w, W, dout)
+
+    def loss(x_, w_, W_):
+        return float(np.sum(dout * L.forward_exact(x_, idx, w_, W_)))
+    eps = 1e-6
+    for (t, c) in [(0, 0), (2, 3), (3, 5)]:
+        xp, xm = x.copy(), x.copy()
+        xp[t, c] += eps; xm[t, c] -= eps
+        assert abs((loss(xp, w, W) - loss(xm, w, W)) / (2 * eps) - dx[t, c]) < 1e-6
+    for (t, j) in [(0, 1), (3, 0)]:
+        wp, wm = w.copy(), w.copy()
+        wp[t, j] += eps; wm[t, j] -= eps
+        assert abs((loss(x, wp, W) - loss(x, wm, W)) / (2 * eps) - dw[t, j]) < 1e-6
+    for e, m, (r, c) in [(0, 0, (1, 2)), (1, 1, (4, 0)), (2, 2, (3, 5)), (1, 2, (0, 1))]:
+        Wp = [list(t) for t in W]; Wm = [list(t) for t in W]
+        Wp[e][m] = W[e][m].copy(); Wm[e][m] = W[e][m].copy()
+        Wp[e][m][r, c] += eps; Wm[e][m][r, c] -= eps
+        fd = (loss(x, w, [tuple(t) for t in Wp]) - loss(x, w, [tuple(t) for t in Wm])) / (2 * eps)
+        assert abs(fd - dW[e][m][r, c]) < 1e-6
+
+
+def test_exact_backward_torch_autograd():
+    torch = pytest.importorskip("torch")
+    x, W, idx, w, dout = _tiny_problem(seed=3, T=6, d=8, f=7, E=4, k=3)
+    dx, dw, dW = L.backward_exact(x, idx, w, W, dout)
+    xt = torch.tensor(x, requires_grad=True)
+    wt = torch.tensor(w, requires_grad=True)
+    Wt = [tuple(torch.tensor(m, requires_grad=True) for m in tri) for tri in W]
+    out = torch.zeros_like(xt)
+    rows = []
+    for t in range(x.shape[0]):
+        acc = 0
+        for j in range(idx.shape[1]):
+            Wg, Wu, Wd = Wt[int(idx[t, j])]
+            g, u = xt[t] @ Wg, xt[t] @ Wu
+            acc = acc + wt[t, j] * ((torch.nn.functional.silu(g) * u) @ Wd)
+        rows.append(acc)
+    out = torch.stack(rows)
+    (out * torch.tensor(dout)).sum().backward()
+    assert np.allclose(xt.grad.numpy(), dx, rtol=1e-12, atol=1e-12)
+    assert np.allclose(wt.grad.numpy(), dw, rtol=1e-12, atol=1e-12)
+    for e in range(len(W)):
+        for m in range(3):
+            g = Wt[e][m].grad
+            g = np.zeros_like(W[e][m]) if g is None else g.numpy()
+            assert np.allclose(g, dW[e][m], rtol=1e-12, atol=1e-12)
+
+
+def test_quantised_backward_with_identity_quantisers_is_exact():
+    case = _case(T=24, d=64, f=64, E=4, k=2, score=1, bias="normal0.5")
+    x, lg, wfn = _inputs(case)
+    dout = synth.make_dout(case)
+    res = L.backward(x, lg, dout, case.k, 1, case.E, wfn, exact=True)
+    W = [wfn(e) for e in range(case.E)]
+    dx, dw, dW = L.backward_exact(L.bf16_bits_to_f64(x), res["idx"], res["w"], W,
+                                  L.bf16_bits_to_f64(dout))
+    assert np.allclose(res["dx"], dx, rtol=1e-11, atol=1e-11)
+    assert np.allclose(res["dw"], dw, rtol=1e-11, atol=1e-11)
+    for e in range(case.E):
+        for m in range(3):
+            assert np.allclose(res["dW"][e][m], dW[e][m], rtol=1e-11, atol=1e-11)
+
+
+def test_quantised_backward_close_to_exact_and_empty_expert_zero():
+    case = _case(T=64, d=128, f=64, E=6, k=2, score=0, bias="skew1.5", seed=5)
+    x, lg, wfn = _inputs(case)
+    dout = synth.make_dout(case)
+    q = L.backward(x, lg, dout, case.k, 0, case.E, wfn)
+    ex = L.backward(x, lg, dout, case.k, 0, case.E, wfn, exact=True)
+
+    def rel(a, b):
+        return np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert rel(q["dx"], ex["dx"]) < 0.15
+    assert rel(q["dw"], ex["dw"]) < 0.15
+    counts = np.bincount(q["idx"].ravel(), minlength=case.E)
+    for e in range(case.E):
+        for m in range(3):
+            if counts[e] == 0:
+                assert not np.any(q["dW"][e][m])
+            else:
+                assert rel(q["dW"][e][m], ex["dW"][e][m]) < 0.15
+
+
+def test_bf16_round_matches_torch_on_fp32_values():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(9)
+    v = np.concatenate([rng.normal(0, 10, 5000), rng.normal(0, 1e-30, 100)]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(L.bf16_round(v.astype(np.float64)), ref)
