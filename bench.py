@@ -1,0 +1,379 @@
+"""Benchmark of the MoE layer hot path on B200: one JSON line on rank 0.
+
+A step is one pass of the layer over one synthetic batch of the DeepSeek-V3-shaped
+configuration (T=8192 tokens, d=7168, f=2048, E=256 experts, top-8 sigmoid-renormalised
+routing, MXFP8 expert GEMMs): route -> layout -> MXFP8 pull dispatch -> grouped GEMM
+gate/up + SwiGLU + requantisation -> grouped GEMM down -> weighted combine (forward), and,
+with --pass fwdbwd, the backward pass on the same batch.  Inputs are resident in HBM when
+the timed region starts; the weights (11.6 GB of MXFP8) exceed the 126 MB L2, so every
+step streams them from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs an independent replica on its own batch (the layer
+on one GPU does not shard; data-parallel replicas only), value = all ranks' tokens over
+the max-over-ranks device time.  --impl reference times the CPU oracle (rank 0 only) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd/bwd tokens/s at 1 B200; % of MXFP8 tensor peak and HBM BW"
+CONFIG_NAME = "dsv3"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def _workload(case, pass_):
+    return (f"{case.name} {pass_} (DeepSeek-V3-shaped MoE layer: T={case.T}, d={case.d}, "
+            f"f={case.f}, E={case.E}, top-{case.k} sigmoid-renorm, MXFP8 E4M3/E8M0, "
+            f"fp32 accumulate, bf16 out)")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        load = [s for s in sm if s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def cpu_baseline(case, budget_s: float = 15.0):
+    """The oracle forward, as it stands, on a bounded sample: the routing/layout and token
+    quantisation of the whole batch plus the expert FFNs of the first experts (index order)
+    until about ``budget_s`` of expert work; tokens/s scaled by the sampled assignments."""
+    import numpy as np
+
+    import synth
+    from oracle import layer as L
+    from oracle import routing as rt
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    x_bits, logits = synth.make_x(case), synth.make_logits(case)
+    t0 = time.perf_counter()
+    idx, w = rt.route(logits, case.k, case.score_fn)
+    counts, offsets, perm, inv = rt.layout(idx, case.E)
+    xq, xs, xhat = L.quantize_tokens(x_bits)
+    t_common = time.perf_counter() - t0
+    done_rows, t_exp, experts = 0, 0.0, 0
+    out = np.zeros((case.T, case.d))
+    wflat = w.reshape(-1)
+    for e in range(case.E):
+        rows = perm[offsets[e]:offsets[e + 1]]
+        if rows.size == 0:
+            continue
+        W = L.ExpertWeights(*synth.expert_weights_f64(case, e))
+        W.fwd()                                  # weight quantisation = preparation, untimed
+        t1 = time.perf_counter()
+        t = rows // case.k
+        y = L.expert_forward(xhat[t], W)[-1]
+        np.add.at(out, t, wflat[rows][:, None] * y)
+        t_exp += time.perf_counter() - t1
+        done_rows += rows.size
+        experts += 1
+        if t_exp >= budget_s:
+            break
+    frac = done_rows / (case.T * case.k)
+    t_total = t_exp + frac * t_common
+    value = (done_rows / case.k) / t_total
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": (f"fp64 NumPy oracle forward: routing/layout/x-quantisation of all "
+                       f"{case.T} tokens (charged pro rata) + expert FFNs of the first "
+                       f"{experts} experts ({done_rows} of {case.T * case.k} assignments); "
+                       f"{t_total:.1f} s"),
+            "host_cores_visible": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args, case):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    peaks = _peaks()
+    del peaks
+    for _ in range(args.warmup):
+        cpu_baseline(case, budget_s=0.5)
+    vals = []
+    t0 = time.perf_counter()
+    info = None
+    for _ in range(args.steps):
+        info = cpu_baseline(case, budget_s=args.ref_budget)
+        vals.append(info["value"])
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * case.T / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": _workload(case, "forward"), "pass": "forward",
+                       "T": case.T, "d": case.d, "f": case.f, "E": case.E, "k": case.k},
+            "impl": "reference",
+            "cpu_baseline": {"kind": "oracle", "cores": info["cores"], "sample": info["sample"],
+                             "value": value, "unit": "tokens/s"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": wall}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, case):
+    import numpy as np
+    import torch
+
+    import synth
+    import token_dispatch_grouped_top_b200 as moe
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    # each rank draws its own batch (seed offset by rank); weights are shared by seed
+    rcase = case.replace(seed=case.seed + 1000 * rank) if rank else case
+    dims = moe.Dims(case.T, case.d, case.f, case.E, case.k, case.score_fn)
+    x_bits, logits_np = synth.make_x(rcase), synth.make_logits(rcase)
+    wg, wu, wd = synth.expert_weights_torch(case, dev)
+    pw = moe.prepare_weights(wg, wu, wd, dims)
+    torch.cuda.synchronize()
+    del wg, wu, wd
+    torch.cuda.empty_cache()
+    x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    logits = torch.from_numpy(logits_np).to(dev)
+    ws = moe.workspace(dims, moe.OP_FORWARD, dev)
+    out = torch.empty((case.T, case.d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.forward(x, logits, pw, ws=ws, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if moe.device_status(ws) != 0:
+        raise RuntimeError("device status latched during warm-up")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    moe.profile_collect()
+    moe.profile_enable(True)
+    with ClockSampler(local) as clk:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+    moe.profile_enable(False)
+    stages = moe.profile_collect()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    status = moe.device_status(ws)
+
+    # end to end through the public API with host buffers: H2D inputs, D2H output per step
+    x_h = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_h = torch.from_numpy(logits_np).pin_memory()
+    out_h = torch.empty((case.T, case.d), dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+    lg_d = torch.empty_like(logits)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        moe.forward(x_d, lg_d, pw, ws=ws, out=out)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    peaks = _peaks()
+    A = case.T * case.k
+    mx_peak = 2.0 * peaks["bf16"]                      # MXFP8 dense = 2 x bf16 (nominal ratio)
+    flops_gateup = 4.0 * A * case.d * case.f
+    flops_down = 2.0 * A * case.d * case.f
+    w_bytes = (moe.load().moe_weights_bytes(__import__("ctypes").byref(dims.c()), 0) +
+               moe.load().moe_weights_bytes(__import__("ctypes").byref(dims.c()), 1))
+    stage_info = {}
+    for name, (tot_ms, n) in stages.items():
+        stage_info[name] = {"ms_per_launch": tot_ms / max(n, 1), "launches": n}
+    R = moe.padded_rows(dims)
+    alg_bytes = {
+        "route": 4 * case.T * case.E + 8 * A + 8 * A,
+        "permute": 2 * case.T * case.d + A * case.d * (1 + 1 / 32),
+        "combine": 4 * A * case.d + 2 * case.T * case.d,
+    }
+    for name, b in alg_bytes.items():
+        if name in stage_info:
+            s = stage_info[name]
+            s["alg_bytes"] = b
+            s["gbs"] = b / (s["ms_per_launch"] * 1e-3) / 1e9
+            s["frac_hbm"] = s["gbs"] / peaks["hbm"]
+    for name, fl in (("gateup", flops_gateup), ("down", flops_down)):
+        if name in stage_info:
+            s = stage_info[name]
+            s["flops"] = fl
+            s["tflops"] = fl / (s["ms_per_launch"] * 1e-3) / 1e12
+            s["frac_mxfp8"] = s["tflops"] / mx_peak
+    g = stage_info.get("gateup", {"ms_per_launch": float("nan"), "tflops": float("nan")})
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as fh:
+            traffic = json.load(fh).get("gateup_bytes_per_launch")
+    ms_step = ms / args.steps
+    value = world * case.T * args.steps / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "mxfp8 (e4m3 x e4m3, e8m0 scales, fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": _workload(case, "forward"), "pass": "forward", "T": case.T,
+                   "d": case.d, "f": case.f, "E": case.E, "k": case.k,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "no flush: every step streams 11.6 GB of MXFP8 weights (> 126 MB L2)"},
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<GATEUP_SWIGLU>",
+                     "achieved": g["tflops"], "peak": mx_peak, "unit": "TFLOP/s",
+                     "frac": g["tflops"] / mx_peak, "traffic": traffic,
+                     "peak_note": f"2 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
+                                  f"MXFP8:bf16 nominal ratio 2"},
+        "layer_tflops": (flops_gateup + flops_down) / (ms_step * 1e-3) / 1e12,
+        "layer_frac_mxfp8": (flops_gateup + flops_down) / (ms_step * 1e-3) / 1e12 / mx_peak,
+        "weights_gbs": w_bytes / (ms_step * 1e-3) / 1e9,
+        "stages": stage_info,
+        "gpu_launches": 6 * args.steps,
+        "device_status": status,
+        "e2e": {"value": world * case.T * args.steps / (ms_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * case.T * case.d + 4 * case.T * case.E,
+                "d2h_bytes_per_step": 2 * case.T * case.d},
+        "clocks": clk.summary(),
+        "padded_rows": R,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=CONFIG_NAME)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=4.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    import synth
+    case = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, case)
+    else:
+        run_ours(args, case)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,222 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) Mixture-of-Experts layer hot path.
+ *
+ * The method is the one described in "Cursor's MoK achieves 2.37x performance boost on
+ * NVIDIA GB300 NVL72" (kucoin news flash article): a single MoE layer that routes tokens
+ * to experts, lays them out contiguously per expert, runs the expert SwiGLU FFNs as a
+ * grouped GEMM on MXFP8 operands and combines the results back into token order with the
+ * routing weights, plus the matching backward pass.  On one GPU the article's dispatch
+ * and combine communications become on-device permutations.
+ *
+ * Conventions for every entry point
+ *   - Pointers are caller-owned DEVICE memory unless stated otherwise; row-major and
+ *     contiguous.  bf16 tensors are passed as uint16_t bit patterns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream), never allocates device memory, never synchronises and never copies
+ *     routing counts to the host (buffers are sized for the worst case instead).
+ *   - Host-side argument checks return an error before anything is launched.  Errors
+ *     found on the device (an index out of bounds, a bounded wait that ran out) are
+ *     latched into a status word inside the workspace and read back with
+ *     moe_get_device_status(); device code never traps.
+ *   - Shapes: d % 256 == 0, f % 256 == 0, 1 <= k <= min(E, 32), 1 <= E <= 1024, T >= 0,
+ *     T*k < 2^31.  Pointers must be 16-byte aligned; workspaces 256-byte aligned, and
+ *     the first 256 bytes of a workspace must be zero when it is first used (they hold
+ *     the latched device status).
+ *
+ * Notation: T tokens, d hidden size, f expert intermediate size, E experts, k experts per
+ * token, A = T*k assignments with id a = t*k + j (j = rank of the expert among the
+ * token's k choices), R = moe_padded_rows(): rows of the expert-contiguous operand
+ * buffers, in which expert e's segment starts at pad_offsets[e] (a multiple of 128).
+ *
+ * MX layouts.  MXFP8 = E4M3 bytes plus one E8M0 scale byte per 32 consecutive elements
+ * along the GEMM reduction axis K (OCP MX v1.0).  "Canonical" scales of a [rows, K]
+ * matrix are [rows, K/32] bytes.  The "UMMA" scale layout (the one the tcgen05
+ * block-scaled MMA consumes) stores the scales of a [rows, K] matrix (rows a multiple of
+ * 128, K a multiple of 128) in 512-byte chunks, one per (128-row block rb, 128-column
+ * group kg), chunk index rb*(K/128) + kg; inside a chunk the scale of row r and 32-block
+ * kb sits at byte (r%32)*16 + ((r%128)/32)*4 + (kb%4).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* outside the shape rules above */
+  MOE_ERR_MISALIGNED = 3,        /* pointer not 16-byte (workspace: 256-byte) aligned */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+  MOE_ERR_CUDA = 5,              /* a CUDA runtime call failed (launch, attribute, ...) */
+  MOE_ERR_DEVICE_TIMEOUT = 6,    /* latched: a bounded device-side wait ran out */
+  MOE_ERR_DEVICE_BOUNDS = 7,     /* latched: a device-side index check failed */
+  MOE_ERR_NO_DEVICE = 8          /* no usable sm_100 device */
+} moe_status;
+
+typedef enum { MOE_SCORE_SOFTMAX_TOPK = 0, MOE_SCORE_SIGMOID_RENORM = 1 } moe_score_fn;
+
+typedef enum { MOE_OP_ROUTE = 0, MOE_OP_FORWARD = 1, MOE_OP_BACKWARD = 2 } moe_op;
+
+typedef struct {
+  int64_t T;         /* tokens */
+  int32_t d, f, E, k;
+  int32_t score_fn;  /* moe_score_fn */
+} moe_dims;
+
+/* Expert weights in the layouts the grouped GEMMs read (written by moe_prepare_weights;
+ * sizes from moe_weights_bytes).  All MX; scales in the UMMA layout of the stated matrix. */
+typedef struct {
+  uint8_t *wgu_q;   /* [E*2f, d] E4M3: per expert, 128-row blocks alternate W_gate^T block j,
+                       W_up^T block j (rows = output features, K = d)                       */
+  uint8_t *wgu_s;   /* UMMA scales of the [E*2f, d] matrix                                 */
+  uint8_t *wd_q;    /* [E*d, f]: W_down^T per expert (rows = output features, K = f)       */
+  uint8_t *wd_s;    /* UMMA scales of the [E*d, f] matrix                                  */
+  uint8_t *wdT_q;   /* backward, nullable: [E*f, d] = W_down as stored, K = d              */
+  uint8_t *wdT_s;
+  uint8_t *wguT_q;  /* backward, nullable: [E*d, 2f] = [W_gate | W_up], K = 2f             */
+  uint8_t *wguT_s;
+} moe_weights;
+
+/* Forward state kept for the backward pass (all device buffers, caller-owned). */
+typedef struct {
+  int32_t *topk_idx;     /* [T,k]  expert of assignment a                                */
+  float   *topk_w;       /* [T,k]  combine weight                                       */
+  int32_t *counts;       /* [E]                                                         */
+  int32_t *offsets;      /* [E+1]  exclusive prefix sum of counts, offsets[E] = A       */
+  int32_t *perm;         /* [A]    position -> assignment id (expert-contiguous)        */
+  int32_t *inv_perm;     /* [A]    assignment id -> position                            */
+  int32_t *pad_offsets;  /* [E+1]  padded segment starts, multiples of 128              */
+  uint8_t *xq;           /* [R,d]  MX codes of x, permuted (row pad_offsets[e]+r)         */
+  uint8_t *xs;           /* UMMA scales of the [R,d] matrix                             */
+  uint8_t *hq;           /* [R,f]  MX codes of silu(g)*u                                */
+  uint8_t *hs;           /* UMMA scales of the [R,f] matrix                             */
+  uint16_t *gu;          /* [R,2f] bf16 SwiGLU pre-activations: g in [0,f), u in [f,2f) */
+} moe_saved;
+
+/* ---- sizes (pure host arithmetic, no CUDA call) -------------------------------------- */
+int64_t moe_padded_rows(const moe_dims* dims);
+/* Bytes of the UMMA scale layout of a [rows, K] matrix (rows rounded up to 128). */
+int64_t moe_umma_scale_bytes(int64_t rows, int64_t K);
+/* Bytes of moe_weights field `field` (0 wgu_q, 1 wgu_s, 2 wd_q, 3 wd_s, 4 wdT_q, 5 wdT_s,
+ * 6 wguT_q, 7 wguT_s); -1 on bad arguments. */
+int64_t moe_weights_bytes(const moe_dims* dims, int32_t field);
+/* Bytes of moe_saved field `field` in struct order (0 topk_idx ... 11 gu); -1 on error. */
+int64_t moe_saved_bytes(const moe_dims* dims, int32_t field);
+/* Workspace bytes for an operation (moe_op); 0 on bad arguments. */
+size_t moe_workspace_bytes(const moe_dims* dims, int32_t op);
+/* Tile-scheduler wave rule: the smallest token count M for which the tile_m x tile_n
+ * output tiles of an M x n_cols GEMM fill `waves` full waves on `num_sms` SMs:
+ * M = ceil(waves * num_sms * tile_m * tile_n / n_cols).  Article §02: a minibatch should
+ * make at least two full waves; 2368 tokens at hidden 7168 / expert intermediate 2048
+ * (gate/up GEMM, n_cols = 2*2048, 148 SMs, 128 x 256 tiles).  -1 on bad arguments. */
+int64_t moe_min_tokens_for_waves(int32_t num_sms, int32_t waves, int32_t tile_m,
+                                 int32_t tile_n, int64_t n_cols);
+
+const char* moe_status_string(moe_status s);
+
+/* ---- S1 + S2: routing and layout ------------------------------------------------------
+ * Article lead and §01 (router picks experts per token; count tokens per expert, decide
+ * placement, keep each expert's tokens contiguous).
+ * logits [T,E] fp32 -> topk_idx [T,k] (top-k by logit, ties to the lower expert index,
+ * slot j = rank), topk_w [T,k] (softmax over the k selected logits, or sigmoid scores
+ * renormalised over the k selected), counts [E], offsets [E+1], perm [A] (stable:
+ * ascending token inside each expert), inv_perm [A].  Indices are exact; weights fp32.
+ * pad_offsets [E+1] (nullable): padded segment starts.  ws: moe_workspace_bytes(ROUTE). */
+moe_status moe_route_layout(const moe_dims* dims, const float* logits, int32_t* topk_idx,
+                            float* topk_w, int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* inv_perm, int32_t* pad_offsets, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* ---- MXFP8 quantiser ------------------------------------------------------------------
+ * Article §02 (MXFP8 activations fused into dispatch, grouped GEMM and SwiGLU); format:
+ * OCP MX v1.0 (s = floor(log2 amax) - 8 clamped to [-127,127], E4M3 round-to-nearest-even
+ * with saturation to 448; an all-zero block gets scale byte 0).
+ * in [rows, K] bf16 with row stride ld (elements) -> q [rows, K] E4M3, scales:
+ * scale_layout 0 = canonical [rows, K/32]; 1 = UMMA layout (K % 128 == 0; the buffer
+ * must hold moe_umma_scale_bytes(rows, K); entries of rows >= rows are not written).
+ * K % 32 == 0. */
+moe_status mxfp8_quantize(const uint16_t* in, int64_t rows, int64_t K, int64_t ld,
+                          uint8_t* q, uint8_t* scales, int32_t scale_layout, void* stream);
+
+/* ---- weight preparation (setup, not part of the timed layer) ---------------------------
+ * W_gate, W_up [E,d,f] and W_down [E,f,d] bf16 (x @ W convention) -> the MX layouts of
+ * moe_weights.  with_backward_copies != 0 also fills wdT_* and wguT_*. */
+moe_status moe_prepare_weights(const moe_dims* dims, const uint16_t* w_gate,
+                               const uint16_t* w_up, const uint16_t* w_down,
+                               int32_t with_backward_copies, const moe_weights* out,
+                               void* stream);
+
+/* ---- S1..S7: forward ------------------------------------------------------------------
+ * Article §02/§03: route -> layout -> pull dispatch with fused MXFP8 quantisation ->
+ * grouped GEMM gate/up with SwiGLU and MXFP8 requantisation in the epilogue -> grouped
+ * GEMM down -> push combine / final weighted merge.
+ * x [T,d] bf16, logits [T,E] fp32 -> out [T,d] bf16, out_t = sum_j w[t,j] * y_{t*k+j}.
+ * saved: nullable (inference); when given, every field must be non-null and is filled
+ * for moe_backward.  ws: moe_workspace_bytes(FORWARD). */
+moe_status moe_forward(const moe_dims* dims, const moe_weights* w, const uint16_t* x,
+                       const float* logits, uint16_t* out, const moe_saved* saved,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---- S8: backward ---------------------------------------------------------------------
+ * Article §01/§02 (backward = pull reverse-combine + push reverse-dispatch).
+ * dout [T,d] bf16 + saved -> dx [T,d] bf16, dw_route [T,k] fp32 (d loss / d topk_w),
+ * dWg, dWu [E,d,f] bf16, dWd [E,f,d] bf16.  Needs the backward weight copies.
+ * Every backward GEMM operand is MX-quantised along that GEMM's K (the weight gradients
+ * along each expert's tokens); accumulation fp32.  ws: moe_workspace_bytes(BACKWARD). */
+moe_status moe_backward(const moe_dims* dims, const moe_weights* w, const moe_saved* saved,
+                        const uint16_t* dout, uint16_t* dx, float* dw_route, uint16_t* dWg,
+                        uint16_t* dWu, uint16_t* dWd, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* ---- grouped block-scaled GEMM (the engine of S4/S5, exposed for direct use) ----------
+ * For each group g and each row r in [128*mtile_prefix[g], 128*mtile_prefix[g+1]):
+ *   D[r, n] = sum_k A[r,k] * B[g*N + n, k],  n < N,  fp32 accumulation, fp32 output
+ * with A [R,K] / B [G*N,K] MX (UMMA scales).  mtile_prefix [G+1] is device memory
+ * (128-row tiles per group, prefix-summed); rows_valid [G] (nullable) limits the rows
+ * written per group.  N % 256 == 0, K % 128 == 0, R = 128*mtile_prefix[G] at most
+ * rows_a.  d_out [rows_a, N] fp32. */
+moe_status moe_grouped_gemm_mx(int32_t G, int64_t rows_a, int32_t N, int32_t K,
+                               const int32_t* mtile_prefix, const int32_t* rows_valid,
+                               const uint8_t* a_q, const uint8_t* a_s, const uint8_t* b_q,
+                               const uint8_t* b_s, float* d_out, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* ---- per-stage timing (measurement support) ------------------------------------------
+ * Stage ids of moe_forward / moe_backward launches. */
+typedef enum {
+  MOE_STAGE_ROUTE = 0,      /* S1+S2: routing, layout, perm/inv scatter                 */
+  MOE_STAGE_PERMUTE = 1,    /* S3: pull dispatch with MXFP8 quantisation                */
+  MOE_STAGE_GATEUP = 2,     /* S4: grouped GEMM gate/up + SwiGLU + requantisation        */
+  MOE_STAGE_DOWN = 3,       /* S5: grouped GEMM down                                    */
+  MOE_STAGE_COMBINE = 4,    /* S6: weighted combine / un-permute                        */
+  MOE_STAGE_BWD_DOUT = 5,   /* S8: dOut quantisation + gather                           */
+  MOE_STAGE_BWD_DGRAD_DOWN = 6,
+  MOE_STAGE_BWD_DGRAD_GATEUP = 7,
+  MOE_STAGE_BWD_DX = 8,
+  MOE_STAGE_BWD_TRANSPOSE = 9,
+  MOE_STAGE_BWD_WGRAD = 10,
+  MOE_NUM_STAGES = 11
+} moe_stage;
+
+/* When enabled, every stage launched by moe_forward / moe_backward is bracketed by CUDA
+ * events on the launch stream (host-side bookkeeping only; not for use during graph
+ * capture).  moe_profile_collect synchronises on the recorded events, writes the summed
+ * milliseconds and the number of bracketed launches per stage id, and clears the record. */
+moe_status moe_profile_enable(int32_t on);
+moe_status moe_profile_collect(double* ms_per_stage, int32_t* launches_per_stage,
+                               int32_t n_stages);
+
+/* ---- device status ------------------------------------------------------------------
+ * Synchronises `stream`, returns the status latched in the workspace (MOE_OK if none)
+ * in *code and clears it. */
+moe_status moe_get_device_status(void* ws, void* stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,638 @@
+// C ABI of the MoE layer (include/moe.h): argument checks, workspace carving, TMA
+// descriptors and the launch sequence of each entry point.  Host code only.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr int64_t kAlign = 256;
+inline int64_t align_up(int64_t x, int64_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------------------
+// argument checks (pure host logic, no CUDA call)
+// ---------------------------------------------------------------------------------------
+moe_status check_dims(const moe_dims* D) {
+  if (!D) return MOE_ERR_INVALID_ARG;
+  if (D->T < 0 || D->d <= 0 || D->f <= 0 || D->E <= 0 || D->k <= 0) return MOE_ERR_INVALID_ARG;
+  if (D->score_fn != MOE_SCORE_SOFTMAX_TOPK && D->score_fn != MOE_SCORE_SIGMOID_RENORM)
+    return MOE_ERR_INVALID_ARG;
+  if (D->E > 1024 || D->k > D->E || D->k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D->d % 256 || D->f % 256) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D->T * D->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// ---------------------------------------------------------------------------------------
+// device properties
+// ---------------------------------------------------------------------------------------
+moe_status device_sms(int* num_sms) {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_NO_DEVICE;
+  if (dev < 64 && cache[dev] > 0) {
+    *num_sms = cache[dev];
+    return MOE_OK;
+  }
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return MOE_ERR_NO_DEVICE;
+  if (major != 10) return MOE_ERR_NO_DEVICE;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_NO_DEVICE;
+  if (dev < 64) cache[dev] = sms;
+  *num_sms = sms;
+  return MOE_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D byte matrix [rows, cols] (cols contiguous), box [box_rows, 128 bytes], 128-byte swizzle.
+moe_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+inline moe_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ---------------------------------------------------------------------------------------
+// optional per-stage timing: when enabled, every stage launch of moe_forward/moe_backward
+// is bracketed by CUDA events on the launch stream; moe_profile_collect() sums them.
+// ---------------------------------------------------------------------------------------
+struct StageMark {
+  int stage;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<StageMark> g_prof_marks;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct StageScope {
+  int stage;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  StageScope(int s, cudaStream_t stream) : stage(s), st(stream) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    if (!g_prof_on) return;
+    a = prof_event();
+    cudaEventRecord(a, st);
+  }
+  ~StageScope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    cudaEvent_t b = prof_event();
+    cudaEventRecord(b, st);
+    g_prof_marks.push_back({stage, a, b});
+  }
+};
+#define MOE_TRY(x)                     \
+  do {                                 \
+    moe_status _s = (x);               \
+    if (_s != MOE_OK) return _s;       \
+  } while (0)
+
+// ---------------------------------------------------------------------------------------
+// workspace layout
+// ---------------------------------------------------------------------------------------
+struct Carve {
+  int64_t off = 0;
+  int64_t take(int64_t bytes) {
+    const int64_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  }
+};
+
+struct WsLayout {
+  // header: [0] status word; [64] tile counter; [68] done counter; [128 ...) flags
+  int64_t zero_begin = 64, zero_bytes = 0;
+  int64_t flags = 0, agg = 0, incl = 0, rank = 0, mtile = 0;
+  int64_t idx = 0, w = 0, counts = 0, offsets = 0, perm = 0, inv = 0, pad = 0;
+  int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0;
+  int64_t total = 0;
+};
+
+int64_t padded_rows(const moe_dims* D) {
+  const int64_t A = D->T * D->k;
+  return align_up(A + static_cast<int64_t>(D->E) * 127, 128);
+}
+
+WsLayout ws_layout(const moe_dims* D, int op) {
+  WsLayout L;
+  const int64_t A = D->T * D->k, E = D->E, R = padded_rows(D);
+  const int64_t nt = route_num_tiles(D->T);
+  Carve c;
+  c.take(128);  // status word + counters
+  L.flags = c.take(4 * std::max<int64_t>(nt, 1));
+  L.zero_bytes = L.flags + 4 * std::max<int64_t>(nt, 1) - L.zero_begin;
+  L.agg = c.take(4 * nt * E);
+  L.incl = c.take(4 * nt * E);
+  L.rank = c.take(4 * A);
+  L.mtile = c.take(4 * (E + 1));
+  if (op >= MOE_OP_FORWARD) {
+    L.idx = c.take(4 * A);
+    L.w = c.take(4 * A);
+    L.counts = c.take(4 * E);
+    L.offsets = c.take(4 * (E + 1));
+    L.perm = c.take(4 * A);
+    L.inv = c.take(4 * A);
+    L.pad = c.take(4 * (E + 1));
+    L.xq = c.take(R * D->d);
+    L.xs = c.take(moe_umma_scale_bytes(R, D->d));
+    L.hq = c.take(R * D->f);
+    L.hs = c.take(moe_umma_scale_bytes(R, D->f));
+    L.y = c.take(4 * R * D->d);
+  }
+  L.total = c.off;
+  return L;
+}
+
+template <class T>
+inline T* at(void* ws, int64_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status run_route(const moe_dims* D, const float* logits, int32_t* idx, float* w,
+                     int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* pad,
+                     void* ws, const WsLayout& L, int num_sms, cudaStream_t st) {
+  const int nt = route_num_tiles(D->T);
+  MOE_TRY(cuda_ok(cudaMemsetAsync(at<uint8_t>(ws, L.zero_begin), 0, L.zero_bytes, st)));
+  RouteParams P;
+  P.logits = logits;
+  P.T = D->T;
+  P.E = D->E;
+  P.k = D->k;
+  P.score_fn = D->score_fn;
+  P.num_tiles = nt;
+  P.topk_idx = idx;
+  P.topk_w = w;
+  P.rank = at<int32_t>(ws, L.rank);
+  P.counts = counts;
+  P.offsets = offsets;
+  P.mtile_prefix = at<int32_t>(ws, L.mtile);
+  P.pad_offsets = pad;
+  P.tile_counter = at<uint32_t>(ws, 64);
+  P.done_counter = at<uint32_t>(ws, 68);
+  P.flags = at<uint32_t>(ws, L.flags);
+  P.agg = at<int32_t>(ws, L.agg);
+  P.incl = at<int32_t>(ws, L.incl);
+  P.status = at<int32_t>(ws, 0);
+  return cuda_ok(launch_route_layout(P, perm, inv, num_sms, st));
+}
+
+// Routing outputs for an empty batch: all counts and offsets are zero.
+moe_status route_empty(const moe_dims* D, int32_t* counts, int32_t* offsets, int32_t* mtile,
+                       int32_t* pad, cudaStream_t st) {
+  MOE_TRY(cuda_ok(cudaMemsetAsync(counts, 0, 4 * D->E, st)));
+  MOE_TRY(cuda_ok(cudaMemsetAsync(offsets, 0, 4 * (D->E + 1), st)));
+  if (mtile) MOE_TRY(cuda_ok(cudaMemsetAsync(mtile, 0, 4 * (D->E + 1), st)));
+  if (pad) MOE_TRY(cuda_ok(cudaMemsetAsync(pad, 0, 4 * (D->E + 1), st)));
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_MISALIGNED: return "misaligned pointer";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS: return "device-side index out of bounds";
+    case MOE_ERR_NO_DEVICE: return "no sm_100 device";
+  }
+  return "unknown status";
+}
+
+int64_t moe_padded_rows(const moe_dims* dims) {
+  if (check_dims(dims) != MOE_OK) return -1;
+  return padded_rows(dims);
+}
+
+int64_t moe_umma_scale_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 128) return -1;
+  return align_up(rows, 128) * (K / 32);
+}
+
+int64_t moe_weights_bytes(const moe_dims* D, int32_t field) {
+  if (check_dims(D) != MOE_OK) return -1;
+  const int64_t E = D->E, d = D->d, f = D->f;
+  switch (field) {
+    case 0: return E * 2 * f * d;
+    case 1: return moe_umma_scale_bytes(E * 2 * f, d);
+    case 2: return E * d * f;
+    case 3: return moe_umma_scale_bytes(E * d, f);
+    case 4: return E * f * d;
+    case 5: return moe_umma_scale_bytes(E * f, d);
+    case 6: return E * d * 2 * f;
+    case 7: return moe_umma_scale_bytes(E * d, 2 * f);
+    default: return -1;
+  }
+}
+
+int64_t moe_saved_bytes(const moe_dims* D, int32_t field) {
+  if (check_dims(D) != MOE_OK) return -1;
+  const int64_t A = D->T * D->k, E = D->E, R = padded_rows(D);
+  switch (field) {
+    case 0: case 1: case 4: case 5: return 4 * A;
+    case 2: return 4 * E;
+    case 3: case 6: return 4 * (E + 1);
+    case 7: return R * D->d;
+    case 8: return moe_umma_scale_bytes(R, D->d);
+    case 9: return R * D->f;
+    case 10: return moe_umma_scale_bytes(R, D->f);
+    case 11: return R * 2 * D->f * 2;
+    default: return -1;
+  }
+}
+
+size_t moe_workspace_bytes(const moe_dims* dims, int32_t op) {
+  if (check_dims(dims) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_BACKWARD) return 0;
+  return static_cast<size_t>(ws_layout(dims, op).total);
+}
+
+int64_t moe_min_tokens_for_waves(int32_t num_sms, int32_t waves, int32_t tile_m, int32_t tile_n,
+                                 int64_t n_cols) {
+  if (num_sms <= 0 || waves <= 0 || tile_m <= 0 || tile_n <= 0 || n_cols <= 0) return -1;
+  // tokens * (n_cols / tile_n) / tile_m tiles >= waves * num_sms
+  const int64_t num = static_cast<int64_t>(waves) * num_sms * tile_m * tile_n;
+  return (num + n_cols - 1) / n_cols;
+}
+
+moe_status moe_route_layout(const moe_dims* D, const float* logits, int32_t* topk_idx,
+                            float* topk_w, int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* inv_perm, int32_t* pad_offsets, void* ws, size_t ws_bytes,
+                            void* stream) {
+  MOE_TRY(check_dims(D));
+  if (!ws || !counts || !offsets || (D->T > 0 && (!logits || !topk_idx || !topk_w || !perm ||
+                                                  !inv_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  const WsLayout L = ws_layout(D, MOE_OP_ROUTE);
+  if (ws_bytes < static_cast<size_t>(L.total)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D->T == 0) return route_empty(D, counts, offsets, at<int32_t>(ws, L.mtile), pad_offsets, st);
+  return run_route(D, logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, pad_offsets, ws,
+                   L, sms, st);
+}
+
+moe_status mxfp8_quantize(const uint16_t* in, int64_t rows, int64_t K, int64_t ld, uint8_t* q,
+                          uint8_t* scales, int32_t scale_layout, void* stream) {
+  if (rows < 0 || K <= 0 || ld < K || (scale_layout != 0 && scale_layout != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (K % 32 || (scale_layout == 1 && K % 128) || ld % 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!in || !q || !scales) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(q) || !aligned16(scales)) return MOE_ERR_MISALIGNED;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  QuantRowsParams P;
+  P.src = in;
+  P.src_ld = ld;
+  P.rows = rows;
+  P.K = K;
+  P.dst = q;
+  P.dst_ld = K;
+  P.dst_col0 = 0;
+  P.scales = scales;
+  P.layout = scale_layout;
+  P.kgroups = K / 128;
+  return cuda_ok(launch_quant_rows(P, sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_prepare_weights(const moe_dims* D, const uint16_t* wg, const uint16_t* wu,
+                               const uint16_t* wd, int32_t with_bwd, const moe_weights* out,
+                               void* stream) {
+  MOE_TRY(check_dims(D));
+  if (!wg || !wu || !wd || !out || !out->wgu_q || !out->wgu_s || !out->wd_q || !out->wd_s)
+    return MOE_ERR_INVALID_ARG;
+  if (with_bwd && (!out->wdT_q || !out->wdT_s || !out->wguT_q || !out->wguT_s))
+    return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {wg, wu, wd, out->wgu_q, out->wgu_s, out->wd_q, out->wd_s};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = D->E, d = D->d, f = D->f;
+  // gate / up: column n of W[e] ([d, f]) along d -> interleaved rows of the [E*2f, d] matrix
+  for (int half = 0; half < 2; ++half) {
+    QuantColsParams P;
+    P.src = half == 0 ? wg : wu;
+    P.G = E;
+    P.K = d;
+    P.ncols = f;
+    P.dst = out->wgu_q;
+    P.scales = out->wgu_s;
+    P.kgroups = d / 128;
+    P.map_mode = 1;
+    P.interleave_half = half;
+    MOE_TRY(cuda_ok(launch_quant_cols(P, st)));
+  }
+  {  // down: column n of W_down[e] ([f, d]) along f -> row e*d + n of the [E*d, f] matrix
+    QuantColsParams P;
+    P.src = wd;
+    P.G = E;
+    P.K = f;
+    P.ncols = d;
+    P.dst = out->wd_q;
+    P.scales = out->wd_s;
+    P.kgroups = f / 128;
+    P.map_mode = 0;
+    P.interleave_half = 0;
+    MOE_TRY(cuda_ok(launch_quant_cols(P, st)));
+  }
+  if (with_bwd) {
+    // W_down as stored: rows [E*f] along d
+    QuantRowsParams P;
+    P.src = wd;
+    P.src_ld = d;
+    P.rows = static_cast<int64_t>(E) * f;
+    P.K = d;
+    P.dst = out->wdT_q;
+    P.dst_ld = d;
+    P.dst_col0 = 0;
+    P.scales = out->wdT_s;
+    P.layout = 1;
+    P.kgroups = d / 128;
+    MOE_TRY(cuda_ok(launch_quant_rows(P, sms, st)));
+    // [W_gate | W_up] rows [E*d] along 2f
+    for (int half = 0; half < 2; ++half) {
+      QuantRowsParams Q;
+      Q.src = half == 0 ? wg : wu;
+      Q.src_ld = f;
+      Q.rows = static_cast<int64_t>(E) * d;
+      Q.K = f;
+      Q.dst = out->wguT_q;
+      Q.dst_ld = 2 * f;
+      Q.dst_col0 = half * f;
+      Q.scales = out->wguT_s;
+      Q.layout = 1;
+      Q.kgroups = 2 * f / 128;
+      MOE_TRY(cuda_ok(launch_quant_rows(Q, sms, st)));
+    }
+  }
+  return MOE_OK;
+}
+
+moe_status moe_grouped_gemm_mx(int32_t G, int64_t rows_a, int32_t N, int32_t K,
+                               const int32_t* mtile_prefix, const int32_t* rows_valid,
+                               const uint8_t* a_q, const uint8_t* a_s, const uint8_t* b_q,
+                               const uint8_t* b_s, float* d_out, void* ws, size_t ws_bytes,
+                               void* stream) {
+  if (G <= 0 || G > 1024 || rows_a < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (N % 256 || K % 128 || rows_a % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!mtile_prefix || !a_q || !a_s || !b_q || !b_s || !d_out || !ws) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < 256) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  const void* ptrs[] = {a_q, a_s, b_q, b_s, d_out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  if (rows_a == 0) return MOE_OK;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  CUtensorMap ta, tb;
+  MOE_TRY(make_tmap(&ta, a_q, rows_a, K, 128));
+  MOE_TRY(make_tmap(&tb, b_q, static_cast<int64_t>(G) * N, K, 256));
+  GemmParams P = {};
+  P.G = G;
+  P.N = N;
+  P.K = K;
+  P.mtile_prefix = mtile_prefix;
+  P.rows_valid = rows_valid;
+  P.sfa = a_s;
+  P.sfb = b_s;
+  P.out_f32 = d_out;
+  P.ld_out = N;
+  P.status = at<int32_t>(ws, 0);
+  return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32, ta, tb, P, sms,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* x,
+                       const float* logits, uint16_t* out, const moe_saved* saved, void* ws,
+                       size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(D));
+  if (!W || !ws || (D->T > 0 && (!x || !logits || !out))) return MOE_ERR_INVALID_ARG;
+  if (!W->wgu_q || !W->wgu_s || !W->wd_q || !W->wd_s) return MOE_ERR_INVALID_ARG;
+  if (saved && (!saved->topk_idx || !saved->topk_w || !saved->counts || !saved->offsets ||
+                !saved->perm || !saved->inv_perm || !saved->pad_offsets || !saved->xq ||
+                !saved->xs || !saved->hq || !saved->hs || !saved->gu))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  {
+    const void* ptrs[] = {x, logits, out, W->wgu_q, W->wgu_s, W->wd_q, W->wd_s};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+    if (saved) {
+      const void* sp[] = {saved->xq, saved->xs, saved->hq, saved->hs, saved->gu};
+      for (const void* p : sp)
+        if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+    }
+  }
+  const WsLayout L = ws_layout(D, MOE_OP_FORWARD);
+  if (ws_bytes < static_cast<size_t>(L.total)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  int32_t* idx = saved ? saved->topk_idx : at<int32_t>(ws, L.idx);
+  float* w = saved ? saved->topk_w : at<float>(ws, L.w);
+  int32_t* counts = saved ? saved->counts : at<int32_t>(ws, L.counts);
+  int32_t* offsets = saved ? saved->offsets : at<int32_t>(ws, L.offsets);
+  int32_t* perm = saved ? saved->perm : at<int32_t>(ws, L.perm);
+  int32_t* inv = saved ? saved->inv_perm : at<int32_t>(ws, L.inv);
+  int32_t* pad = saved ? saved->pad_offsets : at<int32_t>(ws, L.pad);
+  uint8_t* xq = saved ? saved->xq : at<uint8_t>(ws, L.xq);
+  uint8_t* xs = saved ? saved->xs : at<uint8_t>(ws, L.xs);
+  uint8_t* hq = saved ? saved->hq : at<uint8_t>(ws, L.hq);
+  uint8_t* hs = saved ? saved->hs : at<uint8_t>(ws, L.hs);
+  uint16_t* gu = saved ? saved->gu : nullptr;
+  int32_t* mtile = at<int32_t>(ws, L.mtile);
+  float* y = at<float>(ws, L.y);
+  int32_t* status = at<int32_t>(ws, 0);
+
+  if (D->T == 0) return route_empty(D, counts, offsets, mtile, pad, st);
+  {
+    StageScope sc(MOE_STAGE_ROUTE, st);
+    MOE_TRY(run_route(D, logits, idx, w, counts, offsets, perm, inv, pad, ws, L, sms, st));
+  }
+
+  const int64_t R = padded_rows(D);
+  {
+    StageScope sc(MOE_STAGE_PERMUTE, st);
+    PermuteParams P;
+    P.x = x;
+    P.T = D->T;
+    P.d = D->d;
+    P.E = D->E;
+    P.k = D->k;
+    P.offsets = offsets;
+    P.mtile_prefix = mtile;
+    P.perm = perm;
+    P.xq = xq;
+    P.xs = xs;
+    P.status = status;
+    MOE_TRY(cuda_ok(launch_permute_quant(P, sms, st)));
+  }
+  {
+    StageScope sc(MOE_STAGE_GATEUP, st);
+    CUtensorMap ta, tb;
+    MOE_TRY(make_tmap(&ta, xq, R, D->d, 128));
+    MOE_TRY(make_tmap(&tb, W->wgu_q, static_cast<int64_t>(D->E) * 2 * D->f, D->d, 256));
+    GemmParams P = {};
+    P.G = D->E;
+    P.N = 2 * D->f;
+    P.K = D->d;
+    P.f = D->f;
+    P.mtile_prefix = mtile;
+    P.rows_valid = counts;
+    P.sfa = xs;
+    P.sfb = W->wgu_s;
+    P.hq = hq;
+    P.hs = hs;
+    P.gu = gu;
+    P.status = status;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_SWIGLU, ta, tb, P, sms, st)));
+  }
+  {
+    StageScope sc(MOE_STAGE_DOWN, st);
+    CUtensorMap ta, tb;
+    MOE_TRY(make_tmap(&ta, hq, R, D->f, 128));
+    MOE_TRY(make_tmap(&tb, W->wd_q, static_cast<int64_t>(D->E) * D->d, D->f, 256));
+    GemmParams P = {};
+    P.G = D->E;
+    P.N = D->d;
+    P.K = D->f;
+    P.mtile_prefix = mtile;
+    P.rows_valid = counts;
+    P.sfa = hs;
+    P.sfb = W->wd_s;
+    P.out_f32 = y;
+    P.ld_out = D->d;
+    P.status = status;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32, ta, tb, P, sms, st)));
+  }
+  {
+    StageScope sc(MOE_STAGE_COMBINE, st);
+    CombineParams P;
+    P.y = y;
+    P.topk_w = w;
+    P.topk_idx = idx;
+    P.inv = inv;
+    P.offsets = offsets;
+    P.mtile_prefix = mtile;
+    P.T = D->T;
+    P.d = D->d;
+    P.E = D->E;
+    P.k = D->k;
+    P.out = out;
+    P.status = status;
+    MOE_TRY(cuda_ok(launch_combine(P, sms, st)));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved* saved,
+                        const uint16_t* dout, uint16_t* dx, float* dw_route, uint16_t* dWg,
+                        uint16_t* dWu, uint16_t* dWd, void* ws, size_t ws_bytes, void* stream) {
+  (void)W; (void)saved; (void)dout; (void)dx; (void)dw_route; (void)dWg; (void)dWu; (void)dWd;
+  (void)ws; (void)ws_bytes; (void)stream;
+  MOE_TRY(check_dims(D));
+  return MOE_ERR_UNSUPPORTED_SHAPE;
+}
+
+moe_status moe_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = on != 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_collect(double* ms_per_stage, int32_t* launches_per_stage,
+                               int32_t n_stages) {
+  if (!ms_per_stage || !launches_per_stage || n_stages <= 0) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  for (int i = 0; i < n_stages; ++i) {
+    ms_per_stage[i] = 0.0;
+    launches_per_stage[i] = 0;
+  }
+  moe_status rc = MOE_OK;
+  for (const StageMark& m : g_prof_marks) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(m.b) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, m.a, m.b) != cudaSuccess)
+      rc = MOE_ERR_CUDA;
+    if (m.stage >= 0 && m.stage < n_stages) {
+      ms_per_stage[m.stage] += ms;
+      launches_per_stage[m.stage] += 1;
+    }
+    g_prof_pool.push_back(m.a);
+    g_prof_pool.push_back(m.b);
+  }
+  g_prof_marks.clear();
+  return rc;
+}
+
+moe_status moe_get_device_status(void* ws, void* stream, int32_t* code) {
+  if (!ws || !code) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  MOE_TRY(cuda_ok(cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st)));
+  MOE_TRY(cuda_ok(cudaStreamSynchronize(st)));
+  *code = v;
+  if (v != 0) MOE_TRY(cuda_ok(cudaMemsetAsync(ws, 0, sizeof(int32_t), st)));
+  return MOE_OK;
+}
+
+}  // extern "C"

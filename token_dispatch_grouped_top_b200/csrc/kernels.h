@@ -1,0 +1,116 @@
+// Launch interfaces of the MoE-layer kernels (host <-> device plumbing, no torch types).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct RouteParams {
+  const float* logits;
+  int64_t T;
+  int E, k, score_fn;
+  int num_tiles;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* rank;          // [A] rank of each assignment inside its expert
+  int32_t* counts;        // [E]
+  int32_t* offsets;       // [E+1]
+  int32_t* mtile_prefix;  // [E+1] 128-row tiles per expert, prefix-summed
+  int32_t* pad_offsets;   // [E+1] nullable
+  uint32_t* tile_counter;
+  uint32_t* done_counter;
+  uint32_t* flags;        // [num_tiles], zeroed before the launch
+  int32_t* agg;           // [num_tiles, E]
+  int32_t* incl;          // [num_tiles, E]
+  int32_t* status;
+};
+
+cudaError_t launch_route_layout(const RouteParams& P, int32_t* perm, int32_t* inv, int num_sms,
+                                cudaStream_t stream);
+int route_num_tiles(int64_t T);
+
+// Row quantiser: rows of a bf16 matrix -> E4M3 + scales (canonical or UMMA layout).
+struct QuantRowsParams {
+  const uint16_t* src;
+  int64_t src_ld;        // elements
+  int64_t rows;
+  int64_t K;             // elements per row to quantise (multiple of 32)
+  uint8_t* dst;          // row r written at dst + r*dst_ld + dst_col0
+  int64_t dst_ld;
+  int64_t dst_col0;
+  uint8_t* scales;
+  int layout;            // 0 canonical [rows, K/32] (dst_col0 must be 0), 1 UMMA
+  int64_t kgroups;       // UMMA: (total K of the destination matrix) / 128
+};
+cudaError_t launch_quant_rows(const QuantRowsParams& P, int num_sms, cudaStream_t stream);
+
+// Column quantiser for weights: W [G][K][ncols] bf16, column n of group g quantised along K
+// and written as row rowmap(g, n) of a [*, K] E4M3 matrix with UMMA scales.
+struct QuantColsParams {
+  const uint16_t* src;
+  int G, K, ncols;
+  uint8_t* dst;
+  uint8_t* scales;
+  int64_t kgroups;       // K / 128
+  int map_mode;          // 0: row = g*ncols + n; 1: gate/up interleave (see moe.h) with
+  int interleave_half;   //    half (0 gate, 1 up): row = g*2*ncols + (n/128)*256 + half*128 + n%128
+};
+cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream);
+
+// Pull dispatch: Xq[pad_offsets[e] + r] = MX(x[perm[offsets[e] + r] / k]).
+struct PermuteParams {
+  const uint16_t* x;
+  int64_t T;
+  int d, E, k;
+  const int32_t* offsets;
+  const int32_t* mtile_prefix;
+  const int32_t* perm;
+  uint8_t* xq;
+  uint8_t* xs;
+  int32_t* status;
+};
+cudaError_t launch_permute_quant(const PermuteParams& P, int num_sms, cudaStream_t stream);
+
+// Push combine: out[t] = sum_j w[t,j] * Y[pad_offsets[e] + inv[a] - offsets[e]], bf16.
+struct CombineParams {
+  const float* y;        // [R, d] fp32
+  const float* topk_w;
+  const int32_t* topk_idx;
+  const int32_t* inv;
+  const int32_t* offsets;
+  const int32_t* mtile_prefix;
+  int64_t T;
+  int d, E, k;
+  uint16_t* out;
+  int32_t* status;
+};
+cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t stream);
+
+// Grouped block-scaled GEMM.
+enum GemmMode : int {
+  GEMM_STORE_F32 = 0,      // D fp32 [rows, N] (down projection, generic)
+  GEMM_GATEUP_SWIGLU = 1,  // SwiGLU + MX requant of h, optional bf16 g/u save
+};
+
+struct GemmParams {
+  int G;
+  int N;                 // output columns per group (multiple of 256)
+  int K;                 // reduction length (multiple of 128)
+  int f;                 // GATEUP: expert intermediate size (= N/2)
+  const int32_t* mtile_prefix;  // [G+1]
+  const int32_t* rows_valid;    // [G] nullable
+  const uint8_t* sfa;    // UMMA scales of A
+  const uint8_t* sfb;    // UMMA scales of B
+  float* out_f32;        // STORE_F32: [rows, N]
+  int64_t ld_out;
+  uint8_t* hq;           // GATEUP: [rows, f]
+  uint8_t* hs;           // GATEUP: UMMA scales of [rows, f]
+  uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16
+  int32_t* status;
+};
+cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const GemmParams& P, int num_sms, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,241 @@
+// MXFP8 quantisation kernels, the pull-dispatch permute (S3) and the push combine (S6).
+//
+// Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72":
+//   §02 -- pull dispatch: the consumer fetches the rows it needs by source and offset and
+//          lays them out by expert; MXFP8 activations are fused into dispatch, so no
+//          separate quantisation kernel and no extra HBM round trip;
+//   §02/§03 -- push combine returns each expert result to its token's slot, followed by
+//          the final weighted merge.
+// All kernels here are HBM-bound: 16-byte vector loads, one warp per row, grids sized in
+// multiples of the SM count.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kMaxE = 1024;
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& r, float (&v)[8]) {
+  v[0] = bf16_bits_to_f32(r.x & 0xFFFFu);
+  v[1] = bf16_bits_to_f32(r.x >> 16);
+  v[2] = bf16_bits_to_f32(r.y & 0xFFFFu);
+  v[3] = bf16_bits_to_f32(r.y >> 16);
+  v[4] = bf16_bits_to_f32(r.z & 0xFFFFu);
+  v[5] = bf16_bits_to_f32(r.z >> 16);
+  v[6] = bf16_bits_to_f32(r.w & 0xFFFFu);
+  v[7] = bf16_bits_to_f32(r.w >> 16);
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// One warp quantises K bf16 values of one row (K % 32 == 0).  Lane l handles 8 values per
+// 256-column step; four lanes share a 32-element block.  Scales go to the canonical
+// layout (row stride K/32, first block kb0) or to the UMMA layout (kgroups = K_total/128;
+// kb0 % 4 == 0 required).
+__device__ __forceinline__ void warp_quant_row(const uint16_t* __restrict__ src, int64_t K,
+                                               uint8_t* __restrict__ dst,
+                                               uint8_t* __restrict__ scales, int64_t row,
+                                               int64_t kb0, int layout, int64_t canon_stride,
+                                               int64_t kgroups, int lane) {
+  for (int64_t c0 = 0; c0 < K; c0 += 256) {
+    const int64_t col = c0 + lane * 8;
+    const bool in = col < K;
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (in) raw = ld_nc_v4(src + col);
+    float v[8];
+    unpack_bf16x8(raw, v);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    const int s = mx_scale_exp(amax);
+    const float inv = mx_inv_scale(s);
+    uint2 packed;
+    packed.x = pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+    packed.y = pack_e4m3x4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
+    if (in) *reinterpret_cast<uint2*>(dst + col) = packed;
+    const uint32_t sb = static_cast<uint32_t>(s + 127);
+    const int64_t kb = kb0 + (col >> 5);
+    if (layout == 0) {
+      if (in && (lane & 3) == 0) scales[row * canon_stride + kb] = static_cast<uint8_t>(sb);
+    } else {
+      const uint32_t b1 = __shfl_down_sync(kFull, sb, 4);
+      const uint32_t b2 = __shfl_down_sync(kFull, sb, 8);
+      const uint32_t b3 = __shfl_down_sync(kFull, sb, 12);
+      if (in && (lane & 15) == 0)
+        *reinterpret_cast<uint32_t*>(scales + umma_scale_offset(row, kb, kgroups)) =
+            sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsParams P) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t kb0 = P.dst_col0 >> 5;
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < P.rows; r += warps) {
+    warp_quant_row(P.src + r * P.src_ld, P.K, P.dst + r * P.dst_ld + P.dst_col0, P.scales, r,
+                   kb0, P.layout, P.K >> 5, P.kgroups, lane);
+  }
+}
+
+cudaError_t launch_quant_rows(const QuantRowsParams& P, int num_sms, cudaStream_t stream) {
+  if (P.rows <= 0) return cudaSuccess;
+  const int64_t blocks = (P.rows + 7) / 8;
+  const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
+  quant_rows_kernel<<<grid, 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+// Weights: thread per (group, 32-block along K, column); columns fastest so that the
+// strided column reads of a warp are coalesced.
+__global__ void __launch_bounds__(256) quant_cols_kernel(QuantColsParams P) {
+  const int64_t nkb = P.K >> 5;
+  const int64_t total = static_cast<int64_t>(P.G) * nkb * P.ncols;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = idx % P.ncols;
+    const int64_t rest = idx / P.ncols;
+    const int64_t kb = rest % nkb;
+    const int64_t g = rest / nkb;
+    const uint16_t* col = P.src + (g * P.K + kb * 32) * P.ncols + n;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = bf16_bits_to_f32(col[static_cast<int64_t>(i) * P.ncols]);
+    uint32_t q[8];
+    const uint32_t sb = mx_quant_block32(v, q);
+    int64_t row;
+    if (P.map_mode == 0)
+      row = g * P.ncols + n;
+    else
+      row = g * 2 * P.ncols + (n >> 7) * 256 + P.interleave_half * 128 + (n & 127);
+    uint4* dst = reinterpret_cast<uint4*>(P.dst + row * P.K + kb * 32);
+    dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+    dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+    P.scales[umma_scale_offset(row, kb, P.kgroups)] = static_cast<uint8_t>(sb);
+  }
+}
+
+cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(P.G) * (P.K >> 5) * P.ncols;
+  if (total <= 0) return cudaSuccess;
+  const int64_t blocks = (total + 255) / 256;
+  const int grid = static_cast<int>(blocks < 65536 ? blocks : 65536);
+  quant_cols_kernel<<<grid, 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+// S3: one warp per destination row; the row pulls its token by index (pull dispatch) and
+// quantises it on the way (MXFP8 fused into dispatch).
+__global__ void __launch_bounds__(256) permute_quant_kernel(PermuteParams P) {
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_mt[kMaxE + 1];
+  for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
+    s_off[i] = P.offsets[i];
+    s_mt[i] = P.mtile_prefix[i];
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t A = P.T * P.k;
+  const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); q < A;
+       q += warps) {
+    int lo = 0, hi = P.E;  // s_off[lo] <= q < s_off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_off[mid] <= q) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int a = P.perm[q];
+    const int64_t t = a / P.k;
+    const int64_t p = static_cast<int64_t>(s_mt[e]) * 128 + (q - s_off[e]);
+    if (a < 0 || t >= P.T || p >= R) {
+      if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    warp_quant_row(P.x + t * P.d, P.d, P.xq + p * P.d, P.xs, p, 0, 1, 0, P.d >> 7, lane);
+  }
+}
+
+cudaError_t launch_permute_quant(const PermuteParams& P, int num_sms, cudaStream_t stream) {
+  const int64_t A = P.T * P.k;
+  if (A <= 0) return cudaSuccess;
+  const int64_t blocks = (A + 7) / 8;
+  const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
+  permute_quant_kernel<<<grid, 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+// S6: one warp per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
+// ascending, fp32), rounded to bf16.
+__global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_mt[kMaxE + 1];
+  for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
+    s_off[i] = P.offsets[i];
+    s_mt[i] = P.mtile_prefix[i];
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int k = P.k;
+  const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+       t < P.T; t += warps) {
+    int64_t my_row = 0;
+    float my_w = 0.f;
+    bool bad = false;
+    if (lane < k) {
+      const int64_t a = t * k + lane;
+      const int e = P.topk_idx[a];
+      if (e < 0 || e >= P.E) {
+        bad = true;
+      } else {
+        my_row = static_cast<int64_t>(s_mt[e]) * 128 + (P.inv[a] - s_off[e]);
+        my_w = P.topk_w[a];
+        if (my_row < 0 || my_row >= R) bad = true;
+      }
+    }
+    if (__any_sync(kFull, bad)) {
+      if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    for (int64_t c0 = 0; c0 < P.d; c0 += 128) {
+      const int64_t col = c0 + lane * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int j = 0; j < k; ++j) {
+        const int64_t row = __shfl_sync(kFull, my_row, j);
+        const float w = __shfl_sync(kFull, my_w, j);
+        const float4 yv = __ldg(reinterpret_cast<const float4*>(P.y + row * P.d + col));
+        acc.x += w * yv.x;
+        acc.y += w * yv.y;
+        acc.z += w * yv.z;
+        acc.w += w * yv.w;
+      }
+      uint2 o;
+      o.x = f32_to_bf16_bits(acc.x) | (f32_to_bf16_bits(acc.y) << 16);
+      o.y = f32_to_bf16_bits(acc.z) | (f32_to_bf16_bits(acc.w) << 16);
+      *reinterpret_cast<uint2*>(P.out + t * P.d + col) = o;
+    }
+  }
+}
+
+cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t stream) {
+  if (P.T <= 0) return cudaSuccess;
+  const int64_t blocks = (P.T + 7) / 8;
+  const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
+  combine_kernel<<<grid, 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,333 @@
+// S1 + S2: top-k routing and the per-expert layout.
+//
+// Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72":
+//   lead / §01 -- the router picks a few experts per token at every step; before the
+//   tokens can move, the system counts each expert's tokens, decides where every token is
+//   placed and keeps one expert's tokens contiguous, all without a CPU round trip (§02).
+//
+// Two launches:
+//   route_rank_kernel   one CTA per tile of 64 tokens.  Warp-per-token top-k (ties to the
+//                       lower expert index), routing weights, a block histogram over the
+//                       experts with deterministic in-tile ranks (ballot masks, no
+//                       order-dependent atomics), and a decoupled-lookback scan of the
+//                       per-tile expert-count vectors that gives every tile its starting
+//                       rank inside each expert.  The tile that finishes last turns the
+//                       totals into counts, offsets and the padded tile prefix.
+//   scatter_kernel      pos = offsets[e] + rank; perm[pos] = a; inv[a] = pos.
+// The result is the stable counting sort: inside an expert, ascending token.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kRouteTile = 64;     // tokens per CTA
+constexpr int kRouteThreads = 256;
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 32;
+
+enum : uint32_t { FLAG_NONE = 0, FLAG_AGG = 1, FLAG_PREFIX = 2 };
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(kRouteThreads) route_rank_kernel(RouteParams P) {
+  __shared__ int s_idx[kRouteTile][kMaxK];
+  __shared__ int s_rank[kRouteTile][kMaxK];
+  __shared__ uint32_t s_mask[2][kMaxE];
+  __shared__ int s_cnt[2][kMaxE];  // per 32-token group count, then exclusive group prefix
+  __shared__ int s_excl[kMaxE];    // exclusive prefix over preceding tiles
+  __shared__ int s_part[kRouteThreads];
+  __shared__ int s_bid, s_flag, s_last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = P.E, k = P.k;
+
+  if (tid == 0) s_bid = static_cast<int>(atomicAdd(P.tile_counter, 1u));
+  for (int e = tid; e < E; e += kRouteThreads) {
+    s_mask[0][e] = s_mask[1][e] = 0u;
+    s_cnt[0][e] = s_cnt[1][e] = 0;
+  }
+  __syncthreads();
+  const int b = s_bid;
+  const int64_t t0 = static_cast<int64_t>(b) * kRouteTile;
+
+  // ---- 1. top-k per token -----------------------------------------------------------
+  for (int tl = warp; tl < kRouteTile; tl += kRouteThreads / 32) {
+    const int64_t t = t0 + tl;
+    if (t >= P.T) break;
+    const float* row = P.logits + t * E;
+    float v[NPL];
+    uint32_t removed = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = (e < E) ? row[e] : -INFINITY;
+      if (e >= E) removed |= 1u << i;
+    }
+    float sel_v = 0.f;
+    int sel_e = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (!((removed >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
+          bv = v[i];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        const float ov = __shfl_xor_sync(kFull, bv, off);
+        const int oe = __shfl_xor_sync(kFull, be, off);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) removed |= 1u << (be >> 5);
+      if (lane == j) {
+        sel_v = bv;
+        sel_e = be;
+      }
+    }
+    float score;
+    if (P.score_fn == MOE_SCORE_SOFTMAX_TOPK) {
+      const float m = __shfl_sync(kFull, sel_v, 0);  // slot 0 holds the largest logit
+      score = (lane < k) ? expf(sel_v - m) : 0.f;
+    } else {
+      score = (lane < k) ? 1.f / (1.f + expf(-sel_v)) : 0.f;
+    }
+    float sum = score;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    if (lane < k) {
+      P.topk_idx[t * k + lane] = sel_e;
+      P.topk_w[t * k + lane] = score / sum;
+      s_idx[tl][lane] = sel_e;
+    }
+  }
+  __syncthreads();
+
+  // ---- 2. deterministic ranks inside each 32-token group (token = lane) --------------
+  if (warp < kRouteTile / 32) {
+    const int g = warp, tl = 32 * g + lane;
+    const bool valid = t0 + tl < P.T;
+    if (valid)
+      for (int j = 0; j < k; ++j) atomicOr(&s_mask[g][s_idx[tl][j]], 1u << lane);
+    __syncwarp();
+    if (valid) {
+      const uint32_t below = (1u << lane) - 1u;
+      for (int j = 0; j < k; ++j) {
+        const int e = s_idx[tl][j];
+        const uint32_t m = s_mask[g][e];
+        s_rank[tl][j] = __popc(m & below);
+        if ((m & below) == 0u) s_cnt[g][e] = __popc(m);
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- 3. tile histogram, group prefix ----------------------------------------------
+  constexpr int kPer = kMaxE / kRouteThreads;
+  int hist[kPer], excl[kPer];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int e = tid + kRouteThreads * r;
+    hist[r] = 0;
+    excl[r] = 0;
+    if (e < E) {
+      const int c0 = s_cnt[0][e], c1 = s_cnt[1][e];
+      s_cnt[0][e] = 0;
+      s_cnt[1][e] = c0;
+      hist[r] = c0 + c1;
+    }
+  }
+
+  // ---- 4. decoupled lookback over the tiles' count vectors --------------------------
+  const int64_t rowE = static_cast<int64_t>(E);
+  if (b == 0) {
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int e = tid + kRouteThreads * r;
+      if (e < E) P.incl[e] = hist[r];
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release(&P.flags[0], FLAG_PREFIX);
+  } else {
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int e = tid + kRouteThreads * r;
+      if (e < E) P.agg[b * rowE + e] = hist[r];
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release(&P.flags[b], FLAG_AGG);
+    int pred = b - 1;
+    bool failed = false;
+    while (true) {
+      if (tid == 0) {
+        uint32_t f = ld_acquire(&P.flags[pred]);
+        if (f == FLAG_NONE) {
+          const uint64_t start = globaltimer_ns();
+          while ((f = ld_acquire(&P.flags[pred])) == FLAG_NONE) {
+            if (globaltimer_ns() - start > kWaitLimitNs) break;
+            __nanosleep(64);
+          }
+        }
+        s_flag = static_cast<int>(f);
+      }
+      __syncthreads();
+      const int f = s_flag;
+      if (f == FLAG_NONE) {  // bounded wait ran out: latch, publish garbage, carry on
+        failed = true;
+        break;
+      }
+      const int* src = (f == FLAG_PREFIX ? P.incl : P.agg) + pred * rowE;
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int e = tid + kRouteThreads * r;
+        if (e < E) excl[r] += __ldcg(src + e);
+      }
+      __syncthreads();  // s_flag is rewritten in the next round
+      if (f == FLAG_PREFIX) break;
+      --pred;
+    }
+    if (failed && tid == 0) latch(P.status, MOE_ERR_DEVICE_TIMEOUT);
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int e = tid + kRouteThreads * r;
+      if (e < E) P.incl[b * rowE + e] = excl[r] + hist[r];
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release(&P.flags[b], FLAG_PREFIX);
+  }
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int e = tid + kRouteThreads * r;
+    if (e < E) s_excl[e] = excl[r];
+  }
+  __syncthreads();
+
+  // ---- 5. rank of every assignment inside its expert --------------------------------
+  for (int i = tid; i < kRouteTile * k; i += kRouteThreads) {
+    const int tl = i / k, j = i - tl * k;
+    const int64_t t = t0 + tl;
+    if (t >= P.T) continue;
+    const int e = s_idx[tl][j];
+    P.rank[t * k + j] = s_excl[e] + s_cnt[tl >> 5][e] + s_rank[tl][j];
+  }
+
+  // ---- 6. the last tile to finish writes counts, offsets and the tile prefix ---------
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(P.done_counter, 1u) == static_cast<uint32_t>(P.num_tiles - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int* tot = P.incl + static_cast<int64_t>(P.num_tiles - 1) * rowE;
+  int c[kPer], m[kPer], csum = 0, msum = 0;
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {  // thread owns experts kPer*tid .. kPer*tid+kPer-1
+    const int e = kPer * tid + r;
+    c[r] = (e < E) ? __ldcg(tot + e) : 0;
+    m[r] = (c[r] + 127) >> 7;
+    csum += c[r];
+    msum += m[r];
+  }
+  // block exclusive scan of (csum, msum) packed as two passes over s_part
+  int cex = 0, mex = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    s_part[tid] = pass == 0 ? csum : msum;
+    __syncthreads();
+    for (int off = 1; off < kRouteThreads; off <<= 1) {
+      const int add = tid >= off ? s_part[tid - off] : 0;
+      __syncthreads();
+      s_part[tid] += add;
+      __syncthreads();
+    }
+    const int inc = s_part[tid];
+    (pass == 0 ? cex : mex) = inc - (pass == 0 ? csum : msum);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int e = kPer * tid + r;
+    if (e < E) {
+      P.counts[e] = c[r];
+      P.offsets[e] = cex;
+      P.mtile_prefix[e] = mex;
+      if (P.pad_offsets) P.pad_offsets[e] = mex * 128;
+    }
+    cex += c[r];
+    mex += m[r];
+  }
+  if (tid == kRouteThreads - 1) {
+    P.offsets[E] = cex;
+    P.mtile_prefix[E] = mex;
+    if (P.pad_offsets) P.pad_offsets[E] = mex * 128;
+  }
+}
+
+__global__ void scatter_kernel(const int32_t* __restrict__ topk_idx,
+                               const int32_t* __restrict__ rank,
+                               const int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+                               int32_t* __restrict__ inv, int64_t A, int E, int32_t* status) {
+  for (int64_t a = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; a < A;
+       a += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int e = topk_idx[a];
+    if (e < 0 || e >= E) {
+      latch(status, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    const int64_t pos = static_cast<int64_t>(offsets[e]) + rank[a];
+    if (pos < 0 || pos >= A) {
+      latch(status, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    perm[pos] = static_cast<int32_t>(a);
+    inv[a] = static_cast<int32_t>(pos);
+  }
+}
+
+cudaError_t launch_route_layout(const RouteParams& P, int32_t* perm, int32_t* inv,
+                                int num_sms, cudaStream_t stream) {
+  const int grid = P.num_tiles;
+  const int ept = (P.E + 31) / 32;
+  if (ept <= 1)
+    route_rank_kernel<1><<<grid, kRouteThreads, 0, stream>>>(P);
+  else if (ept <= 2)
+    route_rank_kernel<2><<<grid, kRouteThreads, 0, stream>>>(P);
+  else if (ept <= 4)
+    route_rank_kernel<4><<<grid, kRouteThreads, 0, stream>>>(P);
+  else if (ept <= 8)
+    route_rank_kernel<8><<<grid, kRouteThreads, 0, stream>>>(P);
+  else if (ept <= 16)
+    route_rank_kernel<16><<<grid, kRouteThreads, 0, stream>>>(P);
+  else
+    route_rank_kernel<32><<<grid, kRouteThreads, 0, stream>>>(P);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t A = P.T * P.k;
+  const int64_t blocks = (A + 255) / 256;
+  const int sgrid = static_cast<int>(blocks < 8 * num_sms ? blocks : 8 * num_sms);
+  scatter_kernel<<<sgrid, 256, 0, stream>>>(P.topk_idx, P.rank, P.offsets, perm, inv, A, P.E,
+                                            P.status);
+  return cudaGetLastError();
+}
+
+int route_num_tiles(int64_t T) { return static_cast<int>((T + kRouteTile - 1) / kRouteTile); }
+
+}  // namespace moe
