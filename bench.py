@@ -45,9 +45,10 @@ def _peaks():
 
 
 def _workload(case, pass_):
-    return (f"{case.name} {pass_} (DeepSeek-V3-shaped MoE layer: T={case.T}, d={case.d}, "
-            f"f={case.f}, E={case.E}, top-{case.k} sigmoid-renorm, MXFP8 E4M3/E8M0, "
-            f"fp32 accumulate, bf16 out)")
+    score = "sigmoid-renorm" if case.score_fn == 1 else "softmax-top-k"
+    return (f"{case.name} {pass_} (MoE layer: T={case.T}, d={case.d}, f={case.f}, E={case.E}, "
+            f"top-{case.k} {score}, bias {case.bias}, MXFP8 E4M3/E8M0, fp32 accumulate, "
+            f"bf16 out)")
 
 
 class ClockSampler:

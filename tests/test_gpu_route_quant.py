@@ -78,7 +78,7 @@ def test_mxfp8_edge_codes(moe):
     """Every block holds 448 (scale 2^0), so each edge value is converted as is: ties to even,
     saturation, subnormals and the sign of values that round to zero."""
     vals = [0.0, -0.0, 1.0, -1.0, 448.0, 464.0, 480.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -10,
-            1.0625, 1.1875, 2.0 ** -6, -(2.0 ** -11), 255.0, 256.0, 511.0, -464.0, 15 * 2.0 ** -10,
+            1.0625, 1.1875, 2.0 ** -6, -(2.0 ** -11), 255.0, 256.0, 510.0, -464.0, 15 * 2.0 ** -10,
             -(2.0 ** -10), 7 * 2.0 ** -9, -(3 * 2.0 ** -10)]
     x = np.zeros((len(vals), 32), np.float32)
     x[:, 0] = 448.0
