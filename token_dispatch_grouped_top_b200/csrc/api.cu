@@ -153,6 +153,9 @@ struct WsLayout {
   int64_t flags = 0, agg = 0, incl = 0, rank = 0, mtile = 0;
   int64_t idx = 0, w = 0, counts = 0, offsets = 0, perm = 0, inv = 0, pad = 0;
   int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0;
+  // backward
+  int64_t dq = 0, ds = 0, dgu_bf = 0, dgu_q = 0, dgu_s = 0, dxa = 0;
+  int64_t xt_q = 0, xt_s = 0, ht_q = 0, ht_s = 0, gt_q = 0, gt_s = 0, yt_q = 0, yt_s = 0;
   int64_t total = 0;
 };
 
@@ -173,6 +176,25 @@ WsLayout ws_layout(const moe_dims* D, int op) {
   L.incl = c.take(4 * nt * E);
   L.rank = c.take(4 * A);
   L.mtile = c.take(4 * (E + 1));
+  if (op == MOE_OP_BACKWARD) {
+    const int64_t d = D->d, f = D->f;
+    L.dq = c.take(R * d);
+    L.ds = c.take(moe_umma_scale_bytes(R, d));
+    L.dgu_bf = c.take(R * 2 * f * 2);
+    L.dgu_q = c.take(R * 2 * f);
+    L.dgu_s = c.take(moe_umma_scale_bytes(R, 2 * f));
+    L.dxa = c.take(4 * R * d);
+    L.xt_q = c.take(d * R);
+    L.xt_s = c.take(moe_umma_scale_bytes(d, R));
+    L.ht_q = c.take(f * R);
+    L.ht_s = c.take(moe_umma_scale_bytes(f, R));
+    L.gt_q = c.take(2 * f * R);
+    L.gt_s = c.take(moe_umma_scale_bytes(2 * f, R));
+    L.yt_q = c.take(d * R);
+    L.yt_s = c.take(moe_umma_scale_bytes(d, R));
+    L.total = c.off;
+    return L;
+  }
   if (op >= MOE_OP_FORWARD) {
     L.idx = c.take(4 * A);
     L.w = c.take(4 * A);
@@ -520,6 +542,7 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.k = D->k;
     P.offsets = offsets;
     P.mtile_prefix = mtile;
+    P.prefix_shift = 0;
     P.perm = perm;
     P.xq = xq;
     P.xs = xs;
@@ -573,6 +596,7 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.inv = inv;
     P.offsets = offsets;
     P.mtile_prefix = mtile;
+    P.prefix_shift = 0;
     P.T = D->T;
     P.d = D->d;
     P.E = D->E;
@@ -584,13 +608,207 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
   return MOE_OK;
 }
 
-moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved* saved,
+moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved* S,
                         const uint16_t* dout, uint16_t* dx, float* dw_route, uint16_t* dWg,
                         uint16_t* dWu, uint16_t* dWd, void* ws, size_t ws_bytes, void* stream) {
-  (void)W; (void)saved; (void)dout; (void)dx; (void)dw_route; (void)dWg; (void)dWu; (void)dWd;
-  (void)ws; (void)ws_bytes; (void)stream;
   MOE_TRY(check_dims(D));
-  return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!W || !S || !ws || !dWg || !dWu || !dWd) return MOE_ERR_INVALID_ARG;
+  if (!W->wdT_q || !W->wdT_s || !W->wguT_q || !W->wguT_s) return MOE_ERR_INVALID_ARG;
+  if (!S->topk_idx || !S->topk_w || !S->counts || !S->offsets || !S->perm || !S->inv_perm ||
+      !S->pad_offsets || !S->xq || !S->xs || !S->hq || !S->hs || !S->gu)
+    return MOE_ERR_INVALID_ARG;
+  if (D->T > 0 && (!dout || !dx || !dw_route)) return MOE_ERR_INVALID_ARG;
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  {
+    const void* ptrs[] = {dout, dx, dWg, dWu, dWd, W->wdT_q, W->wdT_s, W->wguT_q, W->wguT_s,
+                          S->xq, S->xs, S->hq, S->hs, S->gu};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  const WsLayout L = ws_layout(D, MOE_OP_BACKWARD);
+  if (ws_bytes < static_cast<size_t>(L.total)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t R = padded_rows(D);
+  const int E = D->E, d = D->d, f = D->f;
+  int32_t* status = at<int32_t>(ws, 0);
+  uint8_t* dq = at<uint8_t>(ws, L.dq);
+  uint8_t* dsc = at<uint8_t>(ws, L.ds);
+  uint16_t* dgu_bf = at<uint16_t>(ws, L.dgu_bf);
+  uint8_t* dgu_q = at<uint8_t>(ws, L.dgu_q);
+  uint8_t* dgu_s = at<uint8_t>(ws, L.dgu_s);
+  float* dxa = at<float>(ws, L.dxa);
+
+  if (D->T > 0) {
+    MOE_TRY(cuda_ok(cudaMemsetAsync(dw_route, 0, 4 * D->T * D->k, st)));
+    {  // pull reverse-combine: dOut rows gathered into expert order, MXFP8 along d
+      StageScope sc(MOE_STAGE_BWD_DOUT, st);
+      PermuteParams P;
+      P.x = dout;
+      P.T = D->T;
+      P.d = d;
+      P.E = E;
+      P.k = D->k;
+      P.offsets = S->offsets;
+      P.mtile_prefix = S->pad_offsets;
+      P.prefix_shift = 7;
+      P.perm = S->perm;
+      P.xq = dq;
+      P.xs = dsc;
+      P.status = status;
+      MOE_TRY(cuda_ok(launch_permute_quant(P, sms, st)));
+    }
+    {  // G = dOut^ . Wd'^T, dw_route, SwiGLU backward, dg/du requantisation
+      StageScope sc(MOE_STAGE_BWD_DGRAD_DOWN, st);
+      CUtensorMap ta, tb;
+      MOE_TRY(make_tmap(&ta, dq, R, d, 128));
+      MOE_TRY(make_tmap(&tb, W->wdT_q, static_cast<int64_t>(E) * f, d, 256));
+      GemmParams P = {};
+      P.G = E;
+      P.N = f;
+      P.K = d;
+      P.f = f;
+      P.mtile_prefix = S->pad_offsets;
+      P.prefix_shift = 7;
+      P.rows_valid = S->counts;
+      P.sfa = dsc;
+      P.sfb = W->wdT_s;
+      P.gu = S->gu;
+      P.h_q = S->hq;
+      P.h_s = S->hs;
+      P.perm = S->perm;
+      P.offsets = S->offsets;
+      P.topk_w = S->topk_w;
+      P.dw_route = dw_route;
+      P.dgu_bf = dgu_bf;
+      P.dgu_q = dgu_q;
+      P.dgu_s = dgu_s;
+      P.status = status;
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_DGRAD_SWIGLU, ta, tb, P, sms, st)));
+    }
+    {  // dXa = [dg|du]^ . [Wg|Wu]'^T
+      StageScope sc(MOE_STAGE_BWD_DGRAD_GATEUP, st);
+      CUtensorMap ta, tb;
+      MOE_TRY(make_tmap(&ta, dgu_q, R, 2 * f, 128));
+      MOE_TRY(make_tmap(&tb, W->wguT_q, static_cast<int64_t>(E) * d, 2 * f, 256));
+      GemmParams P = {};
+      P.G = E;
+      P.N = d;
+      P.K = 2 * f;
+      P.mtile_prefix = S->pad_offsets;
+      P.prefix_shift = 7;
+      P.rows_valid = S->counts;
+      P.sfa = dgu_s;
+      P.sfb = W->wguT_s;
+      P.out_f32 = dxa;
+      P.ld_out = d;
+      P.status = status;
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32, ta, tb, P, sms, st)));
+    }
+    {  // push reverse-dispatch: dX[t] = sum_j dXa[row of (t, j)]
+      StageScope sc(MOE_STAGE_BWD_DX, st);
+      CombineParams P;
+      P.y = dxa;
+      P.topk_w = nullptr;
+      P.topk_idx = S->topk_idx;
+      P.inv = S->inv_perm;
+      P.offsets = S->offsets;
+      P.mtile_prefix = S->pad_offsets;
+      P.prefix_shift = 7;
+      P.T = D->T;
+      P.d = d;
+      P.E = E;
+      P.k = D->k;
+      P.out = dx;
+      P.status = status;
+      MOE_TRY(cuda_ok(launch_combine(P, sms, st)));
+    }
+  }
+  uint8_t* xt_q = at<uint8_t>(ws, L.xt_q);
+  uint8_t* xt_s = at<uint8_t>(ws, L.xt_s);
+  uint8_t* ht_q = at<uint8_t>(ws, L.ht_q);
+  uint8_t* ht_s = at<uint8_t>(ws, L.ht_s);
+  uint8_t* gt_q = at<uint8_t>(ws, L.gt_q);
+  uint8_t* gt_s = at<uint8_t>(ws, L.gt_s);
+  uint8_t* yt_q = at<uint8_t>(ws, L.yt_q);
+  uint8_t* yt_s = at<uint8_t>(ws, L.yt_s);
+  if (D->T > 0) {  // token-direction MX operands of the weight gradients
+    StageScope sc(MOE_STAGE_BWD_TRANSPOSE, st);
+    TransposeQuantParams P = {};
+    P.perm = S->perm;
+    P.offsets = S->offsets;
+    P.topk_w = S->topk_w;
+    P.k = D->k;
+    P.pad_offsets = S->pad_offsets;
+    P.counts = S->counts;
+    P.E = E;
+    P.R = R;
+    P.status = status;
+    P.src = TSRC_MX;  // x^ (forward codes) -> X~^T [d, R]
+    P.q = S->xq;
+    P.s = S->xs;
+    P.C = d;
+    P.dst_q = xt_q;
+    P.dst_s = xt_s;
+    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
+    P.q = S->hq;      // h^ -> H~^T [f, R]
+    P.s = S->hs;
+    P.C = f;
+    P.dst_q = ht_q;
+    P.dst_s = ht_s;
+    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
+    P.src = TSRC_BF16;  // bf16 dg | du -> DGU~^T [2f, R]
+    P.bf = dgu_bf;
+    P.ld = 2 * f;
+    P.C = 2 * f;
+    P.dst_q = gt_q;
+    P.dst_s = gt_s;
+    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
+    P.src = TSRC_DY;    // bf16(w * dOut) gathered -> DY~^T [d, R]
+    P.bf = dout;
+    P.ld = d;
+    P.C = d;
+    P.dst_q = yt_q;
+    P.dst_s = yt_s;
+    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
+  } else {
+    // no tokens: every expert's K range is empty; the prefix below is all zeros
+  }
+  {  // weight gradients, K = each expert's token segment
+    StageScope sc(MOE_STAGE_BWD_WGRAD, st);
+    const int32_t* prefix = S->pad_offsets;
+    if (D->T == 0) MOE_TRY(cuda_ok(cudaMemsetAsync(S->pad_offsets, 0, 4 * (E + 1), st)));
+    const int64_t Kt = std::max<int64_t>(R, 128);
+    CUtensorMap ta, tb;
+    MOE_TRY(make_tmap(&ta, xt_q, d, Kt, 128));
+    MOE_TRY(make_tmap(&tb, gt_q, 2 * f, Kt, 256));
+    GemmParams P = {};
+    P.G = E;
+    P.M = d;
+    P.N = 2 * f;
+    P.K = static_cast<int>(Kt);
+    P.mtile_prefix = prefix;
+    P.prefix_shift = 7;
+    P.sfa = xt_s;
+    P.sfb = gt_s;
+    P.out_a = dWg;
+    P.out_b = dWu;
+    P.split = f;
+    P.status = status;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, P, sms, st)));
+    MOE_TRY(make_tmap(&ta, ht_q, f, Kt, 128));
+    MOE_TRY(make_tmap(&tb, yt_q, d, Kt, 256));
+    P.M = f;
+    P.N = d;
+    P.sfa = ht_s;
+    P.sfb = yt_s;
+    P.out_a = dWd;
+    P.out_b = nullptr;
+    P.split = d;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, P, sms, st)));
+  }
+  return MOE_OK;
 }
 
 moe_status moe_profile_enable(int32_t on) {

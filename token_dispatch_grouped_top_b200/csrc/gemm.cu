@@ -20,6 +20,17 @@
 //               column half (w-2)/4.
 // Tile order inside an expert is N-major (all M tiles of one weight tile back to back) so
 // that a weight tile is read from HBM once and re-read by the neighbouring CTAs from L2.
+//
+// Modes (epilogues):
+//   STORE_F32      D in fp32 (the down projection and the dgrad of the expert input).
+//   GATEUP_SWIGLU  h = silu(g) * u on paired gate/up columns, MXFP8 requantisation of h
+//                  along f (the input of the down GEMM), optional bf16 save of g and u.
+//   DGRAD_SWIGLU   backward of the down projection: G = dOut^ . Wd'^T; dw_route[a] +=
+//                  <G, h^> over the tile; dh = w * G; SwiGLU backward with the saved bf16
+//                  g, u; dg, du rounded to bf16 and requantised along f.
+//   WGRAD_BF16     weight gradients: the reduction runs over one expert's (padded) token
+//                  segment, so K varies per group and M, N are fixed; bf16 output, an
+//                  expert without tokens gets an all-zero gradient.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -53,10 +64,13 @@ constexpr size_t kGemmSmemBytes = sizeof(GemmSmem) + 1024;
 
 struct TileInfo {
   int g, i, j;
+  int kb0, nk;  // first K block and number of K blocks
   int64_t a_row0, b_row0;
 };
 
-__device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, int G, int NT, int N) {
+// Variable-M groups (forward, dgrad): group g owns 128-row tiles [prefix[g], prefix[g+1]).
+__device__ __forceinline__ TileInfo decode_tile_var_m(int tile, const int* prefix, int G, int NT,
+                                                      int N, int nk) {
   int lo = 0, hi = G;  // prefix[lo]*NT <= tile < prefix[hi]*NT
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -68,9 +82,119 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, int
   const int local = tile - prefix[lo] * NT;
   t.j = local / mt;
   t.i = local - t.j * mt;
+  t.kb0 = 0;
+  t.nk = nk;
   t.a_row0 = static_cast<int64_t>(prefix[lo] + t.i) * BM;
   t.b_row0 = static_cast<int64_t>(lo) * N + static_cast<int64_t>(t.j) * BN;
   return t;
+}
+
+// Variable-K groups (wgrad): group g reduces over K blocks [prefix[g], prefix[g+1]).
+__device__ __forceinline__ TileInfo decode_tile_var_k(int tile, const int* prefix, int MT, int NT) {
+  TileInfo t;
+  const int per = MT * NT;
+  t.g = tile / per;
+  const int local = tile - t.g * per;
+  t.i = local / NT;
+  t.j = local - t.i * NT;
+  t.kb0 = prefix[t.g];
+  t.nk = prefix[t.g + 1] - prefix[t.g];
+  t.a_row0 = static_cast<int64_t>(t.i) * BM;
+  t.b_row0 = static_cast<int64_t>(t.j) * BN;
+  return t;
+}
+
+template <int MODE>
+__device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const GemmParams& P) {
+  if (MODE == GEMM_WGRAD_BF16) return decode_tile_var_k(tile, prefix, P.M / BM, P.N / BN);
+  return decode_tile_var_m(tile, prefix, P.G, P.N / BN, P.N, P.K / BK);
+}
+
+// E4M3 byte -> fp32, exact (normal: (1 + m/8) 2^(e-7); subnormal: m 2^-9).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
+  const float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20))
+                    : static_cast<float>(m) * 0.001953125f;
+  return (c & 0x80u) ? -v : v;
+}
+
+// E8M0 byte -> 2^(b-127) as fp32 (2^-127 is subnormal).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
+  return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
+  return make_uint4(f32_to_bf16_bits(v[0]) | (f32_to_bf16_bits(v[1]) << 16),
+                    f32_to_bf16_bits(v[2]) | (f32_to_bf16_bits(v[3]) << 16),
+                    f32_to_bf16_bits(v[4]) | (f32_to_bf16_bits(v[5]) << 16),
+                    f32_to_bf16_bits(v[6]) | (f32_to_bf16_bits(v[7]) << 16));
+}
+
+// DGRAD epilogue for 32 features [fc, fc+32) of one row: returns this chunk's part of
+// <G, h^>; writes dg, du (bf16) and their MX codes/scales along f.
+__device__ __forceinline__ float dgrad_chunk(const GemmParams& P, const float (&G)[32],
+                                             int64_t row, int fc, float w) {
+  const int f = P.f;
+  const uint4* hp = reinterpret_cast<const uint4*>(P.h_q + row * f + fc);
+  const uint4 h0 = hp[0], h1 = hp[1];
+  const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  const float hsc = e8m0_to_f32(P.h_s[umma_scale_offset(row, fc >> 5, f >> 7)]);
+  const uint4* gp = reinterpret_cast<const uint4*>(P.gu + row * 2 * f + fc);
+  const uint4* up = reinterpret_cast<const uint4*>(P.gu + row * 2 * f + f + fc);
+  uint32_t dgp[16], dup[16];
+  float dwp = 0.f;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint4 gq = gp[v], uq = up[v];
+    const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+      uint32_t outg = 0, outu = 0;
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const int i = 8 * v + 2 * e2 + hlf;
+        const float g_acc = G[i];
+        const float hv = e4m3_to_f32((hw[i >> 2] >> (8 * (i & 3))) & 0xFFu) * hsc;
+        dwp = fmaf(g_acc, hv, dwp);
+        const float gb = bf16_bits_to_f32((gw[e2] >> (16 * hlf)) & 0xFFFFu);
+        const float ub = bf16_bits_to_f32((uw[e2] >> (16 * hlf)) & 0xFFFFu);
+        const float dh = w * g_acc;
+        const float sg = 1.f / (1.f + expf(-gb));
+        const float dg = dh * ub * sg * (1.f + gb * (1.f - sg));
+        const float du = dh * gb * sg;
+        outg |= f32_to_bf16_bits(dg) << (16 * hlf);
+        outu |= f32_to_bf16_bits(du) << (16 * hlf);
+      }
+      dgp[4 * v + e2] = outg;
+      dup[4 * v + e2] = outu;
+    }
+  }
+  uint4* gdst = reinterpret_cast<uint4*>(P.dgu_bf + row * 2 * f + fc);
+  uint4* udst = reinterpret_cast<uint4*>(P.dgu_bf + row * 2 * f + f + fc);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    gdst[v] = make_uint4(dgp[4 * v], dgp[4 * v + 1], dgp[4 * v + 2], dgp[4 * v + 3]);
+    udst[v] = make_uint4(dup[4 * v], dup[4 * v + 1], dup[4 * v + 2], dup[4 * v + 3]);
+  }
+#pragma unroll
+  for (int which = 0; which < 2; ++which) {  // MX requantisation of bf16 dg / du along f
+    float blk[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t wv = which ? dup[i] : dgp[i];
+      blk[2 * i] = bf16_bits_to_f32(wv & 0xFFFFu);
+      blk[2 * i + 1] = bf16_bits_to_f32(wv >> 16);
+    }
+    uint32_t qw[8];
+    const uint32_t sb = mx_quant_block32(blk, qw);
+    const int col = which * f + fc;
+    uint4* qd = reinterpret_cast<uint4*>(P.dgu_q + row * 2 * f + col);
+    qd[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+    qd[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
+    P.dgu_s[umma_scale_offset(row, col >> 5, (2 * f) >> 7)] = static_cast<uint8_t>(sb);
+  }
+  return dwp;
 }
 
 template <int MODE>
@@ -82,11 +206,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = P.G, N = P.N, NT = P.N / BN;
-  const int nk = P.K / BK;
+  const int G = P.G, NT = P.N / BN;
   const int64_t kgroups = P.K / 128;
 
-  for (int i = tid; i <= G; i += kGemmThreads) S.prefix[i] = P.mtile_prefix[i];
+  for (int i = tid; i <= G; i += kGemmThreads) S.prefix[i] = P.mtile_prefix[i] >> P.prefix_shift;
   for (int i = tid; i < G; i += kGemmThreads)
     S.valid[i] = P.rows_valid ? P.rows_valid[i] : 0x7fffffff;
   if (tid == 0) {
@@ -109,7 +232,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
-  const int total = S.prefix[G] * NT;
+  const int total = MODE == GEMM_WGRAD_BF16 ? G * (P.M / BM) * NT : S.prefix[G] * NT;
   volatile int* abort_flag = &S.abort_flag;
 
   if (warp == 0) {
@@ -118,9 +241,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, S.prefix, G, NT, N);
+        const TileInfo ti = decode_tile<MODE>(tile, S.prefix, P);
         const int64_t rbA = ti.a_row0 >> 7, rbB = ti.b_row0 >> 7;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb0 + ti.nk; ++kb) {
           if (!mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, abort_flag, P.status)) break;
           const uint32_t fb = smem_u32(&S.full[stage]);
           mbar_arrive_expect_tx(fb, kTxBytes);
@@ -144,6 +267,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       const uint32_t idesc = idesc_mxf8_e4m3(BM, BN);
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        const int nk = decode_tile<MODE>(tile, S.prefix, P).nk;
+        if (nk == 0) continue;  // empty expert (wgrad): the epilogue writes zeros
         if (!mbar_wait(smem_u32(&S.tmem_empty), acc_phase ^ 1u, abort_flag, P.status)) break;
         tc_fence_after();
         bool ok = true;
@@ -182,7 +307,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int h = (warp - 2) >> 2;   // column half
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(tile, S.prefix, G, NT, N);
+      const TileInfo ti = decode_tile<MODE>(tile, S.prefix, P);
+      if (MODE == GEMM_WGRAD_BF16 && ti.nk == 0) {
+        const int64_t m = ti.a_row0 + 32 * q + lane;
+        const int n0 = ti.j * BN + 128 * h;
+        const bool first = n0 < P.split;
+        const int ld = first ? P.split : P.N - P.split;
+        uint16_t* base = (first ? P.out_a : P.out_b) +
+                         (static_cast<int64_t>(ti.g) * P.M + m) * ld + (first ? n0 : n0 - P.split);
+        uint4* dst = reinterpret_cast<uint4*>(base);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
       if (!mbar_wait(smem_u32(&S.tmem_full), acc_phase, abort_flag, P.status)) break;
       tc_fence_after();
       const uint32_t taddr = tbase + kAccCol + (static_cast<uint32_t>(32 * q) << 16);
@@ -205,8 +342,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       acc_phase ^= 1u;
 
       const int m = 32 * q + lane;
+      if (MODE == GEMM_WGRAD_BF16) {
+        const int64_t row = ti.a_row0 + m;
+        const int n0 = ti.j * BN + 128 * h;
+        const bool first = n0 < P.split;
+        const int ld = first ? P.split : P.N - P.split;
+        uint16_t* base = (first ? P.out_a : P.out_b) +
+                         (static_cast<int64_t>(ti.g) * P.M + row) * ld +
+                         (first ? n0 : n0 - P.split);
+        uint4* dst = reinterpret_cast<uint4*>(base);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          dst[c] = pack_bf16x8(v0 + 8 * c);
+          dst[4 + c] = pack_bf16x8(v1 + 8 * c);
+          dst[8 + c] = pack_bf16x8(v2 + 8 * c);
+          dst[12 + c] = pack_bf16x8(v3 + 8 * c);
+        }
+        continue;
+      }
       if (ti.i * BM + m >= S.valid[ti.g]) continue;
       const int64_t row = ti.a_row0 + m;
+      if (MODE == GEMM_DGRAD_SWIGLU) {
+        const int64_t q_pos = static_cast<int64_t>(P.offsets[ti.g]) + ti.i * BM + m;
+        const int a = P.perm[q_pos];
+        const float w = P.topk_w[a];
+        const int n0 = ti.j * BN + 128 * h;  // first feature of this thread's 128
+        float dwp = dgrad_chunk(P, v0, row, n0, w);
+        dwp += dgrad_chunk(P, v1, row, n0 + 32, w);
+        dwp += dgrad_chunk(P, v2, row, n0 + 64, w);
+        dwp += dgrad_chunk(P, v3, row, n0 + 96, w);
+        atomicAdd(P.dw_route + a, dwp);
+        continue;
+      }
       if (MODE == GEMM_GATEUP_SWIGLU) {
         const int f = P.f;
         const int fb = BN / 2 * ti.j + 64 * h;  // first feature of this thread's 64
@@ -290,6 +457,10 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensor
       return launch_mode<GEMM_STORE_F32>(tmA, tmB, P, num_sms, stream);
     case GEMM_GATEUP_SWIGLU:
       return launch_mode<GEMM_GATEUP_SWIGLU>(tmA, tmB, P, num_sms, stream);
+    case GEMM_DGRAD_SWIGLU:
+      return launch_mode<GEMM_DGRAD_SWIGLU>(tmA, tmB, P, num_sms, stream);
+    case GEMM_WGRAD_BF16:
+      return launch_mode<GEMM_WGRAD_BF16>(tmA, tmB, P, num_sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

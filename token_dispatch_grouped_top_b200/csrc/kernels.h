@@ -65,7 +65,8 @@ struct PermuteParams {
   int64_t T;
   int d, E, k;
   const int32_t* offsets;
-  const int32_t* mtile_prefix;
+  const int32_t* mtile_prefix;  // or the padded offsets with prefix_shift = 7
+  int prefix_shift;
   const int32_t* perm;
   uint8_t* xq;
   uint8_t* xs;
@@ -74,6 +75,7 @@ struct PermuteParams {
 cudaError_t launch_permute_quant(const PermuteParams& P, int num_sms, cudaStream_t stream);
 
 // Push combine: out[t] = sum_j w[t,j] * Y[pad_offsets[e] + inv[a] - offsets[e]], bf16.
+// topk_w == nullptr: unit weights (the backward's reverse dispatch, dX = sum_j dXa).
 struct CombineParams {
   const float* y;        // [R, d] fp32
   const float* topk_w;
@@ -81,6 +83,7 @@ struct CombineParams {
   const int32_t* inv;
   const int32_t* offsets;
   const int32_t* mtile_prefix;
+  int prefix_shift;
   int64_t T;
   int d, E, k;
   uint16_t* out;
@@ -88,18 +91,52 @@ struct CombineParams {
 };
 cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t stream);
 
+// Token-direction quantiser for the weight gradients: a [R, C] operand in the padded
+// expert-contiguous row order is quantised along its rows (tokens) in blocks of 32 inside
+// each expert segment (rows past the segment's count read as zero) and stored transposed,
+// [C, R] E4M3 with the UMMA scales of the [C, R] matrix.
+enum TransposeSrc : int {
+  TSRC_MX = 0,       // MX codes [R, C] + UMMA scales (kgroups C/128): dequantised exactly
+  TSRC_BF16 = 1,     // bf16 [R, C] with row stride ld
+  TSRC_DY = 2,       // bf16(w_a * dout[t_a]) gathered from dout [T, C] (row stride ld)
+};
+struct TransposeQuantParams {
+  int src;
+  const uint8_t* q;
+  const uint8_t* s;
+  const uint16_t* bf;
+  int64_t ld;
+  const int32_t* perm;
+  const int32_t* offsets;
+  const float* topk_w;
+  int k;
+  const int32_t* pad_offsets;  // [E+1]
+  const int32_t* counts;       // [E]
+  int E;
+  int64_t R;
+  int C;
+  uint8_t* dst_q;
+  uint8_t* dst_s;
+  int32_t* status;
+};
+cudaError_t launch_transpose_quant(const TransposeQuantParams& P, cudaStream_t stream);
+
 // Grouped block-scaled GEMM.
 enum GemmMode : int {
-  GEMM_STORE_F32 = 0,      // D fp32 [rows, N] (down projection, generic)
+  GEMM_STORE_F32 = 0,      // D fp32 [rows, N] (down projection, dgrad of x, generic)
   GEMM_GATEUP_SWIGLU = 1,  // SwiGLU + MX requant of h, optional bf16 g/u save
+  GEMM_DGRAD_SWIGLU = 2,   // G = dOut . Wd^T -> dw_route, SwiGLU backward, dg/du bf16 + MX
+  GEMM_WGRAD_BF16 = 3,     // variable K per group (the group's token segment), bf16 out
 };
 
 struct GemmParams {
   int G;
   int N;                 // output columns per group (multiple of 256)
-  int K;                 // reduction length (multiple of 128)
-  int f;                 // GATEUP: expert intermediate size (= N/2)
-  const int32_t* mtile_prefix;  // [G+1]
+  int K;                 // reduction length (multiple of 128); WGRAD: total K of A and B
+  int M;                 // WGRAD: output rows per group (multiple of 128)
+  int f;                 // GATEUP / DGRAD: expert intermediate size
+  const int32_t* mtile_prefix;  // [G+1] (shifted right by prefix_shift when loaded)
+  int prefix_shift;
   const int32_t* rows_valid;    // [G] nullable
   const uint8_t* sfa;    // UMMA scales of A
   const uint8_t* sfb;    // UMMA scales of B
@@ -107,7 +144,21 @@ struct GemmParams {
   int64_t ld_out;
   uint8_t* hq;           // GATEUP: [rows, f]
   uint8_t* hs;           // GATEUP: UMMA scales of [rows, f]
-  uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16
+  uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16; DGRAD: saved g/u (read)
+  // DGRAD
+  const uint8_t* h_q;    // forward h codes [rows, f] + UMMA scales
+  const uint8_t* h_s;
+  const int32_t* perm;
+  const int32_t* offsets;
+  const float* topk_w;
+  float* dw_route;       // [A] (accumulated with atomics; zeroed before the launch)
+  uint16_t* dgu_bf;      // [rows, 2f] bf16 dg | du
+  uint8_t* dgu_q;        // [rows, 2f] MX codes + UMMA scales of the [rows, 2f] matrix
+  uint8_t* dgu_s;
+  // WGRAD: D[g] rows m < M, cols n < N -> (n < split ? out_a : out_b)[g][m][n mod split]
+  uint16_t* out_a;
+  uint16_t* out_b;
+  int split;
   int32_t* status;
 };
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB,

@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(PermuteParams P) {
   __shared__ int s_mt[kMaxE + 1];
   for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
     s_off[i] = P.offsets[i];
-    s_mt[i] = P.mtile_prefix[i];
+    s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -176,13 +176,14 @@ cudaError_t launch_permute_quant(const PermuteParams& P, int num_sms, cudaStream
 }
 
 // S6: one warp per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
-// ascending, fp32), rounded to bf16.
+// ascending, fp32), rounded to bf16.  With unit weights this is the backward's push
+// reverse-dispatch, dX[t] = sum_j dXa[row of (t, j)].
 __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_mt[kMaxE + 1];
   for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
     s_off[i] = P.offsets[i];
-    s_mt[i] = P.mtile_prefix[i];
+    s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
         bad = true;
       } else {
         my_row = static_cast<int64_t>(s_mt[e]) * 128 + (P.inv[a] - s_off[e]);
-        my_w = P.topk_w[a];
+        my_w = P.topk_w ? P.topk_w[a] : 1.f;
         if (my_row < 0 || my_row >= R) bad = true;
       }
     }
