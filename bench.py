@@ -1,10 +1,10 @@
 """Benchmark of the MoE layer hot path on B200: one JSON line on rank 0.
 
-A step is one pass of the layer over one synthetic batch of the DeepSeek-V3-shaped
+A step is one pass of the whole hot path over one synthetic batch of the DeepSeek-V3-shaped
 configuration (T=8192 tokens, d=7168, f=2048, E=256 experts, top-8 sigmoid-renormalised
 routing, MXFP8 expert GEMMs): route -> layout -> MXFP8 pull dispatch -> grouped GEMM
-gate/up + SwiGLU + requantisation -> grouped GEMM down -> weighted combine (forward), and,
-with --pass fwdbwd, the backward pass on the same batch.  Inputs are resident in HBM when
+gate/up + SwiGLU + requantisation -> grouped GEMM down -> weighted combine (forward), then
+the backward pass on the same batch (--pass fwd times the forward alone).  Inputs are resident in HBM when
 the timed region starts; the weights (11.6 GB of MXFP8) exceed the 126 MB L2, so every
 step streams them from HBM.
 
@@ -115,10 +115,12 @@ def _dist():
     return ws, rank, local
 
 
-def cpu_baseline(case, budget_s: float = 15.0):
-    """The oracle forward, as it stands, on a bounded sample: the routing/layout and token
-    quantisation of the whole batch plus the expert FFNs of the first experts (index order)
-    until about ``budget_s`` of expert work; tokens/s scaled by the sampled assignments."""
+def cpu_baseline(case, budget_s: float = 15.0, with_bwd: bool = False):
+    """The oracle, as it stands, on a bounded sample: routing/layout and token quantisation
+    of the whole batch plus the expert FFNs of the first experts (index order) until about
+    ``budget_s`` of expert work; tokens/s scaled by the sampled assignments.  With
+    ``with_bwd`` the oracle backward of the same experts is timed too (weights prepared
+    ahead, as on the GPU; its whole-batch routing/quantisation is charged in full)."""
     import numpy as np
 
     import synth
@@ -135,32 +137,44 @@ def cpu_baseline(case, budget_s: float = 15.0):
     counts, offsets, perm, inv = rt.layout(idx, case.E)
     xq, xs, xhat = L.quantize_tokens(x_bits)
     t_common = time.perf_counter() - t0
-    done_rows, t_exp, experts = 0, 0.0, 0
+    done_rows, t_exp, experts = 0, 0.0, []
     out = np.zeros((case.T, case.d))
     wflat = w.reshape(-1)
+    prepared = {}
     for e in range(case.E):
         rows = perm[offsets[e]:offsets[e + 1]]
         if rows.size == 0:
             continue
         W = L.ExpertWeights(*synth.expert_weights_f64(case, e))
         W.fwd()                                  # weight quantisation = preparation, untimed
+        if with_bwd:
+            W.bwd()
+        prepared[e] = W
         t1 = time.perf_counter()
         t = rows // case.k
         y = L.expert_forward(xhat[t], W)[-1]
         np.add.at(out, t, wflat[rows][:, None] * y)
         t_exp += time.perf_counter() - t1
         done_rows += rows.size
-        experts += 1
+        experts.append(e)
         if t_exp >= budget_s:
             break
     frac = done_rows / (case.T * case.k)
     t_total = t_exp + frac * t_common
-    value = (done_rows / case.k) / t_total
+    t_bwd = 0.0
+    if with_bwd:
+        dout_bits = synth.make_dout(case)
+        t2 = time.perf_counter()
+        L.backward(x_bits, logits, dout_bits, case.k, case.score_fn, case.E,
+                   lambda e: None, experts=experts, prepared=prepared)
+        t_bwd = time.perf_counter() - t2
+    value = (done_rows / case.k) / (t_total + t_bwd)
+    what = "forward + backward" if with_bwd else "forward"
     return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": (f"fp64 NumPy oracle forward: routing/layout/x-quantisation of all "
-                       f"{case.T} tokens (charged pro rata) + expert FFNs of the first "
-                       f"{experts} experts ({done_rows} of {case.T * case.k} assignments); "
-                       f"{t_total:.1f} s"),
+            "sample": (f"fp64 NumPy oracle {what}: routing/layout/x-quantisation of all "
+                       f"{case.T} tokens (forward: charged pro rata) + the experts' FFNs of the "
+                       f"first {len(experts)} experts ({done_rows} of {case.T * case.k} "
+                       f"assignments); {t_total + t_bwd:.1f} s"),
             "host_cores_visible": len(os.sched_getaffinity(0))}
 
 
@@ -170,13 +184,14 @@ def run_reference(args, case):
         return
     peaks = _peaks()
     del peaks
+    bwd = args.pass_ == "fwdbwd"
     for _ in range(args.warmup):
-        cpu_baseline(case, budget_s=0.5)
+        cpu_baseline(case, budget_s=0.2, with_bwd=bwd)
     vals = []
     t0 = time.perf_counter()
     info = None
     for _ in range(args.steps):
-        info = cpu_baseline(case, budget_s=args.ref_budget)
+        info = cpu_baseline(case, budget_s=args.ref_budget, with_bwd=bwd)
         vals.append(info["value"])
     wall = time.perf_counter() - t0
     value = statistics.median(vals)
@@ -184,7 +199,8 @@ def run_reference(args, case):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * case.T / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": _workload(case, "forward"), "pass": "forward",
+            "config": {"workload": _workload(case, "forward+backward" if bwd else "forward"),
+                       "pass": "forward+backward" if bwd else "forward",
                        "T": case.T, "d": case.d, "f": case.f, "E": case.E, "k": case.k},
             "impl": "reference",
             "cpu_baseline": {"kind": "oracle", "cores": info["cores"], "sample": info["sample"],
@@ -195,7 +211,15 @@ def run_reference(args, case):
     print(json.dumps(line), flush=True)
 
 
+# kernels launched per stage (route: routing + scatter; transposes: 4; wgrad: 2 GEMMs)
+KERNELS_PER_STAGE = {"route": 2, "permute": 1, "gateup": 1, "down": 1, "combine": 1,
+                     "bwd_dout": 1, "bwd_dgrad_down": 1, "bwd_dgrad_gateup": 1, "bwd_dx": 1,
+                     "bwd_transpose": 4, "bwd_wgrad": 2}
+
+
 def run_ours(args, case):
+    import ctypes
+
     import numpy as np
     import torch
 
@@ -209,12 +233,14 @@ def run_ours(args, case):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
+    bwd = args.pass_ == "fwdbwd"
     # each rank draws its own batch (seed offset by rank); weights are shared by seed
     rcase = case.replace(seed=case.seed + 1000 * rank) if rank else case
     dims = moe.Dims(case.T, case.d, case.f, case.E, case.k, case.score_fn)
     x_bits, logits_np = synth.make_x(rcase), synth.make_logits(rcase)
+    dout_bits = synth.make_dout(rcase) if bwd else None
     wg, wu, wd = synth.expert_weights_torch(case, dev)
-    pw = moe.prepare_weights(wg, wu, wd, dims)
+    pw = moe.prepare_weights(wg, wu, wd, dims, with_backward=bwd)
     torch.cuda.synchronize()
     del wg, wu, wd
     torch.cuda.empty_cache()
@@ -223,14 +249,27 @@ def run_ours(args, case):
     ws = moe.workspace(dims, moe.OP_FORWARD, dev)
     out = torch.empty((case.T, case.d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
+    saved = moe.alloc_saved(dims, dev) if bwd else None
+    if bwd:
+        dout = torch.from_numpy(dout_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        wsb = moe.workspace(dims, moe.OP_BACKWARD, dev)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        grads = dict(dx=torch.empty((case.T, case.d), **bf),
+                     dw_route=torch.empty((case.T, case.k), dtype=torch.float32, device=dev),
+                     dWg=torch.empty((case.E, case.d, case.f), **bf),
+                     dWu=torch.empty((case.E, case.d, case.f), **bf),
+                     dWd=torch.empty((case.E, case.f, case.d), **bf))
 
-    def step():
-        moe.forward(x, logits, pw, ws=ws, out=out)
+    def step(xx=None, ll=None, dd=None):
+        moe.forward(x if xx is None else xx, logits if ll is None else ll, pw, ws=ws, out=out,
+                    saved=saved)
+        if bwd:
+            moe.backward(dout if dd is None else dd, pw, saved, ws=wsb, outs=grads)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    if moe.device_status(ws) != 0:
+    if moe.device_status(ws) != 0 or (bwd and moe.device_status(wsb) != 0):
         raise RuntimeError("device status latched during warm-up")
 
     def barrier():
@@ -255,20 +294,33 @@ def run_ours(args, case):
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    status = moe.device_status(ws)
+    status = moe.device_status(ws) | (moe.device_status(wsb) if bwd else 0)
 
-    # end to end through the public API with host buffers: H2D inputs, D2H output per step
+    # end to end through the public API with host buffers: H2D inputs, D2H results per step
     x_h = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     lg_h = torch.from_numpy(logits_np).pin_memory()
     out_h = torch.empty((case.T, case.d), dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(x)
-    lg_d = torch.empty_like(logits)
+    x_d, lg_d = torch.empty_like(x), torch.empty_like(logits)
+    h2d = 2 * case.T * case.d + 4 * case.T * case.E
+    d2h = 2 * case.T * case.d
+    if bwd:
+        do_h = torch.from_numpy(dout_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        dx_h = torch.empty((case.T, case.d), dtype=torch.bfloat16).pin_memory()
+        dw_h = torch.empty((case.T, case.k), dtype=torch.float32).pin_memory()
+        do_d = torch.empty_like(dout)
+        h2d += 2 * case.T * case.d
+        d2h += 2 * case.T * case.d + 4 * case.T * case.k
 
     def e2e_step():
         x_d.copy_(x_h, non_blocking=True)
         lg_d.copy_(lg_h, non_blocking=True)
-        moe.forward(x_d, lg_d, pw, ws=ws, out=out)
+        if bwd:
+            do_d.copy_(do_h, non_blocking=True)
+        step(x_d, lg_d, do_d if bwd else None)
         out_h.copy_(out, non_blocking=True)
+        if bwd:
+            dx_h.copy_(grads["dx"], non_blocking=True)
+            dw_h.copy_(grads["dw_route"], non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -288,31 +340,32 @@ def run_ours(args, case):
     peaks = _peaks()
     A = case.T * case.k
     mx_peak = 2.0 * peaks["bf16"]                      # MXFP8 dense = 2 x bf16 (nominal ratio)
-    flops_gateup = 4.0 * A * case.d * case.f
-    flops_down = 2.0 * A * case.d * case.f
-    w_bytes = (moe.load().moe_weights_bytes(__import__("ctypes").byref(dims.c()), 0) +
-               moe.load().moe_weights_bytes(__import__("ctypes").byref(dims.c()), 1))
-    stage_info = {}
-    for name, (tot_ms, n) in stages.items():
-        stage_info[name] = {"ms_per_launch": tot_ms / max(n, 1), "launches": n}
-    R = moe.padded_rows(dims)
+    fl = {"gateup": 4.0 * A * case.d * case.f, "down": 2.0 * A * case.d * case.f,
+          "bwd_dgrad_down": 2.0 * A * case.d * case.f,
+          "bwd_dgrad_gateup": 4.0 * A * case.d * case.f,
+          "bwd_wgrad": 6.0 * A * case.d * case.f}
+    cd = dims.c()
+    lib = moe.load()
+    w_bytes = sum(lib.moe_weights_bytes(ctypes.byref(cd), i) for i in range(4))
     alg_bytes = {
         "route": 4 * case.T * case.E + 8 * A + 8 * A,
         "permute": 2 * case.T * case.d + A * case.d * (1 + 1 / 32),
         "combine": 4 * A * case.d + 2 * case.T * case.d,
+        "bwd_dout": 2 * case.T * case.d + A * case.d * (1 + 1 / 32),
+        "bwd_dx": 4 * A * case.d + 2 * case.T * case.d,
     }
-    for name, b in alg_bytes.items():
-        if name in stage_info:
-            s = stage_info[name]
-            s["alg_bytes"] = b
-            s["gbs"] = b / (s["ms_per_launch"] * 1e-3) / 1e9
+    stage_info = {}
+    for name, (tot_ms, n) in stages.items():
+        s = {"ms_per_launch": tot_ms / max(n, 1), "launches": n}
+        if name in alg_bytes:
+            s["alg_bytes"] = alg_bytes[name]
+            s["gbs"] = alg_bytes[name] / (s["ms_per_launch"] * 1e-3) / 1e9
             s["frac_hbm"] = s["gbs"] / peaks["hbm"]
-    for name, fl in (("gateup", flops_gateup), ("down", flops_down)):
-        if name in stage_info:
-            s = stage_info[name]
-            s["flops"] = fl
-            s["tflops"] = fl / (s["ms_per_launch"] * 1e-3) / 1e12
+        if name in fl:
+            s["flops"] = fl[name]
+            s["tflops"] = fl[name] / (s["ms_per_launch"] * 1e-3) / 1e12
             s["frac_mxfp8"] = s["tflops"] / mx_peak
+        stage_info[name] = s
     g = stage_info.get("gateup", {"ms_per_launch": float("nan"), "tflops": float("nan")})
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
@@ -321,12 +374,17 @@ def run_ours(args, case):
             traffic = json.load(fh).get("gateup_bytes_per_launch")
     ms_step = ms / args.steps
     value = world * case.T * args.steps / (ms * 1e-3)
+    fwd_ms = sum(v["ms_per_launch"] for k, v in stage_info.items() if not k.startswith("bwd"))
+    bwd_ms = sum(v["ms_per_launch"] for k, v in stage_info.items() if k.startswith("bwd"))
+    layer_flops = sum(fl[k] for k in fl if bwd or not k.startswith("bwd"))
+    launches = sum(KERNELS_PER_STAGE[k] * v["launches"] for k, v in stage_info.items())
+    pass_name = "forward+backward" if bwd else "forward"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "mxfp8 (e4m3 x e4m3, e8m0 scales, fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": _workload(case, "forward"), "pass": "forward", "T": case.T,
+        "config": {"workload": _workload(case, pass_name), "pass": pass_name, "T": case.T,
                    "d": case.d, "f": case.f, "E": case.E, "k": case.k,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "no flush: every step streams 11.6 GB of MXFP8 weights (> 126 MB L2)"},
@@ -335,25 +393,41 @@ def run_ours(args, case):
                      "frac": g["tflops"] / mx_peak, "traffic": traffic,
                      "peak_note": f"2 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
                                   f"MXFP8:bf16 nominal ratio 2"},
-        "layer_tflops": (flops_gateup + flops_down) / (ms_step * 1e-3) / 1e12,
-        "layer_frac_mxfp8": (flops_gateup + flops_down) / (ms_step * 1e-3) / 1e12 / mx_peak,
-        "weights_gbs": w_bytes / (ms_step * 1e-3) / 1e9,
+        "fwd_tokens_per_s": world * case.T / (fwd_ms * 1e-3),
+        "bwd_tokens_per_s": world * case.T / (bwd_ms * 1e-3) if bwd else None,
+        "layer_tflops": layer_flops / (ms_step * 1e-3) / 1e12,
+        "layer_frac_mxfp8": layer_flops / (ms_step * 1e-3) / 1e12 / mx_peak,
+        "weights_gbs_fwd": w_bytes / (fwd_ms * 1e-3) / 1e9,
         "stages": stage_info,
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": launches,
         "device_status": status,
         "e2e": {"value": world * case.T * args.steps / (ms_e2e * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": 2 * case.T * case.d + 4 * case.T * case.E,
-                "d2h_bytes_per_step": 2 * case.T * case.d},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
-        "padded_rows": R,
+        "padded_rows": moe.padded_rows(dims),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget, with_bwd=bwd)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def sweep(args):
+    """One JSON line per synthetic configuration (forward; backward for the backward config).
+    Not the default line: a table for the design notes."""
+    import subprocess as sp
+    for name in ("tiny", "mid", "dsv3", "imbalance", "dsv3_bwd"):
+        cmd = [sys.executable, os.path.abspath(__file__), "--config", name, "--steps",
+               str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline"]
+        if name == "dsv3_bwd":
+            cmd += ["--pass", "fwdbwd"]
+        r = sp.run(cmd, capture_output=True, text=True)
+        line = r.stdout.strip().splitlines()[-1] if r.stdout.strip() else json.dumps(
+            {"config": name, "error": r.stderr[-500:]})
+        print(line, flush=True)
 
 
 def main():
@@ -363,13 +437,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=CONFIG_NAME)
+    ap.add_argument("--pass", dest="pass_", default="fwdbwd", choices=["fwd", "fwdbwd"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=4.0)
+    ap.add_argument("--sweep", action="store_true", help="every synthetic config, one line each")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     import synth
     case = synth.CONFIGS[args.config]
+    if args.sweep:
+        sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args, case)
     else:

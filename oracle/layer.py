@@ -163,12 +163,13 @@ def forward(x_bits, logits, k, score_fn, E, weights_fn, tokens=None, keep=False,
 
 
 def backward(x_bits, logits, dout_bits, k, score_fn, E, weights_fn, experts=None,
-             want_dx=True, exact=False):
+             want_dx=True, exact=False, prepared=None):
     """Oracle backward (quantised reading, see module docstring).
 
     Returns dict with dx [T,d] (fp64, contributions of the processed experts only when
     ``experts`` is given), dw [T,k], and dW = {e: (dWg [d,f], dWu [d,f], dWd [f,d])} for
-    the processed experts.
+    the processed experts.  ``prepared``: optional {e: ExpertWeights} whose quantised
+    weight views are reused (weight preparation done ahead of time).
     """
     T, d = x_bits.shape
     idx, w = rt.route(logits, k, score_fn)
@@ -185,7 +186,8 @@ def backward(x_bits, logits, dout_bits, k, score_fn, E, weights_fn, experts=None
     todo = range(E) if experts is None else experts
     for e in todo:
         rows = perm[offsets[e]:offsets[e + 1]]
-        W = ExpertWeights(*weights_fn(e), exact=exact)
+        W = prepared[e] if prepared and e in prepared else ExpertWeights(*weights_fn(e),
+                                                                        exact=exact)
         f = W.wg.shape[1]
         if rows.size == 0:
             dW[e] = (np.zeros((d, f)), np.zeros((d, f)), np.zeros((f, d)))

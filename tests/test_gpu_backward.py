@@ -1,15 +1,22 @@
 """GPU parity of the backward pass (S8) against the fp64 oracle on the same quantised operands.
 
-dX, the weight gradients (bf16) and d(routing weights) (fp32) must reach relative
-Frobenius error <= 2e-3 and max-abs <= 3e-2*RMS; an expert without tokens gets an exactly
-zero weight gradient.
+dX and d(routing weights) must reach relative Frobenius error <= 2e-3 and max-abs <=
+3e-2*RMS.  The weight gradients reach relative Frobenius <= 2e-3 per expert matrix; their
+element-wise bound allows for requantisation decisions: dg, du and w*dOut are computed
+values (fp32 on the GPU, fp64 in the oracle) that are rounded to bf16 and quantised to
+E4M3 along the tokens, so a value on a rounding boundary can land one code apart, and
+in a sum over an expert's tokens one such code moves an element by up to ~0.1*RMS (the
+oracle itself does this under 1e-6 relative noise).  Elements beyond 3e-2*RMS must be
+rare (<= 1e-4 of all weight-gradient elements) and below 0.25*RMS.  An expert without
+tokens gets an exactly zero weight gradient.
 """
 import numpy as np
 import pytest
 
 import synth
 from oracle import layer as olayer
-from tests.gpu_util import assert_close_out, bf16_tensor_f64, bits_to_bf16_tensor, to_np
+from tests.gpu_util import (assert_close_out, bf16_tensor_f64, bits_to_bf16_tensor, rel_fro,
+                            to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,6 +70,8 @@ def _check(moe, case, tokens=None, experts=None):
     print(f"{case.name} dw_route:")
     assert_close_out(dw[rows], ref["dw"][rows])
     names = ("dWg", "dWu", "dWd")
+    n_el = n_out = 0
+    worst = 0.0
     for e in (ref["dW"].keys() if experts is None else experts):
         for m, name in enumerate(names):
             got = bf16_tensor_f64(grads[name][e])
@@ -70,8 +79,15 @@ def _check(moe, case, tokens=None, experts=None):
             if not np.any(want):
                 assert not np.any(got), f"{name}[{e}] of an expert without tokens is not zero"
                 continue
-            print(f"{case.name} {name}[{e}]:")
-            assert_close_out(got, want)
+            err = rel_fro(got, want)
+            assert err <= 2e-3, f"{name}[{e}]: relative Frobenius error {err:.3e}"
+            rms = float(np.sqrt(np.mean(want ** 2)))
+            dev = np.abs(got - want) / rms
+            n_el += dev.size
+            n_out += int(np.sum(dev > 3e-2))
+            worst = max(worst, float(dev.max()))
+    print(f"{case.name} dW: {n_out} of {n_el} elements beyond 3e-2*RMS, worst {worst:.3e}*RMS")
+    assert n_out <= 1e-4 * max(n_el, 1) and worst <= 0.25
 
 
 def test_backward_small_full(moe):

@@ -2,7 +2,8 @@
 
 * exact GEMM: E4M3 operands that are small integers, with power-of-two block scales, keep
   every fp32 partial sum exact, so the tcgen05 grouped GEMM must equal np.matmul bit for
-  bit -- including ragged groups, empty groups and padding rows.
+  bit -- including ragged groups (whose last tile runs with the operands swapped, as
+  wide as its valid rows) and empty groups.
 * weights: every MX byte and scale equals the oracle's quantisation of the same bf16 bits.
 * forward: routing/layout and the permuted MX activations bit-exact; the requantised
   SwiGLU output equal except for values on a rounding boundary (one code apart); the
@@ -42,6 +43,7 @@ def _umma_pack(scales: np.ndarray) -> np.ndarray:
     (3, 256, 256, [5, 0, 300]),
     (4, 512, 1024, [129, 128, 1, 77]),
     (2, 768, 384, [256, 255]),
+    (5, 256, 512, [16, 17, 112, 113, 127]),
 ])
 def test_grouped_gemm_exact_small_integers(moe, G, N, K, counts):
     import torch
@@ -70,8 +72,6 @@ def test_grouped_gemm_exact_small_integers(moe, G, N, K, counts):
         rows = slice(r0, r0 + counts[g])
         ref = A[rows] @ B[g * N:(g + 1) * N].T
         assert np.array_equal(D[rows].astype(np.float64), ref), f"group {g}"
-        # rows beyond the group's count are not written
-        assert not D[r0 + counts[g]: mt[g + 1] * 128].any()
 
 
 def _weights(case, device="cuda"):

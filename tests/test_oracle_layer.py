@@ -223,3 +223,33 @@ def test_bf16_round_matches_torch_on_fp32_values():
     v = np.concatenate([rng.normal(0, 10, 5000), rng.normal(0, 1e-30, 100)]).astype(np.float32)
     ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
     assert np.array_equal(L.bf16_round(v.astype(np.float64)), ref)
+
+
+def test_weight_gradient_sensitivity(monkeypatch):
+    """The oracle against itself with 1e-6 relative noise on its bf16 roundings (what fp32
+    vs fp64 arithmetic does to dg, du, w*dOut and the saved g, u): requantisation flips move
+    rare weight-gradient elements beyond 3e-2*RMS, which is why the GPU comparison bounds
+    their number (<= 1e-4) and size (<= 0.25*RMS) instead of requiring none; dX keeps the
+    strict bound."""
+    case = synth.MoeCase("bh", 200, 512, 256, 32, 4, 1, "hot4cold16", seed=8)
+    x, lg, wfn = _inputs(case)
+    dout = synth.make_dout(case)
+    ref = L.backward(x, lg, dout, case.k, 1, case.E, wfn)
+    rng = np.random.default_rng(0)
+    plain = L.bf16_round
+    monkeypatch.setattr(L, "_bf", lambda v, exact: np.asarray(v, np.float64) if exact else
+                        plain(np.asarray(v) * (1 + rng.normal(0, 1e-6, np.shape(v)))))
+    got = L.backward(x, lg, dout, case.k, 1, case.E, wfn)
+    n_el = n_out = 0
+    for e, mats in ref["dW"].items():
+        for a, b in zip(got["dW"][e], mats):
+            if not b.any():
+                continue
+            assert np.linalg.norm(a - b) / np.linalg.norm(b) < 2e-3
+            dev = np.abs(a - b) / np.sqrt(np.mean(b ** 2))
+            n_el += dev.size
+            n_out += int(np.sum(dev > 3e-2))
+            assert dev.max() <= 0.25
+    assert 0 < n_out <= 1e-4 * n_el            # flips happen, and they are rare
+    r = np.sqrt(np.mean(ref["dx"] ** 2))
+    assert np.max(np.abs(got["dx"] - ref["dx"])) <= 3e-2 * r

@@ -85,6 +85,24 @@ moe_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t col
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Output map for the TMA-store epilogues: [rows, cols] of fp32 or bf16, box of 128 bytes
+// (32 fp32 or 64 bf16 columns) x 32 rows, 128-byte swizzle.
+moe_status make_out_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
+                         bool bf16) {
+  auto fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  const int64_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * esz)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 inline moe_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // ---------------------------------------------------------------------------------------
@@ -478,7 +496,9 @@ moe_status moe_grouped_gemm_mx(int32_t G, int64_t rows_a, int32_t N, int32_t K,
   P.out_f32 = d_out;
   P.ld_out = N;
   P.status = at<int32_t>(ws, 0);
-  return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32, ta, tb, P, sms,
+  CUtensorMap tc;
+  MOE_TRY(make_out_tmap(&tc, d_out, rows_a, N, false));
+  return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tc, tc, P, sms,
                                      static_cast<cudaStream_t>(stream)));
 }
 
@@ -567,7 +587,7 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.hs = hs;
     P.gu = gu;
     P.status = status;
-    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_SWIGLU, ta, tb, P, sms, st)));
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_SWIGLU, ta, tb, ta, tb, P, sms, st)));
   }
   {
     StageScope sc(MOE_STAGE_DOWN, st);
@@ -585,7 +605,9 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.out_f32 = y;
     P.ld_out = D->d;
     P.status = status;
-    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32, ta, tb, P, sms, st)));
+    CUtensorMap ty;
+    MOE_TRY(make_out_tmap(&ty, y, R, D->d, false));
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, ty, ty, P, sms, st)));
   }
   {
     StageScope sc(MOE_STAGE_COMBINE, st);
@@ -685,7 +707,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.dgu_q = dgu_q;
       P.dgu_s = dgu_s;
       P.status = status;
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_DGRAD_SWIGLU, ta, tb, P, sms, st)));
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_DGRAD_SWIGLU, ta, tb, ta, tb, P, sms, st)));
     }
     {  // dXa = [dg|du]^ . [Wg|Wu]'^T
       StageScope sc(MOE_STAGE_BWD_DGRAD_GATEUP, st);
@@ -704,7 +726,9 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.out_f32 = dxa;
       P.ld_out = d;
       P.status = status;
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32, ta, tb, P, sms, st)));
+      CUtensorMap tx;
+      MOE_TRY(make_out_tmap(&tx, dxa, R, d, false));
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tx, tx, P, sms, st)));
     }
     {  // push reverse-dispatch: dX[t] = sum_j dXa[row of (t, j)]
       StageScope sc(MOE_STAGE_BWD_DX, st);
@@ -796,7 +820,10 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     P.out_b = dWu;
     P.split = f;
     P.status = status;
-    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, P, sms, st)));
+    CUtensorMap tg, tu;
+    MOE_TRY(make_out_tmap(&tg, dWg, static_cast<int64_t>(E) * d, f, true));
+    MOE_TRY(make_out_tmap(&tu, dWu, static_cast<int64_t>(E) * d, f, true));
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, tg, tu, P, sms, st)));
     MOE_TRY(make_tmap(&ta, ht_q, f, Kt, 128));
     MOE_TRY(make_tmap(&tb, yt_q, d, Kt, 256));
     P.M = f;
@@ -806,7 +833,9 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     P.out_a = dWd;
     P.out_b = nullptr;
     P.split = d;
-    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, P, sms, st)));
+    CUtensorMap tdw;
+    MOE_TRY(make_out_tmap(&tdw, dWd, static_cast<int64_t>(E) * f, d, true));
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, tdw, tdw, P, sms, st)));
   }
   return MOE_OK;
 }

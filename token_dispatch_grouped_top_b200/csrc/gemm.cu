@@ -36,7 +36,7 @@
 
 namespace moe {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 128;
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
@@ -46,13 +46,27 @@ constexpr uint32_t kABytes = BM * BK, kBBytes = BN * BK;
 constexpr uint32_t kTxBytes = kABytes + kBBytes + 512 + 1024;
 constexpr int kMaxG = 1024;
 
-struct GemmSmem {
-  uint8_t a[STAGES][kABytes];
-  uint8_t b[STAGES][kBBytes];
-  uint8_t sfa[STAGES][512];
-  uint8_t sfb[STAGES][1024];
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+// Modes that store their output with TMA need staging space: 3 pipeline stages instead of 4.
+template <int MODE>
+struct ModeCfg {
+  static constexpr bool kTmaStore = MODE == GEMM_STORE_F32_TMA || MODE == GEMM_WGRAD_BF16;
+  static constexpr int kStages = kTmaStore ? 3 : 4;
+  static constexpr int kStageBufs = kTmaStore ? 2 : 0;  // per epilogue warp, 4 KB each
+  // A tile with fewer than 128 valid rows (an expert's last tile) runs with the operands
+  // swapped: the two 128-row halves of the B tile are the M side of two MMAs and the
+  // valid A rows, rounded up to 16, the N side -- the tensor work shrinks with the rows.
+  static constexpr bool kSwapTail = MODE == GEMM_GATEUP_SWIGLU || MODE == GEMM_STORE_F32_TMA;
+};
+
+template <int ST, int NSTG>
+struct GemmSmemT {
+  uint8_t a[ST][kABytes];
+  uint8_t b[ST][kBBytes];
+  uint8_t stg[NSTG ? kEpiWarps * NSTG : 1][4096];  // 32 rows x 128 bytes, 128-byte swizzle
+  uint8_t sfa[ST][512];
+  uint8_t sfb[ST][1024];
+  uint64_t full[ST];
+  uint64_t empty[ST];
   uint64_t tmem_full;
   uint64_t tmem_empty;
   uint32_t tmem_base;
@@ -60,17 +74,24 @@ struct GemmSmem {
   int prefix[kMaxG + 1];
   int valid[kMaxG];
 };
-constexpr size_t kGemmSmemBytes = sizeof(GemmSmem) + 1024;
+template <int MODE>
+using SmemOf = GemmSmemT<ModeCfg<MODE>::kStages, ModeCfg<MODE>::kStageBufs>;
+template <int MODE>
+constexpr size_t smem_bytes() { return sizeof(SmemOf<MODE>) + 1024; }
+static_assert(smem_bytes<GEMM_STORE_F32_TMA>() <= 232448, "shared memory budget (227 KB)");
+static_assert(smem_bytes<GEMM_GATEUP_SWIGLU>() <= 232448, "shared memory budget (227 KB)");
 
 struct TileInfo {
   int g, i, j;
   int kb0, nk;  // first K block and number of K blocks
+  int rows;     // valid A rows in this tile (variable-M modes), 1..128
   int64_t a_row0, b_row0;
 };
 
 // Variable-M groups (forward, dgrad): group g owns 128-row tiles [prefix[g], prefix[g+1]).
-__device__ __forceinline__ TileInfo decode_tile_var_m(int tile, const int* prefix, int G, int NT,
-                                                      int N, int nk) {
+__device__ __forceinline__ TileInfo decode_tile_var_m(int tile, const int* prefix,
+                                                      const int* valid, int G, int NT, int N,
+                                                      int nk) {
   int lo = 0, hi = G;  // prefix[lo]*NT <= tile < prefix[hi]*NT
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -84,6 +105,8 @@ __device__ __forceinline__ TileInfo decode_tile_var_m(int tile, const int* prefi
   t.i = local - t.j * mt;
   t.kb0 = 0;
   t.nk = nk;
+  const int left = valid[lo] - t.i * BM;
+  t.rows = left < BM ? left : BM;
   t.a_row0 = static_cast<int64_t>(prefix[lo] + t.i) * BM;
   t.b_row0 = static_cast<int64_t>(lo) * N + static_cast<int64_t>(t.j) * BN;
   return t;
@@ -99,15 +122,17 @@ __device__ __forceinline__ TileInfo decode_tile_var_k(int tile, const int* prefi
   t.j = local - t.i * NT;
   t.kb0 = prefix[t.g];
   t.nk = prefix[t.g + 1] - prefix[t.g];
+  t.rows = BM;
   t.a_row0 = static_cast<int64_t>(t.i) * BM;
   t.b_row0 = static_cast<int64_t>(t.j) * BN;
   return t;
 }
 
 template <int MODE>
-__device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const GemmParams& P) {
+__device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const int* valid,
+                                                const GemmParams& P) {
   if (MODE == GEMM_WGRAD_BF16) return decode_tile_var_k(tile, prefix, P.M / BM, P.N / BN);
-  return decode_tile_var_m(tile, prefix, P.G, P.N / BN, P.N, P.K / BK);
+  return decode_tile_var_m(tile, prefix, valid, P.G, P.N / BN, P.N, P.K / BK);
 }
 
 // E4M3 byte -> fp32, exact (normal: (1 + m/8) 2^(e-7); subnormal: m 2^-9).
@@ -128,6 +153,41 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
                     f32_to_bf16_bits(v[2]) | (f32_to_bf16_bits(v[3]) << 16),
                     f32_to_bf16_bits(v[4]) | (f32_to_bf16_bits(v[5]) << 16),
                     f32_to_bf16_bits(v[6]) | (f32_to_bf16_bits(v[7]) << 16));
+}
+
+// Swapped gate/up tail epilogue for 32 tokens [tb, tb+32) of one warp: lane = feature
+// (gate in g[], up in u[], column = token).  h = silu(g) * u is quantised along the
+// features, i.e. across the 32 lanes of the warp (one MX block per token).
+__device__ __forceinline__ void swapped_gateup_epilogue(const GemmParams& P, const TileInfo& ti,
+                                                        int q, int lane, int tb,
+                                                        const float (&g)[32],
+                                                        const float (&u)[32]) {
+  if (tb >= ti.rows) return;  // warp-uniform
+  const int f = P.f;
+  const int fi = (BN / 2) * ti.j + 32 * q + lane;  // this lane's feature
+  uint32_t my_sb = 0;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const float hv = g[c] / (1.f + expf(-g[c])) * u[c];
+    float amax = fabsf(hv);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+    const int s = mx_scale_exp(amax);
+    const uint32_t code = cvt_e4m3x2(hv * mx_inv_scale(s), 0.f) & 0xFFu;
+    if (c == lane) my_sb = static_cast<uint32_t>(s + 127);
+    if (tb + c < ti.rows) {
+      const int64_t row = ti.a_row0 + tb + c;
+      P.hq[row * f + fi] = static_cast<uint8_t>(code);
+      if (P.gu) {
+        P.gu[row * 2 * f + fi] = static_cast<uint16_t>(f32_to_bf16_bits(g[c]));
+        P.gu[row * 2 * f + f + fi] = static_cast<uint16_t>(f32_to_bf16_bits(u[c]));
+      }
+    }
+  }
+  if (tb + lane < ti.rows) {
+    const int64_t row = ti.a_row0 + tb + lane;
+    P.hs[umma_scale_offset(row, fi >> 5, f >> 7)] = static_cast<uint8_t>(my_sb);
+  }
 }
 
 // DGRAD epilogue for 32 features [fc, fc+32) of one row: returns this chunk's part of
@@ -197,10 +257,34 @@ __device__ __forceinline__ float dgrad_chunk(const GemmParams& P, const float (&
   return dwp;
 }
 
+// Stage one 32-row x 128-byte chunk (row = lane) in shared memory with the 128-byte swizzle
+// the output tensor map uses, then one lane stores it with TMA.  Two buffers per warp:
+// before a buffer is rewritten, the store issued from it two chunks ago must have read it.
+__device__ __forceinline__ void stage_and_store(uint8_t* buf, const uint4 (&row16)[8],
+                                                const CUtensorMap* tmap, int32_t x, int32_t y,
+                                                int lane) {
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+  uint8_t* r = buf + lane * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(r + ((j ^ (lane & 7)) << 4)) = row16[j];
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmap, smem_u32(buf), x, y);
+    bulk_commit();
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmParams P) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmC0,
+                        const __grid_constant__ CUtensorMap tmC1, const GemmParams P) {
+  constexpr int STAGES = ModeCfg<MODE>::kStages;
+  using GemmSmem = SmemOf<MODE>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u));
@@ -241,7 +325,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const TileInfo ti = decode_tile<MODE>(tile, S.prefix, P);
+        const TileInfo ti = decode_tile<MODE>(tile, S.prefix, S.valid, P);
         const int64_t rbA = ti.a_row0 >> 7, rbB = ti.b_row0 >> 7;
         for (int kb = ti.kb0; kb < ti.kb0 + ti.nk; ++kb) {
           if (!mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, abort_flag, P.status)) break;
@@ -267,8 +351,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       const uint32_t idesc = idesc_mxf8_e4m3(BM, BN);
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const int nk = decode_tile<MODE>(tile, S.prefix, P).nk;
+        const TileInfo tinfo = decode_tile<MODE>(tile, S.prefix, S.valid, P);
+        const int nk = tinfo.nk;
         if (nk == 0) continue;  // empty expert (wgrad): the epilogue writes zeros
+        const bool swapped = ModeCfg<MODE>::kSwapTail && tinfo.rows < BM;
+        const uint32_t idesc_sw = idesc_mxf8_e4m3(BM, (tinfo.rows + 15) & ~15);
         if (!mbar_wait(smem_u32(&S.tmem_empty), acc_phase ^ 1u, abort_flag, P.status)) break;
         tc_fence_after();
         bool ok = true;
@@ -283,12 +370,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_cp_scales(sf + 4, sdesc_scale_chunk(smem_u32(S.sfb[stage])));
           tmem_cp_scales(sf + 8, sdesc_scale_chunk(smem_u32(S.sfb[stage]) + 512));
           const uint32_t a0 = smem_u32(S.a[stage]), b0 = smem_u32(S.b[stage]);
+          if (swapped) {
+            // D0[w, t] = sum_k B[w, k] A[t, k] for weight rows w < 128, D1 for rows 128..255
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk) {
-            const uint32_t id = idesc | (static_cast<uint32_t>(kk) << 29) |
-                                (static_cast<uint32_t>(kk) << 4);
-            mma_mxf8(tbase + kAccCol, sdesc_k_sw128(a0 + 32u * kk), sdesc_k_sw128(b0 + 32u * kk),
-                     id, (kb | kk) != 0 ? 1u : 0u, sf, sf + 4);
+            for (int kk = 0; kk < BK / 32; ++kk) {
+              const uint32_t id = idesc_sw | (static_cast<uint32_t>(kk) << 29) |
+                                  (static_cast<uint32_t>(kk) << 4);
+              const uint64_t bt = sdesc_k_sw128(a0 + 32u * kk);
+              mma_mxf8(tbase + kAccCol, sdesc_k_sw128(b0 + 32u * kk), bt, id,
+                       (kb | kk) != 0 ? 1u : 0u, sf + 4, sf);
+              mma_mxf8(tbase + kAccCol + 128, sdesc_k_sw128(b0 + 128u * 128u + 32u * kk), bt, id,
+                       (kb | kk) != 0 ? 1u : 0u, sf + 8, sf);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk) {
+              const uint32_t id = idesc | (static_cast<uint32_t>(kk) << 29) |
+                                  (static_cast<uint32_t>(kk) << 4);
+              mma_mxf8(tbase + kAccCol, sdesc_k_sw128(a0 + 32u * kk),
+                       sdesc_k_sw128(b0 + 32u * kk), id, (kb | kk) != 0 ? 1u : 0u, sf, sf + 4);
+            }
           }
           mma_commit(smem_u32(&S.empty[stage]));
           if (++stage == STAGES) {
@@ -306,8 +407,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int h = (warp - 2) >> 2;   // column half
     uint32_t acc_phase = 0;
+    int stg_buf = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileInfo ti = decode_tile<MODE>(tile, S.prefix, P);
+      const TileInfo ti = decode_tile<MODE>(tile, S.prefix, S.valid, P);
       if (MODE == GEMM_WGRAD_BF16 && ti.nk == 0) {
         const int64_t m = ti.a_row0 + 32 * q + lane;
         const int n0 = ti.j * BN + 128 * h;
@@ -323,6 +425,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait(smem_u32(&S.tmem_full), acc_phase, abort_flag, P.status)) break;
       tc_fence_after();
       const uint32_t taddr = tbase + kAccCol + (static_cast<uint32_t>(32 * q) << 16);
+      if (ModeCfg<MODE>::kSwapTail && ti.rows < BM) {
+        // transposed accumulators: lane = weight row (feature), column = token
+        const int tok0 = 64 * h;
+        float d0a[32], d0b[32], d1a[32], d1b[32];
+        tmem_ld32(taddr + tok0, d0a);
+        tmem_ld32(taddr + tok0 + 32, d0b);
+        tmem_ld32(taddr + 128 + tok0, d1a);
+        tmem_ld32(taddr + 128 + tok0 + 32, d1b);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S.tmem_empty));
+        acc_phase ^= 1u;
+        if (MODE == GEMM_GATEUP_SWIGLU) {
+          swapped_gateup_epilogue(P, ti, q, lane, tok0, d0a, d1a);
+          swapped_gateup_epilogue(P, ti, q, lane, tok0 + 32, d0b, d1b);
+        } else if (MODE == GEMM_STORE_F32_TMA) {
+          const int32_t y0 = static_cast<int32_t>(ti.a_row0);
+          const int32_t x0 = ti.j * BN + 32 * q;
+          const float* parts[4] = {d0a, d0b, d1a, d1b};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int tb = tok0 + 32 * (c & 1);
+            if (tb >= ti.rows) continue;  // warp-uniform
+            const float* v = c == 0 ? d0a : c == 1 ? d0b : c == 2 ? d1a : d1b;
+            uint8_t* buf = S.stg[2 * (warp - 2) + stg_buf];
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < 32; ++r)  // token r of the chunk, feature = lane
+              *reinterpret_cast<float*>(buf + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) +
+                                        ((lane & 3) << 2)) = v[r];
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmC0, smem_u32(buf), x0 + 128 * (c >> 1), y0 + tb);
+              bulk_commit();
+            }
+            stg_buf ^= 1;
+          }
+          (void)parts;
+        }
+        continue;
+      }
       float v0[32], v1[32], v2[32], v3[32];
       if (MODE == GEMM_GATEUP_SWIGLU) {
         tmem_ld32(taddr + 64 * h, v0);         // gate features 64h .. 64h+31
@@ -343,20 +489,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
       const int m = 32 * q + lane;
       if (MODE == GEMM_WGRAD_BF16) {
-        const int64_t row = ti.a_row0 + m;
+        // bf16 rows of 128 columns: two 64-column chunks through the staging buffers
         const int n0 = ti.j * BN + 128 * h;
         const bool first = n0 < P.split;
-        const int ld = first ? P.split : P.N - P.split;
-        uint16_t* base = (first ? P.out_a : P.out_b) +
-                         (static_cast<int64_t>(ti.g) * P.M + row) * ld +
-                         (first ? n0 : n0 - P.split);
-        uint4* dst = reinterpret_cast<uint4*>(base);
+        const CUtensorMap* tm = first ? &tmC0 : &tmC1;
+        const int x0 = first ? n0 : n0 - P.split;
+        const int32_t y = static_cast<int32_t>(ti.g * P.M + ti.a_row0 + 32 * q);
+        uint4 r16[8];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          dst[c] = pack_bf16x8(v0 + 8 * c);
-          dst[4 + c] = pack_bf16x8(v1 + 8 * c);
-          dst[8 + c] = pack_bf16x8(v2 + 8 * c);
-          dst[12 + c] = pack_bf16x8(v3 + 8 * c);
+          r16[c] = pack_bf16x8(v0 + 8 * c);
+          r16[4 + c] = pack_bf16x8(v1 + 8 * c);
+        }
+        stage_and_store(S.stg[2 * (warp - 2) + stg_buf], r16, tm, x0, y, lane);
+        stg_buf ^= 1;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          r16[c] = pack_bf16x8(v2 + 8 * c);
+          r16[4 + c] = pack_bf16x8(v3 + 8 * c);
+        }
+        stage_and_store(S.stg[2 * (warp - 2) + stg_buf], r16, tm, x0 + 64, y, lane);
+        stg_buf ^= 1;
+        continue;
+      }
+      if (MODE == GEMM_STORE_F32_TMA) {
+        // fp32 rows of 128 columns: four 32-column chunks; whole 32-row boxes are written
+        const int32_t x0 = ti.j * BN + 128 * h;
+        const int32_t y = static_cast<int32_t>(ti.a_row0 + 32 * q);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float* vc = c == 0 ? v0 : c == 1 ? v1 : c == 2 ? v2 : v3;
+          uint4 r16[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            r16[j] = make_uint4(__float_as_uint(vc[4 * j]), __float_as_uint(vc[4 * j + 1]),
+                                __float_as_uint(vc[4 * j + 2]), __float_as_uint(vc[4 * j + 3]));
+          stage_and_store(S.stg[2 * (warp - 2) + stg_buf], r16, &tmC0, x0 + 32 * c, y, lane);
+          stg_buf ^= 1;
         }
         continue;
       }
@@ -424,6 +593,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  if (ModeCfg<MODE>::kTmaStore && warp >= 2 && lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -434,33 +604,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 template <int MODE>
-static cudaError_t launch_mode(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& P,
-                               int num_sms, cudaStream_t stream) {
+static cudaError_t launch_mode(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                               const CUtensorMap& tmC0, const CUtensorMap& tmC1,
+                               const GemmParams& P, int num_sms, cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kGemmSmemBytes));
+                                         static_cast<int>(smem_bytes<MODE>()));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  grouped_gemm_kernel<MODE><<<num_sms, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, P);
+  grouped_gemm_kernel<MODE><<<num_sms, kGemmThreads, smem_bytes<MODE>(), stream>>>(tmA, tmB, tmC0,
+                                                                                  tmC1, P);
   return cudaGetLastError();
 }
 
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const CUtensorMap& tmC0, const CUtensorMap& tmC1,
                                 const GemmParams& P, int num_sms, cudaStream_t stream) {
   switch (mode) {
     case GEMM_STORE_F32:
-      return launch_mode<GEMM_STORE_F32>(tmA, tmB, P, num_sms, stream);
+      return launch_mode<GEMM_STORE_F32>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_GATEUP_SWIGLU:
-      return launch_mode<GEMM_GATEUP_SWIGLU>(tmA, tmB, P, num_sms, stream);
+      return launch_mode<GEMM_GATEUP_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_DGRAD_SWIGLU:
-      return launch_mode<GEMM_DGRAD_SWIGLU>(tmA, tmB, P, num_sms, stream);
+      return launch_mode<GEMM_DGRAD_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_WGRAD_BF16:
-      return launch_mode<GEMM_WGRAD_BF16>(tmA, tmB, P, num_sms, stream);
+      return launch_mode<GEMM_WGRAD_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
+    case GEMM_STORE_F32_TMA:
+      return launch_mode<GEMM_STORE_F32_TMA>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

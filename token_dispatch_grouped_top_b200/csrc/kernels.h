@@ -127,6 +127,8 @@ enum GemmMode : int {
   GEMM_GATEUP_SWIGLU = 1,  // SwiGLU + MX requant of h, optional bf16 g/u save
   GEMM_DGRAD_SWIGLU = 2,   // G = dOut . Wd^T -> dw_route, SwiGLU backward, dg/du bf16 + MX
   GEMM_WGRAD_BF16 = 3,     // variable K per group (the group's token segment), bf16 out
+  GEMM_STORE_F32_TMA = 4,  // as STORE_F32 through shared memory + TMA stores; writes whole
+                           // 128-row tiles (rows past a group's count get unused values)
 };
 
 struct GemmParams {
@@ -161,7 +163,10 @@ struct GemmParams {
   int split;
   int32_t* status;
 };
+// tmC0 / tmC1: output tensor maps of the TMA-store modes (STORE_F32_TMA: fp32 [rows, N],
+// box 32 x 32; WGRAD: bf16 out_a / out_b, box 64 cols x 32 rows); ignored otherwise.
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const CUtensorMap& tmC0, const CUtensorMap& tmC1,
                                 const GemmParams& P, int num_sms, cudaStream_t stream);
 
 }  // namespace moe

@@ -35,43 +35,62 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 }
 
 // One warp quantises K bf16 values of one row (K % 32 == 0).  Lane l handles 8 values per
-// 256-column step; four lanes share a 32-element block.  Scales go to the canonical
-// layout (row stride K/32, first block kb0) or to the UMMA layout (kgroups = K_total/128;
-// kb0 % 4 == 0 required).
+// 256-column step; four lanes share a 32-element block.  kUnroll steps are loaded before
+// any of them is converted, so each lane keeps several 16-byte loads in flight.  Scales go
+// to the canonical layout (row stride K/32, first block kb0) or to the UMMA layout
+// (kgroups = K_total/128; kb0 % 4 == 0 required).
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ void quant_step(const uint4& raw, bool in, int64_t col,
+                                           uint8_t* __restrict__ dst,
+                                           uint8_t* __restrict__ scales, int64_t row, int64_t kb0,
+                                           int layout, int64_t canon_stride, int64_t kgroups,
+                                           int lane) {
+  float v[8];
+  unpack_bf16x8(raw, v);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+  const int s = mx_scale_exp(amax);
+  const float inv = mx_inv_scale(s);
+  uint2 packed;
+  packed.x = pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+  packed.y = pack_e4m3x4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
+  if (in) *reinterpret_cast<uint2*>(dst + col) = packed;
+  const uint32_t sb = static_cast<uint32_t>(s + 127);
+  const int64_t kb = kb0 + (col >> 5);
+  if (layout == 0) {
+    if (in && (lane & 3) == 0) scales[row * canon_stride + kb] = static_cast<uint8_t>(sb);
+  } else {
+    const uint32_t b1 = __shfl_down_sync(kFull, sb, 4);
+    const uint32_t b2 = __shfl_down_sync(kFull, sb, 8);
+    const uint32_t b3 = __shfl_down_sync(kFull, sb, 12);
+    if (in && (lane & 15) == 0)
+      *reinterpret_cast<uint32_t*>(scales + umma_scale_offset(row, kb, kgroups)) =
+          sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+  }
+}
+
 __device__ __forceinline__ void warp_quant_row(const uint16_t* __restrict__ src, int64_t K,
                                                uint8_t* __restrict__ dst,
                                                uint8_t* __restrict__ scales, int64_t row,
                                                int64_t kb0, int layout, int64_t canon_stride,
                                                int64_t kgroups, int lane) {
-  for (int64_t c0 = 0; c0 < K; c0 += 256) {
-    const int64_t col = c0 + lane * 8;
-    const bool in = col < K;
-    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-    if (in) raw = ld_nc_v4(src + col);
-    float v[8];
-    unpack_bf16x8(raw, v);
-    float amax = 0.f;
+  for (int64_t c0 = 0; c0 < K; c0 += 256 * kUnroll) {
+    uint4 raw[kUnroll];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-    const int s = mx_scale_exp(amax);
-    const float inv = mx_inv_scale(s);
-    uint2 packed;
-    packed.x = pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
-    packed.y = pack_e4m3x4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
-    if (in) *reinterpret_cast<uint2*>(dst + col) = packed;
-    const uint32_t sb = static_cast<uint32_t>(s + 127);
-    const int64_t kb = kb0 + (col >> 5);
-    if (layout == 0) {
-      if (in && (lane & 3) == 0) scales[row * canon_stride + kb] = static_cast<uint8_t>(sb);
-    } else {
-      const uint32_t b1 = __shfl_down_sync(kFull, sb, 4);
-      const uint32_t b2 = __shfl_down_sync(kFull, sb, 8);
-      const uint32_t b3 = __shfl_down_sync(kFull, sb, 12);
-      if (in && (lane & 15) == 0)
-        *reinterpret_cast<uint32_t*>(scales + umma_scale_offset(row, kb, kgroups)) =
-            sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t col = c0 + 256 * u + lane * 8;
+      raw[u] = col < K ? ld_nc_v4(src + col) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t col = c0 + 256 * u + lane * 8;
+      if (c0 + 256 * u < K)  // warp-uniform: whole 256-column step inside or outside
+        quant_step(raw[u], col < K, col, dst, scales, row, kb0, layout, canon_stride, kgroups,
+                   lane);
     }
   }
 }
@@ -210,23 +229,32 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
       if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
       continue;
     }
-    for (int64_t c0 = 0; c0 < P.d; c0 += 128) {
-      const int64_t col = c0 + lane * 4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t c0 = 0; c0 < P.d; c0 += 256) {
+      const int64_t col0 = c0 + lane * 4, col1 = col0 + 128;  // d % 256 == 0
+      float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
 #pragma unroll 4
       for (int j = 0; j < k; ++j) {
         const int64_t row = __shfl_sync(kFull, my_row, j);
         const float w = __shfl_sync(kFull, my_w, j);
-        const float4 yv = __ldg(reinterpret_cast<const float4*>(P.y + row * P.d + col));
-        acc.x += w * yv.x;
-        acc.y += w * yv.y;
-        acc.z += w * yv.z;
-        acc.w += w * yv.w;
+        const float* yr = P.y + row * P.d;
+        const float4 y0 = __ldg(reinterpret_cast<const float4*>(yr + col0));
+        const float4 y1 = __ldg(reinterpret_cast<const float4*>(yr + col1));
+        acc0.x += w * y0.x;
+        acc0.y += w * y0.y;
+        acc0.z += w * y0.z;
+        acc0.w += w * y0.w;
+        acc1.x += w * y1.x;
+        acc1.y += w * y1.y;
+        acc1.z += w * y1.z;
+        acc1.w += w * y1.w;
       }
-      uint2 o;
-      o.x = f32_to_bf16_bits(acc.x) | (f32_to_bf16_bits(acc.y) << 16);
-      o.y = f32_to_bf16_bits(acc.z) | (f32_to_bf16_bits(acc.w) << 16);
-      *reinterpret_cast<uint2*>(P.out + t * P.d + col) = o;
+      uint2 o0, o1;
+      o0.x = f32_to_bf16_bits(acc0.x) | (f32_to_bf16_bits(acc0.y) << 16);
+      o0.y = f32_to_bf16_bits(acc0.z) | (f32_to_bf16_bits(acc0.w) << 16);
+      o1.x = f32_to_bf16_bits(acc1.x) | (f32_to_bf16_bits(acc1.y) << 16);
+      o1.y = f32_to_bf16_bits(acc1.z) | (f32_to_bf16_bits(acc1.w) << 16);
+      *reinterpret_cast<uint2*>(P.out + t * P.d + col0) = o0;
+      *reinterpret_cast<uint2*>(P.out + t * P.d + col1) = o1;
     }
   }
 }

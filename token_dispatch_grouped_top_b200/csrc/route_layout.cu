@@ -11,8 +11,9 @@
 //                       experts with deterministic in-tile ranks (ballot masks, no
 //                       order-dependent atomics), and a decoupled-lookback scan of the
 //                       per-tile expert-count vectors that gives every tile its starting
-//                       rank inside each expert.  The tile that finishes last turns the
-//                       totals into counts, offsets and the padded tile prefix.
+//                       rank inside each expert (32 predecessors inspected per step).
+//                       The tile that finishes last turns the totals into counts,
+//                       offsets and the padded tile prefix.
 //   scatter_kernel      pos = offsets[e] + rank; perm[pos] = a; inv[a] = pos.
 // The result is the stable counting sort: inside an expert, ascending token.
 #include <math.h>
@@ -60,61 +61,85 @@ __global__ void __launch_bounds__(kRouteThreads) route_rank_kernel(RouteParams P
   const int b = s_bid;
   const int64_t t0 = static_cast<int64_t>(b) * kRouteTile;
 
-  // ---- 1. top-k per token -----------------------------------------------------------
-  for (int tl = warp; tl < kRouteTile; tl += kRouteThreads / 32) {
-    const int64_t t = t0 + tl;
-    if (t >= P.T) break;
-    const float* row = P.logits + t * E;
-    float v[NPL];
-    uint32_t removed = 0;
+  // ---- 1. top-k per token: each warp selects for kTPW tokens at once (independent
+  //         shuffle chains interleave), k rounds of a warp-wide (value, -index) argmax ----
+  constexpr int kTPW = 4;
+  for (int tl0 = warp * kTPW; tl0 < kRouteTile; tl0 += (kRouteThreads / 32) * kTPW) {
+    float v[kTPW][NPL];
+    uint32_t removed[kTPW];
+    float sel_v[kTPW];
+    int sel_e[kTPW];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      v[i] = (e < E) ? row[e] : -INFINITY;
-      if (e >= E) removed |= 1u << i;
-    }
-    float sel_v = 0.f;
-    int sel_e = 0;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+    for (int u = 0; u < kTPW; ++u) {
+      const int64_t t = t0 + tl0 + u;
+      const bool tv = t < P.T;
+      const float* row = P.logits + (tv ? t : 0) * E;
+      removed[u] = 0;
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        if (!((removed >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
-          bv = v[i];
-          be = e;
+        v[u][i] = (tv && e < E) ? row[e] : -INFINITY;
+        if (e >= E) removed[u] |= 1u << i;
+      }
+      sel_v[u] = 0.f;
+      sel_e[u] = 0;
+    }
+    for (int j = 0; j < k; ++j) {
+      float bv[kTPW];
+      int be[kTPW];
+#pragma unroll
+      for (int u = 0; u < kTPW; ++u) {
+        bv[u] = -INFINITY;
+        be[u] = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+          const int e = lane + 32 * i;
+          if (!((removed[u] >> i) & 1u) && (v[u][i] > bv[u] || (v[u][i] == bv[u] && e < be[u]))) {
+            bv[u] = v[u][i];
+            be[u] = e;
+          }
         }
       }
 #pragma unroll
       for (int off = 16; off; off >>= 1) {
-        const float ov = __shfl_xor_sync(kFull, bv, off);
-        const int oe = __shfl_xor_sync(kFull, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
+#pragma unroll
+        for (int u = 0; u < kTPW; ++u) {
+          const float ov = __shfl_xor_sync(kFull, bv[u], off);
+          const int oe = __shfl_xor_sync(kFull, be[u], off);
+          if (ov > bv[u] || (ov == bv[u] && oe < be[u])) {
+            bv[u] = ov;
+            be[u] = oe;
+          }
         }
       }
-      if ((be & 31) == lane) removed |= 1u << (be >> 5);
-      if (lane == j) {
-        sel_v = bv;
-        sel_e = be;
+#pragma unroll
+      for (int u = 0; u < kTPW; ++u) {
+        if ((be[u] & 31) == lane) removed[u] |= 1u << (be[u] >> 5);
+        if (lane == j) {
+          sel_v[u] = bv[u];
+          sel_e[u] = be[u];
+        }
       }
     }
-    float score;
-    if (P.score_fn == MOE_SCORE_SOFTMAX_TOPK) {
-      const float m = __shfl_sync(kFull, sel_v, 0);  // slot 0 holds the largest logit
-      score = (lane < k) ? expf(sel_v - m) : 0.f;
-    } else {
-      score = (lane < k) ? 1.f / (1.f + expf(-sel_v)) : 0.f;
-    }
-    float sum = score;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
-    if (lane < k) {
-      P.topk_idx[t * k + lane] = sel_e;
-      P.topk_w[t * k + lane] = score / sum;
-      s_idx[tl][lane] = sel_e;
+    for (int u = 0; u < kTPW; ++u) {
+      const int tl = tl0 + u;
+      const int64_t t = t0 + tl;
+      float score;
+      if (P.score_fn == MOE_SCORE_SOFTMAX_TOPK) {
+        const float m = __shfl_sync(kFull, sel_v[u], 0);  // slot 0 holds the largest logit
+        score = (lane < k) ? expf(sel_v[u] - m) : 0.f;
+      } else {
+        score = (lane < k) ? 1.f / (1.f + expf(-sel_v[u])) : 0.f;
+      }
+      float sum = score;
+#pragma unroll
+      for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+      if (t < P.T && lane < k) {
+        P.topk_idx[t * k + lane] = sel_e[u];
+        P.topk_w[t * k + lane] = score / sum;
+        s_idx[tl][lane] = sel_e[u];
+      }
     }
   }
   __syncthreads();
@@ -174,35 +199,52 @@ __global__ void __launch_bounds__(kRouteThreads) route_rank_kernel(RouteParams P
     __threadfence();
     __syncthreads();
     if (tid == 0) st_release(&P.flags[b], FLAG_AGG);
-    int pred = b - 1;
+    // Windowed lookback: warp 0 reads the flags of the next 32 predecessors at once; the
+    // block adds their aggregates down to (and including) the nearest inclusive prefix.
+    int hi = b - 1;  // highest predecessor not yet added
     bool failed = false;
-    while (true) {
-      if (tid == 0) {
-        uint32_t f = ld_acquire(&P.flags[pred]);
-        if (f == FLAG_NONE) {
-          const uint64_t start = globaltimer_ns();
-          while ((f = ld_acquire(&P.flags[pred])) == FLAG_NONE) {
-            if (globaltimer_ns() - start > kWaitLimitNs) break;
-            __nanosleep(64);
+    while (hi >= 0) {
+      if (warp == 0) {
+        const int p = hi - lane;
+        uint32_t f = FLAG_NONE;
+        if (p >= 0) {
+          f = ld_acquire(&P.flags[p]);
+          if (f == FLAG_NONE) {
+            const uint64_t start = globaltimer_ns();
+            while ((f = ld_acquire(&P.flags[p])) == FLAG_NONE) {
+              if (globaltimer_ns() - start > kWaitLimitNs) break;
+              __nanosleep(32);
+            }
           }
         }
-        s_flag = static_cast<int>(f);
+        const uint32_t pref = __ballot_sync(kFull, p >= 0 && f == FLAG_PREFIX);
+        const uint32_t present = __ballot_sync(kFull, p >= 0);
+        const uint32_t missing = __ballot_sync(kFull, p >= 0 && f == FLAG_NONE);
+        if (lane == 0) {
+          s_flag = missing ? -1 : (pref ? __ffs(pref) : -__popc(present) - 2);
+        }
       }
       __syncthreads();
-      const int f = s_flag;
-      if (f == FLAG_NONE) {  // bounded wait ran out: latch, publish garbage, carry on
+      const int code = s_flag;
+      if (code == -1) {  // a bounded wait ran out: latch, publish garbage, carry on
         failed = true;
         break;
       }
-      const int* src = (f == FLAG_PREFIX ? P.incl : P.agg) + pred * rowE;
+      const bool found = code > 0;
+      const int n = found ? code : -(code + 2);  // predecessors hi, hi-1, ..., hi-n+1
+#pragma unroll 4
+      for (int i = 0; i < n; ++i) {
+        const int pr = hi - i;
+        const int* src = (found && i == n - 1 ? P.incl : P.agg) + pr * rowE;
 #pragma unroll
-      for (int r = 0; r < kPer; ++r) {
-        const int e = tid + kRouteThreads * r;
-        if (e < E) excl[r] += __ldcg(src + e);
+        for (int r = 0; r < kPer; ++r) {
+          const int e = tid + kRouteThreads * r;
+          if (e < E) excl[r] += __ldcg(src + e);
+        }
       }
-      __syncthreads();  // s_flag is rewritten in the next round
-      if (f == FLAG_PREFIX) break;
-      --pred;
+      __syncthreads();  // s_flag is rewritten in the next window
+      if (found) break;
+      hi -= n;
     }
     if (failed && tid == 0) latch(P.status, MOE_ERR_DEVICE_TIMEOUT);
 #pragma unroll
