@@ -177,9 +177,11 @@ moe_status moe_backward(const moe_dims* dims, const moe_weights* w, const moe_sa
  * For each group g and each row r in [128*mtile_prefix[g], 128*mtile_prefix[g+1]):
  *   D[r, n] = sum_k A[r,k] * B[g*N + n, k],  n < N,  fp32 accumulation, fp32 output
  * with A [R,K] / B [G*N,K] MX (UMMA scales).  mtile_prefix [G+1] is device memory
- * (128-row tiles per group, prefix-summed); rows_valid [G] (nullable) limits the rows
- * written per group.  N % 256 == 0, K % 128 == 0, R = 128*mtile_prefix[G] at most
- * rows_a.  d_out [rows_a, N] fp32. */
+ * (128-row tiles per group, prefix-summed); rows_valid [G] (nullable) gives the valid
+ * rows of each group: a group's last tile then runs only as wide as its valid rows, and
+ * rows past rows_valid[g] inside the group's tiles receive unspecified values.
+ * N % 256 == 0, K % 128 == 0, R = 128*mtile_prefix[G] at most rows_a; d_out [rows_a, N]
+ * fp32, 16-byte aligned with N*4 a multiple of 16. */
 moe_status moe_grouped_gemm_mx(int32_t G, int64_t rows_a, int32_t N, int32_t K,
                                const int32_t* mtile_prefix, const int32_t* rows_valid,
                                const uint8_t* a_q, const uint8_t* a_s, const uint8_t* b_q,
