@@ -132,6 +132,28 @@ moe_status moe_route_layout(const moe_dims* dims, const float* logits, int32_t* 
                             int32_t* inv_perm, int32_t* pad_offsets, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* ---- routing and layout without a workspace ---------------------------------------
+ * No counterpart in the article: an addition for callers that cannot allocate device
+ * memory themselves (a plugin whose host framework owns every device allocation, an
+ * embedded runtime with a fixed memory budget, or a latency-critical path where
+ * cudaMalloc's implicit device synchronisation is not acceptable).  Same inputs, outputs
+ * and results as moe_route_layout, but the scratch lives in a fixed 8 MiB array inside
+ * the library (held by every GPU that loads the library until the process exits);
+ * nothing is allocated and no workspace is passed.
+ *  - Problems whose scratch exceeds 8 MiB return MOE_ERR_UNSUPPORTED_SHAPE before any
+ *    launch.  The scratch is 256 + 4*nt + 8*nt*E + 4*T*k + 4*(E+1) bytes (each term
+ *    rounded up to 256) with nt = ceil(T/64): e.g. E = 256, k = 8 fits T <= 130896.
+ *  - The first call on a device looks up the array's device address for that device
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call shares the one array: calls whose executions overlap on the GPU race on
+ *    it and give wrong results.  Each call clears the parts that must start at zero.
+ *  - status (nullable, device int32, zeroed by the caller): device-side errors are
+ *    latched there (first error wins) instead of in a workspace. */
+moe_status moe_route_layout_noalloc(const moe_dims* dims, const float* logits,
+                                    int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                    int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                                    int32_t* pad_offsets, int32_t* status, void* stream);
+
 /* ---- MXFP8 quantiser ------------------------------------------------------------------
  * Article §02 (MXFP8 activations fused into dispatch, grouped GEMM and SwiGLU); format:
  * OCP MX v1.0 (s = floor(log2 amax) - 8 clamped to [-127,127], E4M3 round-to-nearest-even

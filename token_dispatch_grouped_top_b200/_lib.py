@@ -48,6 +48,8 @@ SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [c_i32]),
     "moe_route_layout": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                  c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "moe_route_layout_noalloc": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp,
+                                         c_vp, c_vp, c_vp, c_vp, c_vp]),
     "mxfp8_quantize": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp]),
     "moe_prepare_weights": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_i32,
                                     ctypes.POINTER(MoeWeights), c_vp]),
