@@ -214,7 +214,7 @@ def run_reference(args, case):
 # kernels launched per stage (route: routing + scatter; transposes: 4; wgrad: 2 GEMMs)
 KERNELS_PER_STAGE = {"route": 2, "permute": 1, "gateup": 1, "down": 1, "combine": 1,
                      "bwd_dout": 1, "bwd_dgrad_down": 1, "bwd_dgrad_gateup": 1, "bwd_dx": 1,
-                     "bwd_transpose": 4, "bwd_wgrad": 2}
+                     "bwd_transpose": 4, "bwd_wgrad": 2, "bwd_swiglu": 1}
 
 
 def run_ours(args, case):
@@ -353,6 +353,8 @@ def run_ours(args, case):
         "combine": 4 * A * case.d + 2 * case.T * case.d,
         "bwd_dout": 2 * case.T * case.d + A * case.d * (1 + 1 / 32),
         "bwd_dx": 4 * A * case.d + 2 * case.T * case.d,
+        # G fp32 + saved g|u bf16 + h MX read, dg|du MX written, per assignment row
+        "bwd_swiglu": A * case.f * (4 + 4 + 1 + 2) * (1 + 1 / 64),
     }
     stage_info = {}
     for name, (tot_ms, n) in stages.items():

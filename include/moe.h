@@ -224,7 +224,8 @@ typedef enum {
   MOE_STAGE_BWD_DX = 8,
   MOE_STAGE_BWD_TRANSPOSE = 9,
   MOE_STAGE_BWD_WGRAD = 10,
-  MOE_NUM_STAGES = 11
+  MOE_STAGE_BWD_SWIGLU = 11, /* S8: d(router weights) + SwiGLU backward + MX of dg|du   */
+  MOE_NUM_STAGES = 12
 } moe_stage;
 
 /* When enabled, every stage launched by moe_forward / moe_backward is bracketed by CUDA

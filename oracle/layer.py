@@ -20,8 +20,9 @@ Definitions used (the configuration fills what the pages leave open):
     out_t  = sum_j w[t,j] * y_{t*k+j}
   backward (readings: the quantiser is a straight-through estimator; every backward
   GEMM operand is MX-quantised along that GEMM's K axis; the saved SwiGLU
-  pre-activations g, u are kept in bf16; dg, du and dy = w*dOut are materialised in bf16
-  before they are quantised):
+  pre-activations g, u are kept in bf16; every weight-gradient operand is the
+  token-direction requantisation of the dequantised MX operand the data path already
+  holds -- x^, h^, w*dout^ and [dg|du]^):
     dout^_t   = MX(dOut_t) along d
     G_a       = dout^_t . Wd'_e^T          (Wd' = W_down quantised along d)
     dw[t,j]   = <G_a, h^_a>                (gradient w.r.t. the combine weight)
@@ -31,7 +32,8 @@ Definitions used (the configuration fills what the pages leave open):
     dX_t      = sum_j dxa_{t*k+j}
     dWd_e     = H~_e^T . DY~_e,   dWg_e = X~_e^T . DG~_e,   dWu_e = X~_e^T . DU~_e
       where ~ is MX quantisation along the tokens of expert e's segment (blocks of 32
-      rows in ascending-token order, zero-padded), H = h^, X = x^, DY = w * dOut.
+      rows in ascending-token order, zero-padded), H = h^, X = x^, DY = w * dout^ and
+      [DG|DU] = [dg|du]^ (the operand of the dX GEMM).
 """
 from __future__ import annotations
 
@@ -200,15 +202,16 @@ def backward(x_bits, logits, dout_bits, k, score_fn, E, weights_fn, experts=None
         dw[rows] = np.sum(G * hhat, axis=1)
         dh = wflat[rows][:, None] * G
         s = sigmoid(gb)
-        dg = _bf(dh * ub * s * (1.0 + gb * (1.0 - s)), exact)
-        du = _bf(dh * gb * s, exact)
+        dg = dh * ub * s * (1.0 + gb * (1.0 - s))
+        du = dh * gb * s
         dgu_hat = _fq(np.concatenate([dg, du], axis=1), exact)
         if want_dx:
             np.add.at(dx, t, dgu_hat @ wgu_k.T)
-        # weight gradients: operands quantised along this expert's tokens
-        dy = _bf(wflat[rows][:, None] * dout[t], exact)
+        # weight gradients: the data path's MX operands requantised along the tokens
+        dy = wflat[rows][:, None] * dhat[t]
         Ht, DYt = _tok_fake(hhat, exact), _tok_fake(dy, exact)
-        Xt, DGt, DUt = _tok_fake(xhat[t], exact), _tok_fake(dg, exact), _tok_fake(du, exact)
+        Xt = _tok_fake(xhat[t], exact)
+        DGt, DUt = _tok_fake(dgu_hat[:, :f], exact), _tok_fake(dgu_hat[:, f:], exact)
         dW[e] = (Xt.T @ DGt, Xt.T @ DUt, Ht.T @ DYt)
     return dict(idx=idx, w=w, counts=counts, offsets=offsets, perm=perm, inv=inv,
                 dx=dx, dw=dw.reshape(T, k), dW=dW)

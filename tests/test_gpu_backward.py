@@ -2,11 +2,11 @@
 
 dX and d(routing weights) must reach relative Frobenius error <= 2e-3 and max-abs <=
 3e-2*RMS.  The weight gradients reach relative Frobenius <= 2e-3 per expert matrix; their
-element-wise bound allows for requantisation decisions: dg, du and w*dOut are computed
-values (fp32 on the GPU, fp64 in the oracle) that are rounded to bf16 and quantised to
-E4M3 along the tokens, so a value on a rounding boundary can land one code apart, and
-in a sum over an expert's tokens one such code moves an element by up to ~0.1*RMS (the
-oracle itself does this under 1e-6 relative noise).  Elements beyond 3e-2*RMS must be
+element-wise bound allows for requantisation decisions: the saved g, u (bf16) and dg, du
+(MX along f, then along the tokens) are computed values (fp32 on the GPU, fp64 in the
+oracle), so a value on a rounding boundary can land one code apart, and in a sum over an
+expert's tokens one such code moves an element by up to ~0.1*RMS (the oracle itself does
+this under 1e-6 relative noise).  Elements beyond 3e-2*RMS must be
 rare (<= 1e-4 of all weight-gradient elements) and below 0.25*RMS.  An expert without
 tokens gets an exactly zero weight gradient.
 """

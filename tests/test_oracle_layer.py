@@ -226,11 +226,11 @@ def test_bf16_round_matches_torch_on_fp32_values():
 
 
 def test_weight_gradient_sensitivity(monkeypatch):
-    """The oracle against itself with 1e-6 relative noise on its bf16 roundings (what fp32
-    vs fp64 arithmetic does to dg, du, w*dOut and the saved g, u): requantisation flips move
-    rare weight-gradient elements beyond 3e-2*RMS, which is why the GPU comparison bounds
-    their number (<= 1e-4) and size (<= 0.25*RMS) instead of requiring none; dX keeps the
-    strict bound."""
+    """The oracle against itself with 1e-6 relative noise on the saved bf16 pre-activations
+    (about what fp32 vs fp64 arithmetic does to them and to dg, du downstream):
+    requantisation flips move rare weight-gradient elements beyond 3e-2*RMS, which is why
+    the GPU comparison bounds their number (<= 1e-4) and size (<= 0.25*RMS) instead of
+    requiring none; dX keeps the strict bound."""
     case = synth.MoeCase("bh", 200, 512, 256, 32, 4, 1, "hot4cold16", seed=8)
     x, lg, wfn = _inputs(case)
     dout = synth.make_dout(case)

@@ -16,7 +16,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned
 OP_ROUTE, OP_FORWARD, OP_BACKWARD = 0, 1, 2
 
 STAGES = ["route", "permute", "gateup", "down", "combine", "bwd_dout", "bwd_dgrad_down",
-          "bwd_dgrad_gateup", "bwd_dx", "bwd_transpose", "bwd_wgrad"]
+          "bwd_dgrad_gateup", "bwd_dx", "bwd_transpose", "bwd_wgrad", "bwd_swiglu"]
 
 
 class MoeDims(ctypes.Structure):

@@ -172,7 +172,7 @@ struct WsLayout {
   int64_t idx = 0, w = 0, counts = 0, offsets = 0, perm = 0, inv = 0, pad = 0;
   int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0;
   // backward
-  int64_t dq = 0, ds = 0, dgu_bf = 0, dgu_q = 0, dgu_s = 0, dxa = 0;
+  int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, gbuf = 0;
   int64_t xt_q = 0, xt_s = 0, ht_q = 0, ht_s = 0, gt_q = 0, gt_s = 0, yt_q = 0, yt_s = 0;
   int64_t total = 0;
 };
@@ -198,10 +198,10 @@ WsLayout ws_layout(const moe_dims* D, int op) {
     const int64_t d = D->d, f = D->f;
     L.dq = c.take(R * d);
     L.ds = c.take(moe_umma_scale_bytes(R, d));
-    L.dgu_bf = c.take(R * 2 * f * 2);
     L.dgu_q = c.take(R * 2 * f);
     L.dgu_s = c.take(moe_umma_scale_bytes(R, 2 * f));
     L.dxa = c.take(4 * R * d);
+    L.gbuf = c.take(4 * R * f);
     L.xt_q = c.take(d * R);
     L.xt_s = c.take(moe_umma_scale_bytes(d, R));
     L.ht_q = c.take(f * R);
@@ -657,13 +657,12 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
   int32_t* status = at<int32_t>(ws, 0);
   uint8_t* dq = at<uint8_t>(ws, L.dq);
   uint8_t* dsc = at<uint8_t>(ws, L.ds);
-  uint16_t* dgu_bf = at<uint16_t>(ws, L.dgu_bf);
   uint8_t* dgu_q = at<uint8_t>(ws, L.dgu_q);
   uint8_t* dgu_s = at<uint8_t>(ws, L.dgu_s);
   float* dxa = at<float>(ws, L.dxa);
+  float* gbuf = at<float>(ws, L.gbuf);
 
   if (D->T > 0) {
-    MOE_TRY(cuda_ok(cudaMemsetAsync(dw_route, 0, 4 * D->T * D->k, st)));
     {  // pull reverse-combine: dOut rows gathered into expert order, MXFP8 along d
       StageScope sc(MOE_STAGE_BWD_DOUT, st);
       PermuteParams P;
@@ -681,33 +680,44 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.status = status;
       MOE_TRY(cuda_ok(launch_permute_quant(P, sms, st)));
     }
-    {  // G = dOut^ . Wd'^T, dw_route, SwiGLU backward, dg/du requantisation
+    {  // G = dout^ . Wd'^T (fp32, padded expert order)
       StageScope sc(MOE_STAGE_BWD_DGRAD_DOWN, st);
-      CUtensorMap ta, tb;
+      CUtensorMap ta, tb, tg;
       MOE_TRY(make_tmap(&ta, dq, R, d, 128));
       MOE_TRY(make_tmap(&tb, W->wdT_q, static_cast<int64_t>(E) * f, d, 256));
+      MOE_TRY(make_out_tmap(&tg, gbuf, R, f, false));
       GemmParams P = {};
       P.G = E;
       P.N = f;
       P.K = d;
-      P.f = f;
       P.mtile_prefix = S->pad_offsets;
       P.prefix_shift = 7;
       P.rows_valid = S->counts;
       P.sfa = dsc;
       P.sfb = W->wdT_s;
+      P.out_f32 = gbuf;
+      P.ld_out = f;
+      P.status = status;
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg, P, sms, st)));
+    }
+    {  // d(router weights), SwiGLU backward, [dg|du] -> MXFP8 along f
+      StageScope sc(MOE_STAGE_BWD_SWIGLU, st);
+      SwigluBwdParams P;
+      P.G = gbuf;
       P.gu = S->gu;
       P.h_q = S->hq;
       P.h_s = S->hs;
       P.perm = S->perm;
       P.offsets = S->offsets;
+      P.pad_offsets = S->pad_offsets;
       P.topk_w = S->topk_w;
+      P.A = D->T * D->k;
+      P.E = E;
+      P.f = f;
       P.dw_route = dw_route;
-      P.dgu_bf = dgu_bf;
       P.dgu_q = dgu_q;
       P.dgu_s = dgu_s;
-      P.status = status;
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_DGRAD_SWIGLU, ta, tb, ta, tb, P, sms, st)));
+      MOE_TRY(cuda_ok(launch_swiglu_bwd(P, sms, st)));
     }
     {  // dXa = [dg|du]^ . [Wg|Wu]'^T
       StageScope sc(MOE_STAGE_BWD_DGRAD_GATEUP, st);
@@ -782,16 +792,15 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     P.dst_q = ht_q;
     P.dst_s = ht_s;
     MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
-    P.src = TSRC_BF16;  // bf16 dg | du -> DGU~^T [2f, R]
-    P.bf = dgu_bf;
-    P.ld = 2 * f;
+    P.q = dgu_q;      // [dg|du]^ -> DGU~^T [2f, R]
+    P.s = dgu_s;
     P.C = 2 * f;
     P.dst_q = gt_q;
     P.dst_s = gt_s;
     MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
-    P.src = TSRC_DY;    // bf16(w * dOut) gathered -> DY~^T [d, R]
-    P.bf = dout;
-    P.ld = d;
+    P.src = TSRC_MX_W;  // w * dout^ -> DY~^T [d, R]
+    P.q = dq;
+    P.s = dsc;
     P.C = d;
     P.dst_q = yt_q;
     P.dst_s = yt_s;

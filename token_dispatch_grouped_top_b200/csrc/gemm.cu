@@ -22,12 +22,11 @@
 // that a weight tile is read from HBM once and re-read by the neighbouring CTAs from L2.
 //
 // Modes (epilogues):
-//   STORE_F32      D in fp32 (the down projection and the dgrad of the expert input).
+//   STORE_F32      D in fp32 (per-thread row stores; the generic path).
+//   STORE_F32_TMA  D in fp32 through shared memory and TMA stores (the down projection
+//                  and both dgrad GEMMs of the backward).
 //   GATEUP_SWIGLU  h = silu(g) * u on paired gate/up columns, MXFP8 requantisation of h
 //                  along f (the input of the down GEMM), optional bf16 save of g and u.
-//   DGRAD_SWIGLU   backward of the down projection: G = dOut^ . Wd'^T; dw_route[a] +=
-//                  <G, h^> over the tile; dh = w * G; SwiGLU backward with the saved bf16
-//                  g, u; dg, du rounded to bf16 and requantised along f.
 //   WGRAD_BF16     weight gradients: the reduction runs over one expert's (padded) token
 //                  segment, so K varies per group and M, N are fixed; bf16 output, an
 //                  expert without tokens gets an all-zero gradient.
@@ -55,7 +54,10 @@ struct ModeCfg {
   // A tile with fewer than 128 valid rows (an expert's last tile) runs with the operands
   // swapped: the two 128-row halves of the B tile are the M side of two MMAs and the
   // valid A rows, rounded up to 16, the N side -- the tensor work shrinks with the rows.
-  static constexpr bool kSwapTail = MODE == GEMM_GATEUP_SWIGLU || MODE == GEMM_STORE_F32_TMA;
+  // (Measured: a gain for the fp32-output GEMMs; with the SwiGLU epilogue, whose
+  // transposed form quantises across lanes, the gate/up GEMM became slower, so it keeps
+  // full tiles.)
+  static constexpr bool kSwapTail = MODE == GEMM_STORE_F32_TMA;
 };
 
 template <int ST, int NSTG>
@@ -135,6 +137,12 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
   return decode_tile_var_m(tile, prefix, valid, P.G, P.N / BN, P.N, P.K / BK);
 }
 
+// sigmoid(x) = 1 / (1 + e^-x) with the fast exponential and a rounded reciprocal: the
+// epilogues evaluate it once per output element, and the IEEE exp + division sequence
+// kept the transcendental pipe busy for as long as the MMA main loop of a short-K tile.
+// Relative error ~1e-6 (large |x|: e^-x -> 0 or inf gives exactly 1 or 0).
+__device__ __forceinline__ float sigmoid_fast(float x) { return __frcp_rn(1.f + __expf(-x)); }
+
 // E4M3 byte -> fp32, exact (normal: (1 + m/8) 2^(e-7); subnormal: m 2^-9).
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
   const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
@@ -168,7 +176,7 @@ __device__ __forceinline__ void swapped_gateup_epilogue(const GemmParams& P, con
   uint32_t my_sb = 0;
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    const float hv = g[c] / (1.f + expf(-g[c])) * u[c];
+    const float hv = g[c] * sigmoid_fast(g[c]) * u[c];
     float amax = fabsf(hv);
 #pragma unroll
     for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
@@ -188,73 +196,6 @@ __device__ __forceinline__ void swapped_gateup_epilogue(const GemmParams& P, con
     const int64_t row = ti.a_row0 + tb + lane;
     P.hs[umma_scale_offset(row, fi >> 5, f >> 7)] = static_cast<uint8_t>(my_sb);
   }
-}
-
-// DGRAD epilogue for 32 features [fc, fc+32) of one row: returns this chunk's part of
-// <G, h^>; writes dg, du (bf16) and their MX codes/scales along f.
-__device__ __forceinline__ float dgrad_chunk(const GemmParams& P, const float (&G)[32],
-                                             int64_t row, int fc, float w) {
-  const int f = P.f;
-  const uint4* hp = reinterpret_cast<const uint4*>(P.h_q + row * f + fc);
-  const uint4 h0 = hp[0], h1 = hp[1];
-  const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-  const float hsc = e8m0_to_f32(P.h_s[umma_scale_offset(row, fc >> 5, f >> 7)]);
-  const uint4* gp = reinterpret_cast<const uint4*>(P.gu + row * 2 * f + fc);
-  const uint4* up = reinterpret_cast<const uint4*>(P.gu + row * 2 * f + f + fc);
-  uint32_t dgp[16], dup[16];
-  float dwp = 0.f;
-#pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    const uint4 gq = gp[v], uq = up[v];
-    const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
-    const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
-#pragma unroll
-    for (int e2 = 0; e2 < 4; ++e2) {
-      uint32_t outg = 0, outu = 0;
-#pragma unroll
-      for (int hlf = 0; hlf < 2; ++hlf) {
-        const int i = 8 * v + 2 * e2 + hlf;
-        const float g_acc = G[i];
-        const float hv = e4m3_to_f32((hw[i >> 2] >> (8 * (i & 3))) & 0xFFu) * hsc;
-        dwp = fmaf(g_acc, hv, dwp);
-        const float gb = bf16_bits_to_f32((gw[e2] >> (16 * hlf)) & 0xFFFFu);
-        const float ub = bf16_bits_to_f32((uw[e2] >> (16 * hlf)) & 0xFFFFu);
-        const float dh = w * g_acc;
-        const float sg = 1.f / (1.f + expf(-gb));
-        const float dg = dh * ub * sg * (1.f + gb * (1.f - sg));
-        const float du = dh * gb * sg;
-        outg |= f32_to_bf16_bits(dg) << (16 * hlf);
-        outu |= f32_to_bf16_bits(du) << (16 * hlf);
-      }
-      dgp[4 * v + e2] = outg;
-      dup[4 * v + e2] = outu;
-    }
-  }
-  uint4* gdst = reinterpret_cast<uint4*>(P.dgu_bf + row * 2 * f + fc);
-  uint4* udst = reinterpret_cast<uint4*>(P.dgu_bf + row * 2 * f + f + fc);
-#pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    gdst[v] = make_uint4(dgp[4 * v], dgp[4 * v + 1], dgp[4 * v + 2], dgp[4 * v + 3]);
-    udst[v] = make_uint4(dup[4 * v], dup[4 * v + 1], dup[4 * v + 2], dup[4 * v + 3]);
-  }
-#pragma unroll
-  for (int which = 0; which < 2; ++which) {  // MX requantisation of bf16 dg / du along f
-    float blk[32];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t wv = which ? dup[i] : dgp[i];
-      blk[2 * i] = bf16_bits_to_f32(wv & 0xFFFFu);
-      blk[2 * i + 1] = bf16_bits_to_f32(wv >> 16);
-    }
-    uint32_t qw[8];
-    const uint32_t sb = mx_quant_block32(blk, qw);
-    const int col = which * f + fc;
-    uint4* qd = reinterpret_cast<uint4*>(P.dgu_q + row * 2 * f + col);
-    qd[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
-    qd[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
-    P.dgu_s[umma_scale_offset(row, col >> 5, (2 * f) >> 7)] = static_cast<uint8_t>(sb);
-  }
-  return dwp;
 }
 
 // Stage one 32-row x 128-byte chunk (row = lane) in shared memory with the 128-byte swizzle
@@ -531,18 +472,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (ti.i * BM + m >= S.valid[ti.g]) continue;
       const int64_t row = ti.a_row0 + m;
-      if (MODE == GEMM_DGRAD_SWIGLU) {
-        const int64_t q_pos = static_cast<int64_t>(P.offsets[ti.g]) + ti.i * BM + m;
-        const int a = P.perm[q_pos];
-        const float w = P.topk_w[a];
-        const int n0 = ti.j * BN + 128 * h;  // first feature of this thread's 128
-        float dwp = dgrad_chunk(P, v0, row, n0, w);
-        dwp += dgrad_chunk(P, v1, row, n0 + 32, w);
-        dwp += dgrad_chunk(P, v2, row, n0 + 64, w);
-        dwp += dgrad_chunk(P, v3, row, n0 + 96, w);
-        atomicAdd(P.dw_route + a, dwp);
-        continue;
-      }
       if (MODE == GEMM_GATEUP_SWIGLU) {
         const int f = P.f;
         const int fb = BN / 2 * ti.j + 64 * h;  // first feature of this thread's 64
@@ -566,8 +495,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // h = silu(g) * u, in place over the gate registers
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          v0[c] = v0[c] / (1.f + expf(-v0[c])) * v2[c];
-          v1[c] = v1[c] / (1.f + expf(-v1[c])) * v3[c];
+          v0[c] = v0[c] * sigmoid_fast(v0[c]) * v2[c];
+          v1[c] = v1[c] * sigmoid_fast(v1[c]) * v3[c];
         }
         uint32_t q0[8], q1[8];
         const uint32_t s0 = mx_quant_block32(v0, q0);
@@ -630,8 +559,6 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensor
       return launch_mode<GEMM_STORE_F32>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_GATEUP_SWIGLU:
       return launch_mode<GEMM_GATEUP_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
-    case GEMM_DGRAD_SWIGLU:
-      return launch_mode<GEMM_DGRAD_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_WGRAD_BF16:
       return launch_mode<GEMM_WGRAD_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_STORE_F32_TMA:

@@ -97,15 +97,12 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
 // [C, R] E4M3 with the UMMA scales of the [C, R] matrix.
 enum TransposeSrc : int {
   TSRC_MX = 0,       // MX codes [R, C] + UMMA scales (kgroups C/128): dequantised exactly
-  TSRC_BF16 = 1,     // bf16 [R, C] with row stride ld
-  TSRC_DY = 2,       // bf16(w_a * dout[t_a]) gathered from dout [T, C] (row stride ld)
+  TSRC_MX_W = 1,     // the same, each row times the combine weight of its assignment
 };
 struct TransposeQuantParams {
   int src;
   const uint8_t* q;
   const uint8_t* s;
-  const uint16_t* bf;
-  int64_t ld;
   const int32_t* perm;
   const int32_t* offsets;
   const float* topk_w;
@@ -121,11 +118,28 @@ struct TransposeQuantParams {
 };
 cudaError_t launch_transpose_quant(const TransposeQuantParams& P, cudaStream_t stream);
 
+// SwiGLU backward + d(router weights) per assignment row, from G = dout^ . Wd'^T.
+struct SwigluBwdParams {
+  const float* G;           // [R, f] fp32, padded expert order
+  const uint16_t* gu;       // [R, 2f] saved bf16 g | u
+  const uint8_t* h_q;       // [R, f] forward h codes + UMMA scales
+  const uint8_t* h_s;
+  const int32_t* perm;
+  const int32_t* offsets;
+  const int32_t* pad_offsets;
+  const float* topk_w;
+  int64_t A;
+  int E, f;
+  float* dw_route;          // [A]
+  uint8_t* dgu_q;           // [R, 2f] MX codes of dg | du + UMMA scales
+  uint8_t* dgu_s;
+};
+cudaError_t launch_swiglu_bwd(const SwigluBwdParams& P, int num_sms, cudaStream_t stream);
+
 // Grouped block-scaled GEMM.
 enum GemmMode : int {
   GEMM_STORE_F32 = 0,      // D fp32 [rows, N] (down projection, dgrad of x, generic)
   GEMM_GATEUP_SWIGLU = 1,  // SwiGLU + MX requant of h, optional bf16 g/u save
-  GEMM_DGRAD_SWIGLU = 2,   // G = dOut . Wd^T -> dw_route, SwiGLU backward, dg/du bf16 + MX
   GEMM_WGRAD_BF16 = 3,     // variable K per group (the group's token segment), bf16 out
   GEMM_STORE_F32_TMA = 4,  // as STORE_F32 through shared memory + TMA stores; writes whole
                            // 128-row tiles (rows past a group's count get unused values)
@@ -146,17 +160,7 @@ struct GemmParams {
   int64_t ld_out;
   uint8_t* hq;           // GATEUP: [rows, f]
   uint8_t* hs;           // GATEUP: UMMA scales of [rows, f]
-  uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16; DGRAD: saved g/u (read)
-  // DGRAD
-  const uint8_t* h_q;    // forward h codes [rows, f] + UMMA scales
-  const uint8_t* h_s;
-  const int32_t* perm;
-  const int32_t* offsets;
-  const float* topk_w;
-  float* dw_route;       // [A] (accumulated with atomics; zeroed before the launch)
-  uint16_t* dgu_bf;      // [rows, 2f] bf16 dg | du
-  uint8_t* dgu_q;        // [rows, 2f] MX codes + UMMA scales of the [rows, 2f] matrix
-  uint8_t* dgu_s;
+  uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16 save of g | u
   // WGRAD: D[g] rows m < M, cols n < N -> (n < split ? out_a : out_b)[g][m][n mod split]
   uint16_t* out_a;
   uint16_t* out_b;
