@@ -211,9 +211,10 @@ def run_reference(args, case):
     print(json.dumps(line), flush=True)
 
 
-# kernels launched per stage (route: routing + scatter; transposes: 4; wgrad: 2 GEMMs)
-KERNELS_PER_STAGE = {"route": 2, "permute": 1, "gateup": 1, "down": 1, "combine": 1,
-                     "bwd_dout": 1, "bwd_dgrad_down": 1, "bwd_dgrad_gateup": 1, "bwd_dx": 1,
+# kernels launched per stage (route: routing + scatter; permute / bwd_dout: per-token
+# quantisation + pull gather; transposes: 4; wgrad: 2 GEMMs)
+KERNELS_PER_STAGE = {"route": 2, "permute": 2, "gateup": 1, "down": 1, "combine": 1,
+                     "bwd_dout": 2, "bwd_dgrad_down": 1, "bwd_dgrad_gateup": 1, "bwd_dx": 1,
                      "bwd_transpose": 4, "bwd_wgrad": 2, "bwd_swiglu": 1}
 
 

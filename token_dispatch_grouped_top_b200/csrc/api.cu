@@ -171,6 +171,7 @@ struct WsLayout {
   int64_t flags = 0, agg = 0, incl = 0, rank = 0, mtile = 0;
   int64_t idx = 0, w = 0, counts = 0, offsets = 0, perm = 0, inv = 0, pad = 0;
   int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0;
+  int64_t tq = 0, ts = 0;  // per-token MX copy of x (forward) or dout (backward)
   // backward
   int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, gbuf = 0;
   int64_t xt_q = 0, xt_s = 0, ht_q = 0, ht_s = 0, gt_q = 0, gt_s = 0, yt_q = 0, yt_s = 0;
@@ -194,6 +195,10 @@ WsLayout ws_layout(const moe_dims* D, int op) {
   L.incl = c.take(4 * nt * E);
   L.rank = c.take(4 * A);
   L.mtile = c.take(4 * (E + 1));
+  if (op >= MOE_OP_FORWARD) {
+    L.tq = c.take(D->T * D->d);
+    L.ts = c.take(D->T * (D->d / 32));
+  }
   if (op == MOE_OP_BACKWARD) {
     const int64_t d = D->d, f = D->f;
     L.dq = c.take(R * d);
@@ -272,6 +277,41 @@ moe_status route_empty(const moe_dims* D, int32_t* counts, int32_t* offsets, int
   if (mtile) MOE_TRY(cuda_ok(cudaMemsetAsync(mtile, 0, 4 * (D->E + 1), st)));
   if (pad) MOE_TRY(cuda_ok(cudaMemsetAsync(pad, 0, 4 * (D->E + 1), st)));
   return MOE_OK;
+}
+
+// Pull dispatch: quantise every token row once (MXFP8 along d, canonical scales), then
+// each expert row pulls its token's codes and scales by index into the padded layout.
+moe_status dispatch_pull(const moe_dims* D, const uint16_t* src, const int32_t* offsets,
+                         const int32_t* prefix, int prefix_shift, const int32_t* perm,
+                         uint8_t* tok_q, uint8_t* tok_s, uint8_t* out_q, uint8_t* out_s,
+                         int32_t* status, int sms, cudaStream_t st) {
+  QuantRowsParams Q;
+  Q.src = src;
+  Q.src_ld = D->d;
+  Q.rows = D->T;
+  Q.K = D->d;
+  Q.dst = tok_q;
+  Q.dst_ld = D->d;
+  Q.dst_col0 = 0;
+  Q.scales = tok_s;
+  Q.layout = 0;
+  Q.kgroups = D->d / 128;
+  MOE_TRY(cuda_ok(launch_quant_rows(Q, sms, st)));
+  GatherParams G;
+  G.q_tok = tok_q;
+  G.s_tok = tok_s;
+  G.T = D->T;
+  G.d = D->d;
+  G.E = D->E;
+  G.k = D->k;
+  G.offsets = offsets;
+  G.mtile_prefix = prefix;
+  G.prefix_shift = prefix_shift;
+  G.perm = perm;
+  G.q_out = out_q;
+  G.s_out = out_s;
+  G.status = status;
+  return cuda_ok(launch_gather_rows(G, sms, st));
 }
 
 }  // namespace
@@ -554,20 +594,8 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
   const int64_t R = padded_rows(D);
   {
     StageScope sc(MOE_STAGE_PERMUTE, st);
-    PermuteParams P;
-    P.x = x;
-    P.T = D->T;
-    P.d = D->d;
-    P.E = D->E;
-    P.k = D->k;
-    P.offsets = offsets;
-    P.mtile_prefix = mtile;
-    P.prefix_shift = 0;
-    P.perm = perm;
-    P.xq = xq;
-    P.xs = xs;
-    P.status = status;
-    MOE_TRY(cuda_ok(launch_permute_quant(P, sms, st)));
+    MOE_TRY(dispatch_pull(D, x, offsets, mtile, 0, perm, at<uint8_t>(ws, L.tq),
+                          at<uint8_t>(ws, L.ts), xq, xs, status, sms, st));
   }
   {
     StageScope sc(MOE_STAGE_GATEUP, st);
@@ -665,20 +693,9 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
   if (D->T > 0) {
     {  // pull reverse-combine: dOut rows gathered into expert order, MXFP8 along d
       StageScope sc(MOE_STAGE_BWD_DOUT, st);
-      PermuteParams P;
-      P.x = dout;
-      P.T = D->T;
-      P.d = d;
-      P.E = E;
-      P.k = D->k;
-      P.offsets = S->offsets;
-      P.mtile_prefix = S->pad_offsets;
-      P.prefix_shift = 7;
-      P.perm = S->perm;
-      P.xq = dq;
-      P.xs = dsc;
-      P.status = status;
-      MOE_TRY(cuda_ok(launch_permute_quant(P, sms, st)));
+      MOE_TRY(dispatch_pull(D, dout, S->offsets, S->pad_offsets, 7, S->perm,
+                            at<uint8_t>(ws, L.tq), at<uint8_t>(ws, L.ts), dq, dsc, status, sms,
+                            st));
     }
     {  // G = dout^ . Wd'^T (fp32, padded expert order)
       StageScope sc(MOE_STAGE_BWD_DGRAD_DOWN, st);

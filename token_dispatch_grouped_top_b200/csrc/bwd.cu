@@ -43,10 +43,8 @@ constexpr int kTqMaxE = 1024;
 // along the rows and writes 32 bytes of the transposed output.
 __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(TransposeQuantParams P) {
   __shared__ __align__(16) uint8_t s_codes[kTqRows][kTqPitch];
-  __shared__ uint32_t s_scales[kTqRows];
-  __shared__ float s_row_w[kTqRows];
+  __shared__ float s_mul[kTqCols / 32][kTqRows];  // 2^s of (row, 32-column block) x weight
   __shared__ int s_pad[kTqMaxE + 1];
-  __shared__ int s_nvalid[kTqRows / 32];
   const int64_t p0 = static_cast<int64_t>(blockIdx.y) * kTqRows;  // first row of the block
   const int c0 = blockIdx.x * kTqCols;                              // first column
   const int tid = threadIdx.x;
@@ -62,20 +60,17 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(TransposeQu
   int nv_blk = static_cast<int>(P.counts[lo] - rel);
   if (p0 >= s_pad[P.E]) nv_blk = 0;
   nv_blk = nv_blk < 0 ? 0 : (nv_blk > kTqRows ? kTqRows : nv_blk);
-  if (tid < kTqRows / 32) {
-    const int n = nv_blk - 32 * tid;
-    s_nvalid[tid] = n < 0 ? 0 : (n > 32 ? 32 : n);
-  }
   if (tid < kTqRows) {
-    float w = 1.f;
+    float w = 0.f;
     uint32_t sw = 0;
     if (tid < nv_blk) {
-      if (P.src == TSRC_MX_W) w = P.topk_w[P.perm[P.offsets[lo] + rel + tid]];
+      w = P.src == TSRC_MX_W ? P.topk_w[P.perm[P.offsets[lo] + rel + tid]] : 1.f;
       sw = *reinterpret_cast<const uint32_t*>(P.s + umma_scale_offset(p0 + tid, c0 >> 5,
                                                                        P.C >> 7));
     }
-    s_row_w[tid] = w;
-    s_scales[tid] = sw;
+#pragma unroll
+    for (int cb = 0; cb < kTqCols / 32; ++cb)
+      s_mul[cb][tid] = e8m0_to_f32_t((sw >> (8 * cb)) & 0xFFu) * w;
   }
   // codes: 128 rows x 128 bytes, 8 threads per row, 16 bytes each
 #pragma unroll
@@ -90,11 +85,10 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(TransposeQu
   __syncthreads();
   const int c = tid & (kTqCols - 1);  // column within the block
   const int hb = tid >> 7;            // 32-row blocks hb and hb + 2
-  const int sbyte = (c >> 5) * 8;     // shift of this column's scale in a row's word
+  const float* mul = s_mul[c >> 5];
 #pragma unroll 1
   for (int bb = 0; bb < 2; ++bb) {
     const int b = hb + 2 * bb;
-    const int nv = s_nvalid[b];
     float v[32];
 #pragma unroll
     for (int r = 0; r < 32; r += 2) {  // rows r, r+1: one hardware E4M3x2 -> f16x2 decode
@@ -103,12 +97,10 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(TransposeQu
                             (static_cast<uint32_t>(s_codes[rr + 1][c]) << 8);
       uint32_t h2;
       asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
-      const float lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-      const float hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
-      v[r] = r < nv ? lo * e8m0_to_f32_t((s_scales[rr] >> sbyte) & 0xFFu) * s_row_w[rr] : 0.f;
-      v[r + 1] = r + 1 < nv
-                     ? hi * e8m0_to_f32_t((s_scales[rr + 1] >> sbyte) & 0xFFu) * s_row_w[rr + 1]
-                     : 0.f;
+      // rows past the segment's count have multiplier 0 (and zero codes)
+      v[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu))) * mul[rr];
+      v[r + 1] =
+          __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16))) * mul[rr + 1];
     }
     uint32_t qw[8];
     const uint32_t sb = mx_quant_block32(v, qw);

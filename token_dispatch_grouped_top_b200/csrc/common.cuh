@@ -292,10 +292,16 @@ __host__ __device__ __forceinline__ int64_t umma_scale_offset(int64_t r, int64_t
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
-// fp32 -> bf16 bits, round to nearest even (inputs are finite).
+// Two fp32 -> two bf16 (lo in bits 0-15), round to nearest even, one instruction.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// fp32 -> bf16 bits, round to nearest even.
 __device__ __forceinline__ uint32_t f32_to_bf16_bits(float x) {
-  uint32_t u = __float_as_uint(x);
-  return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+  return pack_bf16x2(x, 0.f) & 0xFFFFu;
 }
 
 }  // namespace moe

@@ -32,6 +32,7 @@
 //                  expert without tokens gets an all-zero gradient.
 #include "common.cuh"
 #include "kernels.h"
+#include "tile_store.cuh"
 
 namespace moe {
 
@@ -154,68 +155,6 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
 // E8M0 byte -> 2^(b-127) as fp32 (2^-127 is subnormal).
 __device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
   return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
-}
-
-__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
-  return make_uint4(f32_to_bf16_bits(v[0]) | (f32_to_bf16_bits(v[1]) << 16),
-                    f32_to_bf16_bits(v[2]) | (f32_to_bf16_bits(v[3]) << 16),
-                    f32_to_bf16_bits(v[4]) | (f32_to_bf16_bits(v[5]) << 16),
-                    f32_to_bf16_bits(v[6]) | (f32_to_bf16_bits(v[7]) << 16));
-}
-
-// Swapped gate/up tail epilogue for 32 tokens [tb, tb+32) of one warp: lane = feature
-// (gate in g[], up in u[], column = token).  h = silu(g) * u is quantised along the
-// features, i.e. across the 32 lanes of the warp (one MX block per token).
-__device__ __forceinline__ void swapped_gateup_epilogue(const GemmParams& P, const TileInfo& ti,
-                                                        int q, int lane, int tb,
-                                                        const float (&g)[32],
-                                                        const float (&u)[32]) {
-  if (tb >= ti.rows) return;  // warp-uniform
-  const int f = P.f;
-  const int fi = (BN / 2) * ti.j + 32 * q + lane;  // this lane's feature
-  uint32_t my_sb = 0;
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    const float hv = g[c] * sigmoid_fast(g[c]) * u[c];
-    float amax = fabsf(hv);
-#pragma unroll
-    for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
-    const int s = mx_scale_exp(amax);
-    const uint32_t code = cvt_e4m3x2(hv * mx_inv_scale(s), 0.f) & 0xFFu;
-    if (c == lane) my_sb = static_cast<uint32_t>(s + 127);
-    if (tb + c < ti.rows) {
-      const int64_t row = ti.a_row0 + tb + c;
-      P.hq[row * f + fi] = static_cast<uint8_t>(code);
-      if (P.gu) {
-        P.gu[row * 2 * f + fi] = static_cast<uint16_t>(f32_to_bf16_bits(g[c]));
-        P.gu[row * 2 * f + f + fi] = static_cast<uint16_t>(f32_to_bf16_bits(u[c]));
-      }
-    }
-  }
-  if (tb + lane < ti.rows) {
-    const int64_t row = ti.a_row0 + tb + lane;
-    P.hs[umma_scale_offset(row, fi >> 5, f >> 7)] = static_cast<uint8_t>(my_sb);
-  }
-}
-
-// Stage one 32-row x 128-byte chunk (row = lane) in shared memory with the 128-byte swizzle
-// the output tensor map uses, then one lane stores it with TMA.  Two buffers per warp:
-// before a buffer is rewritten, the store issued from it two chunks ago must have read it.
-__device__ __forceinline__ void stage_and_store(uint8_t* buf, const uint4 (&row16)[8],
-                                                const CUtensorMap* tmap, int32_t x, int32_t y,
-                                                int lane) {
-  if (lane == 0) bulk_wait_read<1>();
-  __syncwarp();
-  uint8_t* r = buf + lane * 128;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    *reinterpret_cast<uint4*>(r + ((j ^ (lane & 7)) << 4)) = row16[j];
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_2d(tmap, smem_u32(buf), x, y);
-    bulk_commit();
-  }
 }
 
 template <int MODE>
@@ -379,13 +318,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&S.tmem_empty));
         acc_phase ^= 1u;
-        if (MODE == GEMM_GATEUP_SWIGLU) {
-          swapped_gateup_epilogue(P, ti, q, lane, tok0, d0a, d1a);
-          swapped_gateup_epilogue(P, ti, q, lane, tok0 + 32, d0b, d1b);
-        } else if (MODE == GEMM_STORE_F32_TMA) {
+        if (MODE == GEMM_STORE_F32_TMA) {
           const int32_t y0 = static_cast<int32_t>(ti.a_row0);
           const int32_t x0 = ti.j * BN + 32 * q;
-          const float* parts[4] = {d0a, d0b, d1a, d1b};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const int tb = tok0 + 32 * (c & 1);
@@ -406,7 +341,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             stg_buf ^= 1;
           }
-          (void)parts;
         }
         continue;
       }
@@ -482,14 +416,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int c = 0; c < 8; ++c) {
             const float* g = c < 4 ? v0 + 8 * c : v1 + 8 * (c - 4);
             const float* u = c < 4 ? v2 + 8 * c : v3 + 8 * (c - 4);
-            gdst[c] = make_uint4(f32_to_bf16_bits(g[0]) | (f32_to_bf16_bits(g[1]) << 16),
-                                 f32_to_bf16_bits(g[2]) | (f32_to_bf16_bits(g[3]) << 16),
-                                 f32_to_bf16_bits(g[4]) | (f32_to_bf16_bits(g[5]) << 16),
-                                 f32_to_bf16_bits(g[6]) | (f32_to_bf16_bits(g[7]) << 16));
-            udst[c] = make_uint4(f32_to_bf16_bits(u[0]) | (f32_to_bf16_bits(u[1]) << 16),
-                                 f32_to_bf16_bits(u[2]) | (f32_to_bf16_bits(u[3]) << 16),
-                                 f32_to_bf16_bits(u[4]) | (f32_to_bf16_bits(u[5]) << 16),
-                                 f32_to_bf16_bits(u[6]) | (f32_to_bf16_bits(u[7]) << 16));
+            gdst[c] = pack_bf16x8(g);
+            udst[c] = pack_bf16x8(u);
           }
         }
         // h = silu(g) * u, in place over the gate registers

@@ -59,20 +59,22 @@ struct QuantColsParams {
 };
 cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream);
 
-// Pull dispatch: Xq[pad_offsets[e] + r] = MX(x[perm[offsets[e] + r] / k]).
-struct PermuteParams {
-  const uint16_t* x;
+// Pull gather of per-token MX rows: q_out[pad_offsets[e] + r] = q_tok[perm[offsets[e]+r]/k],
+// scales from the canonical per-token layout [T, d/32] into the UMMA layout of [R, d].
+struct GatherParams {
+  const uint8_t* q_tok;
+  const uint8_t* s_tok;
   int64_t T;
   int d, E, k;
   const int32_t* offsets;
-  const int32_t* mtile_prefix;  // or the padded offsets with prefix_shift = 7
+  const int32_t* mtile_prefix;
   int prefix_shift;
   const int32_t* perm;
-  uint8_t* xq;
-  uint8_t* xs;
+  uint8_t* q_out;
+  uint8_t* s_out;
   int32_t* status;
 };
-cudaError_t launch_permute_quant(const PermuteParams& P, int num_sms, cudaStream_t stream);
+cudaError_t launch_gather_rows(const GatherParams& P, int num_sms, cudaStream_t stream);
 
 // Push combine: out[t] = sum_j w[t,j] * Y[pad_offsets[e] + inv[a] - offsets[e]], bf16.
 // topk_w == nullptr: unit weights (the backward's reverse dispatch, dX = sum_j dXa).

@@ -1,9 +1,10 @@
-// MXFP8 quantisation kernels, the pull-dispatch permute (S3) and the push combine (S6).
+// MXFP8 quantisation kernels, the pull-dispatch gather (S3) and the push combine (S6).
 //
 // Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72":
 //   §02 -- pull dispatch: the consumer fetches the rows it needs by source and offset and
-//          lays them out by expert; MXFP8 activations are fused into dispatch, so no
-//          separate quantisation kernel and no extra HBM round trip;
+//          lays them out by expert; MXFP8 activations travel through dispatch: each token
+//          is quantised once (the copy stays in L2) and every expert row pulls its token's
+//          codes, so the bf16 rows are read from HBM once instead of k times;
 //   §02/§03 -- push combine returns each expert result to its token's slot, followed by
 //          the final weighted merge.
 // All kernels here are HBM-bound: 16-byte vector loads, one warp per row, grids sized in
@@ -152,48 +153,6 @@ cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// S3: one warp per destination row; the row pulls its token by index (pull dispatch) and
-// quantises it on the way (MXFP8 fused into dispatch).
-__global__ void __launch_bounds__(256) permute_quant_kernel(PermuteParams P) {
-  __shared__ int s_off[kMaxE + 1];
-  __shared__ int s_mt[kMaxE + 1];
-  for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
-    s_off[i] = P.offsets[i];
-    s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int64_t A = P.T * P.k;
-  const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); q < A;
-       q += warps) {
-    int lo = 0, hi = P.E;  // s_off[lo] <= q < s_off[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (s_off[mid] <= q) lo = mid; else hi = mid;
-    }
-    const int e = lo;
-    const int a = P.perm[q];
-    const int64_t t = a / P.k;
-    const int64_t p = static_cast<int64_t>(s_mt[e]) * 128 + (q - s_off[e]);
-    if (a < 0 || t >= P.T || p >= R) {
-      if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
-      continue;
-    }
-    warp_quant_row(P.x + t * P.d, P.d, P.xq + p * P.d, P.xs, p, 0, 1, 0, P.d >> 7, lane);
-  }
-}
-
-cudaError_t launch_permute_quant(const PermuteParams& P, int num_sms, cudaStream_t stream) {
-  const int64_t A = P.T * P.k;
-  if (A <= 0) return cudaSuccess;
-  const int64_t blocks = (A + 7) / 8;
-  const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
-  permute_quant_kernel<<<grid, 256, 0, stream>>>(P);
-  return cudaGetLastError();
-}
-
 // S6: one warp per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
 // ascending, fp32), rounded to bf16.  With unit weights this is the backward's push
 // reverse-dispatch, dX[t] = sum_j dXa[row of (t, j)].
@@ -249,10 +208,10 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
         acc1.w += w * y1.w;
       }
       uint2 o0, o1;
-      o0.x = f32_to_bf16_bits(acc0.x) | (f32_to_bf16_bits(acc0.y) << 16);
-      o0.y = f32_to_bf16_bits(acc0.z) | (f32_to_bf16_bits(acc0.w) << 16);
-      o1.x = f32_to_bf16_bits(acc1.x) | (f32_to_bf16_bits(acc1.y) << 16);
-      o1.y = f32_to_bf16_bits(acc1.z) | (f32_to_bf16_bits(acc1.w) << 16);
+      o0.x = pack_bf16x2(acc0.x, acc0.y);
+      o0.y = pack_bf16x2(acc0.z, acc0.w);
+      o1.x = pack_bf16x2(acc1.x, acc1.y);
+      o1.y = pack_bf16x2(acc1.z, acc1.w);
       *reinterpret_cast<uint2*>(P.out + t * P.d + col0) = o0;
       *reinterpret_cast<uint2*>(P.out + t * P.d + col1) = o1;
     }
@@ -264,6 +223,58 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
   const int64_t blocks = (P.T + 7) / 8;
   const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
   combine_kernel<<<grid, 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+// S3, second half: the pull gather.  Each expert row (one warp) fetches the MX codes and
+// scales of its token by index from the per-token quantised copy (x quantised once per
+// token, small enough to stay in L2) and writes them to its padded position: codes with
+// 16-byte copies, scales re-laid into the UMMA layout one 4-byte K-group word at a time.
+__global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_mt[kMaxE + 1];
+  for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
+    s_off[i] = P.offsets[i];
+    s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t A = P.T * P.k;
+  const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
+  const int d = P.d;
+  const int64_t kg = d >> 7;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); q < A;
+       q += warps) {
+    int lo = 0, hi = P.E;  // s_off[lo] <= q < s_off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_off[mid] <= q) lo = mid; else hi = mid;
+    }
+    const int a = P.perm[q];
+    const int64_t t = a / P.k;
+    const int64_t p = static_cast<int64_t>(s_mt[lo]) * 128 + (q - s_off[lo]);
+    if (a < 0 || t >= P.T || p >= R) {
+      if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * d);
+    uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * d);
+    const int n16 = d >> 4;
+#pragma unroll 4
+    for (int i = lane; i < n16; i += 32) dst[i] = src[i];
+    const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
+    for (int g = lane; g < kg; g += 32)
+      *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
+  }
+}
+
+cudaError_t launch_gather_rows(const GatherParams& P, int num_sms, cudaStream_t stream) {
+  const int64_t A = P.T * P.k;
+  if (A <= 0) return cudaSuccess;
+  const int64_t blocks = (A + 7) / 8;
+  const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
+  gather_rows_kernel<<<grid, 256, 0, stream>>>(P);
   return cudaGetLastError();
 }
 
