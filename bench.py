@@ -33,6 +33,11 @@ METRIC = "MoE-layer fwd/bwd tokens/s at 1 B200; % of MXFP8 tensor peak and HBM B
 CONFIG_NAME = "dsv3"
 
 
+# Pure-write HBM stream (torch fill_ of 4 GiB, CUDA events) measured on this machine's B200s:
+# the ceiling of an output-dominated kernel such as the weight-gradient GEMM.
+WRITE_ONLY_GBS = 3911.0
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -357,6 +362,12 @@ def run_ours(args, case):
         # G fp32 + saved g|u bf16 + h MX read, dg|du MX written, per assignment row
         "bwd_swiglu": A * case.f * (4 + 4 + 1 + 2) * (1 + 1 / 64),
     }
+    if bwd:
+        # rows inside some expert segment (the transposes and the wgrad K ranges cover these)
+        r_used = int(saved["pad_offsets"][case.E].item())
+        cols = 2 * case.d + 3 * case.f      # x^, w*dout^ (d), h^ (f), [dg|du]^ (2f)
+        alg_bytes["bwd_transpose"] = 2 * r_used * cols * (1 + 1 / 32)
+        alg_bytes["bwd_wgrad"] = 2 * case.E * 3 * case.d * case.f + r_used * cols * (1 + 1 / 32)
     stage_info = {}
     for name, (tot_ms, n) in stages.items():
         s = {"ms_per_launch": tot_ms / max(n, 1), "launches": n}
@@ -370,11 +381,29 @@ def run_ours(args, case):
             s["frac_mxfp8"] = s["tflops"] / mx_peak
         stage_info[name] = s
     g = stage_info.get("gateup", {"ms_per_launch": float("nan"), "tflops": float("nan")})
-    traffic = None
+    tr = {}
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as fh:
-            traffic = json.load(fh).get("gateup_bytes_per_launch")
+            tr = json.load(fh)
+    roof_gateup = {"bound": "tensor", "kernel": "grouped_gemm_kernel<GATEUP_SWIGLU>",
+                   "achieved": g["tflops"], "peak": mx_peak, "unit": "TFLOP/s",
+                   "frac": g["tflops"] / mx_peak,
+                   "traffic": tr.get("gateup_bytes_per_launch") if case.name == "dsv3" else None,
+                   "peak_note": f"2 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
+                                f"MXFP8:bf16 nominal ratio 2"}
+    roofline = roof_gateup
+    if bwd and "bwd_wgrad" in stage_info:
+        # the dominant kernel of a forward+backward step: the weight-gradient GEMM, whose
+        # bf16 output (22.5 GB at this shape) makes it an HBM-write-bound launch pair
+        w = stage_info["bwd_wgrad"]
+        roofline = {"bound": "hbm", "kernel": "grouped_gemm_kernel<WGRAD_BF16> (2 launches)",
+                    "achieved": w["gbs"], "peak": peaks["hbm"], "unit": "GB/s",
+                    "frac": w["gbs"] / peaks["hbm"],
+                    "traffic": tr.get("wgrad_bytes_per_stage") if case.name == "dsv3" else None,
+                    "peak_note": f"{peaks['src']} copy bandwidth (read+write); pure-write "
+                                 f"streams on this pool measured {WRITE_ONLY_GBS:.0f} GB/s",
+                    "frac_of_write_only": w["gbs"] / WRITE_ONLY_GBS}
     ms_step = ms / args.steps
     value = world * case.T * args.steps / (ms * 1e-3)
     fwd_ms = sum(v["ms_per_launch"] for k, v in stage_info.items() if not k.startswith("bwd"))
@@ -391,11 +420,8 @@ def run_ours(args, case):
                    "d": case.d, "f": case.f, "E": case.E, "k": case.k,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "no flush: every step streams 11.6 GB of MXFP8 weights (> 126 MB L2)"},
-        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<GATEUP_SWIGLU>",
-                     "achieved": g["tflops"], "peak": mx_peak, "unit": "TFLOP/s",
-                     "frac": g["tflops"] / mx_peak, "traffic": traffic,
-                     "peak_note": f"2 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
-                                  f"MXFP8:bf16 nominal ratio 2"},
+        "roofline": roofline,
+        "roofline_gateup": roof_gateup,
         "fwd_tokens_per_s": world * case.T / (fwd_ms * 1e-3),
         "bwd_tokens_per_s": world * case.T / (bwd_ms * 1e-3) if bwd else None,
         "layer_tflops": layer_flops / (ms_step * 1e-3) / 1e12,

@@ -72,7 +72,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D byte matrix [rows, cols] (cols contiguous), box [box_rows, 128 bytes], 128-byte swizzle.
-moe_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+moe_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
+                     bool swizzle = true) {
   auto fn = encode_fn();
   if (!fn) return MOE_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -80,7 +81,8 @@ moe_status make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t col
   cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -796,32 +798,23 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     P.E = E;
     P.R = R;
     P.status = status;
-    P.src = TSRC_MX;  // x^ (forward codes) -> X~^T [d, R]
-    P.q = S->xq;
-    P.s = S->xs;
-    P.C = d;
-    P.dst_q = xt_q;
-    P.dst_s = xt_s;
-    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
-    P.q = S->hq;      // h^ -> H~^T [f, R]
-    P.s = S->hs;
-    P.C = f;
-    P.dst_q = ht_q;
-    P.dst_s = ht_s;
-    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
-    P.q = dgu_q;      // [dg|du]^ -> DGU~^T [2f, R]
-    P.s = dgu_s;
-    P.C = 2 * f;
-    P.dst_q = gt_q;
-    P.dst_s = gt_s;
-    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
-    P.src = TSRC_MX_W;  // w * dout^ -> DY~^T [d, R]
-    P.q = dq;
-    P.s = dsc;
-    P.C = d;
-    P.dst_q = yt_q;
-    P.dst_s = yt_s;
-    MOE_TRY(cuda_ok(launch_transpose_quant(P, st)));
+    auto run = [&](int src, const uint8_t* q, const uint8_t* s, int C, uint8_t* dq_out,
+                   uint8_t* ds_out) -> moe_status {
+      P.src = src;
+      P.q = q;
+      P.s = s;
+      P.C = C;
+      P.dst_q = dq_out;
+      P.dst_s = ds_out;
+      CUtensorMap tsrc, tdst;
+      MOE_TRY(make_tmap(&tsrc, q, R, C, 128, false));
+      MOE_TRY(make_tmap(&tdst, dq_out, C, R, 128, true));
+      return cuda_ok(launch_transpose_quant(tsrc, tdst, P, sms, st));
+    };
+    MOE_TRY(run(TSRC_MX, S->xq, S->xs, d, xt_q, xt_s));         // x^ -> X~^T [d, R]
+    MOE_TRY(run(TSRC_MX, S->hq, S->hs, f, ht_q, ht_s));         // h^ -> H~^T [f, R]
+    MOE_TRY(run(TSRC_MX, dgu_q, dgu_s, 2 * f, gt_q, gt_s));     // [dg|du]^ -> DGU~^T [2f, R]
+    MOE_TRY(run(TSRC_MX_W, dq, dsc, d, yt_q, yt_s));            // w * dout^ -> DY~^T [d, R]
   } else {
     // no tokens: every expert's K range is empty; the prefix below is all zeros
   }

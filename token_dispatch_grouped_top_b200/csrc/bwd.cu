@@ -11,8 +11,10 @@
 // boundaries, so a block never straddles two experts; rows past the segment's count are
 // zeros).  The result is stored transposed ([C, R], K-major for the GEMM).
 //
-// Shared-memory staged: see transpose_quant_kernel.  C % 128 == 0 (d, f, 2f all are).
+// TMA-staged 128 x 128 tiles: see transpose_quant_kernel.  C % 128 == 0 (d, f, 2f all are).
 #include <cuda_fp16.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -31,91 +33,172 @@ __device__ __forceinline__ float e8m0_to_f32_t(uint32_t b) {
 }
 
 constexpr int kTqThreads = 256;
-constexpr int kTqRows = 128;     // rows (tokens) per block: four 32-row quantisation blocks
-constexpr int kTqCols = 128;     // columns per block
-constexpr int kTqPitch = kTqCols + 16;
+constexpr int kTqCtasPerSm = 3;
+constexpr uint32_t kTqTile = 128 * 128;  // bytes of codes per 128 x 128 tile
 constexpr int kTqMaxE = 1024;
 
-// Block = 128 rows x 128 columns.  Codes are staged in shared memory with coalesced
-// 16-byte loads (8 threads per 128-byte row) and each row's four scales of these columns
-// arrive as one 32-bit word; then thread (column c, half hb) walks down column c for two
-// 32-row blocks, dequantises (times the row's combine weight for w * dout^), requantises
-// along the rows and writes 32 bytes of the transposed output.
-__global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(TransposeQuantParams P) {
-  __shared__ __align__(16) uint8_t s_codes[kTqRows][kTqPitch];
-  __shared__ float s_mul[kTqCols / 32][kTqRows];  // 2^s of (row, 32-column block) x weight
-  __shared__ int s_pad[kTqMaxE + 1];
-  const int64_t p0 = static_cast<int64_t>(blockIdx.y) * kTqRows;  // first row of the block
-  const int c0 = blockIdx.x * kTqCols;                              // first column
-  const int tid = threadIdx.x;
-  for (int i = tid; i <= P.E; i += kTqThreads) s_pad[i] = P.pad_offsets[i];
-  __syncthreads();
-  // expert of the 128-row block (segments start on 128-row boundaries) and valid rows
-  int lo = 0, hi = P.E;  // s_pad[lo] <= p0 < s_pad[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (s_pad[mid] <= p0) lo = mid; else hi = mid;
-  }
-  const int64_t rel = p0 - s_pad[lo];
-  int nv_blk = static_cast<int>(P.counts[lo] - rel);
-  if (p0 >= s_pad[P.E]) nv_blk = 0;
-  nv_blk = nv_blk < 0 ? 0 : (nv_blk > kTqRows ? kTqRows : nv_blk);
-  if (tid < kTqRows) {
-    float w = 0.f;
-    uint32_t sw = 0;
-    if (tid < nv_blk) {
-      w = P.src == TSRC_MX_W ? P.topk_w[P.perm[P.offsets[lo] + rel + tid]] : 1.f;
-      sw = *reinterpret_cast<const uint32_t*>(P.s + umma_scale_offset(p0 + tid, c0 >> 5,
-                                                                       P.C >> 7));
-    }
-#pragma unroll
-    for (int cb = 0; cb < kTqCols / 32; ++cb)
-      s_mul[cb][tid] = e8m0_to_f32_t((sw >> (8 * cb)) & 0xFFu) * w;
-  }
-  // codes: 128 rows x 128 bytes, 8 threads per row, 16 bytes each
-#pragma unroll
-  for (int it = 0; it < (kTqRows * kTqCols / 16) / kTqThreads; ++it) {
-    const int idx = it * kTqThreads + tid;
-    const int r = idx >> 3, ch = idx & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < nv_blk)
-      v = *reinterpret_cast<const uint4*>(P.q + (p0 + r) * P.C + c0 + ch * 16);
-    *reinterpret_cast<uint4*>(&s_codes[r][ch * 16]) = v;
-  }
-  __syncthreads();
-  const int c = tid & (kTqCols - 1);  // column within the block
-  const int hb = tid >> 7;            // 32-row blocks hb and hb + 2
-  const float* mul = s_mul[c >> 5];
-#pragma unroll 1
-  for (int bb = 0; bb < 2; ++bb) {
-    const int b = hb + 2 * bb;
-    float v[32];
-#pragma unroll
-    for (int r = 0; r < 32; r += 2) {  // rows r, r+1: one hardware E4M3x2 -> f16x2 decode
-      const int rr = 32 * b + r;
-      const uint32_t pair = static_cast<uint32_t>(s_codes[rr][c]) |
-                            (static_cast<uint32_t>(s_codes[rr + 1][c]) << 8);
-      uint32_t h2;
-      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
-      // rows past the segment's count have multiplier 0 (and zero codes)
-      v[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu))) * mul[rr];
-      v[r + 1] =
-          __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16))) * mul[rr + 1];
-    }
-    uint32_t qw[8];
-    const uint32_t sb = mx_quant_block32(v, qw);
-    const int64_t pb = p0 + 32 * b;
-    uint4* dst = reinterpret_cast<uint4*>(P.dst_q + static_cast<int64_t>(c0 + c) * P.R + pb);
-    dst[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
-    dst[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
-    P.dst_s[umma_scale_offset(c0 + c, pb >> 5, P.R >> 7)] = static_cast<uint8_t>(sb);
-  }
+// Per-CTA shared memory: two tiles in flight each way.
+struct TqSmem {
+  uint8_t in[2][kTqTile];    // source codes, 128-byte rows (TMA, no swizzle)
+  uint8_t out[2][kTqTile];   // transposed codes, 128-byte swizzle (TMA store layout)
+  uint8_t sin[2][512];       // the source's UMMA scale chunk of the tile
+  uint8_t sout[2][512];      // the output's UMMA scale chunk of the tile
+  float mul[4][128];         // 2^s(row, 32-column block) x weight of the row
+  uint64_t full[2];
+  int abort_flag;
+  int pad[kTqMaxE + 1];
+};
+constexpr size_t kTqSmemBytes = sizeof(TqSmem) + 1024;
+
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_src), "r"(bytes)
+               : "memory");
 }
 
-cudaError_t launch_transpose_quant(const TransposeQuantParams& P, cudaStream_t stream) {
+// One thread: column c of the tile, 32-row block b: decode 32 codes down the column,
+// scale them (rows at or past `lim` are zero), requantise along the rows, write the
+// 32 output bytes into row c of the swizzled output tile and the scale byte into the
+// output chunk.
+template <bool kRagged>
+__device__ __forceinline__ void tq_column_block(const uint8_t* col, const float* mul, int b,
+                                                int lim, uint8_t* orow, int c, uint8_t* sout) {
+  float v[32];
+#pragma unroll
+  for (int r = 0; r < 32; r += 2) {  // rows r, r+1: one hardware E4M3x2 -> f16x2 decode
+    const int rr = 32 * b + r;
+    const uint32_t pair = static_cast<uint32_t>(col[rr * 128]) |
+                          (static_cast<uint32_t>(col[(rr + 1) * 128]) << 8);
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
+    v[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu))) * mul[rr];
+    v[r + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16))) * mul[rr + 1];
+    if (kRagged) {
+      if (r >= lim) v[r] = 0.f;
+      if (r + 1 >= lim) v[r + 1] = 0.f;
+    }
+  }
+  uint32_t qw[8];
+  const uint32_t sb = mx_quant_block32(v, qw);
+  *reinterpret_cast<uint4*>(orow + (((2 * b) ^ (c & 7)) << 4)) =
+      make_uint4(qw[0], qw[1], qw[2], qw[3]);
+  *reinterpret_cast<uint4*>(orow + (((2 * b + 1) ^ (c & 7)) << 4)) =
+      make_uint4(qw[4], qw[5], qw[6], qw[7]);
+  sout[(c & 31) * 16 + (c >> 5) * 4 + b] = static_cast<uint8_t>(sb);
+}
+
+// Persistent: each CTA walks 128 x 128 tiles (column block fastest) of the rows that
+// belong to some expert segment (rows [0, pad_offsets[E]); the rest of the R-row buffer is
+// never read by the weight-gradient GEMM).  Thread 0 keeps the next tile's codes (TMA,
+// 16 KB) and scale chunk (512 B) in flight while all threads work on the current one;
+// the transposed tile and its scale chunk leave through TMA / bulk stores, so global
+// memory sees whole 128-byte lines both ways.  Thread (c, h) handles column c for the
+// 32-row blocks h and h + 2.
+__global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(
+    const __grid_constant__ CUtensorMap tm_src, const __grid_constant__ CUtensorMap tm_dst,
+    const TransposeQuantParams P) {
+  extern __shared__ uint8_t tq_raw[];
+  const uint32_t raw_addr = smem_u32(tq_raw);
+  TqSmem& S = *reinterpret_cast<TqSmem*>(tq_raw + ((1024u - (raw_addr & 1023u)) & 1023u));
+  const int tid = threadIdx.x;
+  for (int i = tid; i <= P.E; i += kTqThreads) S.pad[i] = P.pad_offsets[i];
+  if (tid == 0) {
+    mbar_init(smem_u32(&S.full[0]), 1);
+    mbar_init(smem_u32(&S.full[1]), 1);
+    S.abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tm_src);
+    prefetch_tmap(&tm_dst);
+  }
+  __syncthreads();
+  const int ncb = P.C >> 7;
+  const int ntiles = (S.pad[P.E] >> 7) * ncb;
+  const int64_t kg_src = P.C >> 7, kg_dst = P.R >> 7;
+  auto issue = [&](int tile, int buf) {
+    const int rb = tile / ncb, cb = tile - rb * ncb;
+    const uint32_t fb = smem_u32(&S.full[buf]);
+    mbar_arrive_expect_tx(fb, kTqTile + 512);
+    tma_load_2d(smem_u32(S.in[buf]), &tm_src, fb, cb * 128, rb * 128);
+    bulk_load(smem_u32(S.sin[buf]), P.s + ((static_cast<int64_t>(rb) * kg_src + cb) << 9), 512,
+              fb);
+  };
+  if (tid == 0 && static_cast<int>(blockIdx.x) < ntiles) issue(blockIdx.x, 0);
+  const int c = tid & 127, hb = tid >> 7;
+  int it = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int buf = it & 1;
+    if (tid == 0) {
+      const int next = tile + gridDim.x;
+      if (next < ntiles) issue(next, buf ^ 1);  // buf ^ 1 was released at the last barrier
+      bulk_wait_read<1>();  // the stores issued from out[buf] two tiles ago have read it
+    }
+    const int rb = tile / ncb, cb = tile - rb * ncb;
+    const int64_t p0 = static_cast<int64_t>(rb) * 128;
+    int lo = 0, hi = P.E;  // pad[lo] <= p0 < pad[hi]: the expert owning these rows
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (S.pad[mid] <= p0) lo = mid; else hi = mid;
+    }
+    const int64_t rel = p0 - S.pad[lo];
+    int nv = static_cast<int>(P.counts[lo] - rel);
+    nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
+    float w = 0.f;
+    if (tid < 128 && tid < nv)
+      w = P.src == TSRC_MX_W ? P.topk_w[P.perm[P.offsets[lo] + rel + tid]] : 1.f;
+    const bool ok = mbar_wait(smem_u32(&S.full[buf]), (it >> 1) & 1, &S.abort_flag, P.status);
+    if (tid < 128) {
+      const uint32_t sw = *reinterpret_cast<const uint32_t*>(S.sin[buf] + (tid & 31) * 16 +
+                                                             (tid >> 5) * 4);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t e = (sw >> (8 * q)) & 0xFFu;
+        S.mul[q][tid] = tid < nv ? e8m0_to_f32_t(e) * w : 0.f;
+      }
+    }
+    if (__syncthreads_or(!ok)) break;
+    const uint8_t* col = S.in[buf] + c;
+    const float* mul = S.mul[c >> 5];
+    uint8_t* orow = S.out[buf] + c * 128;
+#pragma unroll 1
+    for (int bb = 0; bb < 2; ++bb) {
+      const int b = hb + 2 * bb;
+      const int lim = nv - 32 * b;
+      if (lim >= 32)
+        tq_column_block<false>(col, mul, b, lim, orow, c, S.sout[buf]);
+      else
+        tq_column_block<true>(col, mul, b, lim, orow, c, S.sout[buf]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tma_store_2d(&tm_dst, smem_u32(S.out[buf]), static_cast<int32_t>(p0), cb * 128);
+      bulk_store(P.dst_s + ((static_cast<int64_t>(cb) * kg_dst + rb) << 9), smem_u32(S.sout[buf]),
+                 512);
+      bulk_commit();
+    }
+  }
+  if (tid == 0) bulk_wait_all();
+}
+
+cudaError_t launch_transpose_quant(const CUtensorMap& tm_src, const CUtensorMap& tm_dst,
+                                   const TransposeQuantParams& P, int num_sms,
+                                   cudaStream_t stream) {
   if (P.R <= 0 || P.C <= 0) return cudaSuccess;
-  dim3 grid(P.C / kTqCols, static_cast<unsigned>(P.R / kTqRows));
-  transpose_quant_kernel<<<grid, kTqThreads, 0, stream>>>(P);
+  if (P.E > kTqMaxE) return cudaErrorInvalidValue;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64 || !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(transpose_quant_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(kTqSmemBytes));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const int64_t max_tiles = (P.R / 128) * (P.C / 128);
+  const int64_t grid = std::min<int64_t>(max_tiles, static_cast<int64_t>(num_sms) * kTqCtasPerSm);
+  transpose_quant_kernel<<<static_cast<unsigned>(grid), kTqThreads, kTqSmemBytes, stream>>>(
+      tm_src, tm_dst, P);
   return cudaGetLastError();
 }
 

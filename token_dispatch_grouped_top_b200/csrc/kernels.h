@@ -96,15 +96,16 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
 // Token-direction quantiser for the weight gradients: a [R, C] operand in the padded
 // expert-contiguous row order is quantised along its rows (tokens) in blocks of 32 inside
 // each expert segment (rows past the segment's count read as zero) and stored transposed,
-// [C, R] E4M3 with the UMMA scales of the [C, R] matrix.
+// [C, R] E4M3 with the UMMA scales of the [C, R] matrix.  Only columns [0, pad_offsets[E])
+// of the output are written: no expert's K range reaches past them.
 enum TransposeSrc : int {
   TSRC_MX = 0,       // MX codes [R, C] + UMMA scales (kgroups C/128): dequantised exactly
   TSRC_MX_W = 1,     // the same, each row times the combine weight of its assignment
 };
 struct TransposeQuantParams {
   int src;
-  const uint8_t* q;
-  const uint8_t* s;
+  const uint8_t* q;            // [R, C] codes (read through tm_src: 128 x 128 box, no swizzle)
+  const uint8_t* s;            // their UMMA scales
   const int32_t* perm;
   const int32_t* offsets;
   const float* topk_w;
@@ -114,11 +115,13 @@ struct TransposeQuantParams {
   int E;
   int64_t R;
   int C;
-  uint8_t* dst_q;
+  uint8_t* dst_q;              // [C, R] (written through tm_dst: 128 x 128 box, 128B swizzle)
   uint8_t* dst_s;
   int32_t* status;
 };
-cudaError_t launch_transpose_quant(const TransposeQuantParams& P, cudaStream_t stream);
+cudaError_t launch_transpose_quant(const CUtensorMap& tm_src, const CUtensorMap& tm_dst,
+                                   const TransposeQuantParams& P, int num_sms,
+                                   cudaStream_t stream);
 
 // SwiGLU backward + d(router weights) per assignment row, from G = dout^ . Wd'^T.
 struct SwigluBwdParams {
