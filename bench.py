@@ -33,9 +33,10 @@ METRIC = "MoE-layer fwd/bwd tokens/s at 1 B200; % of MXFP8 tensor peak and HBM B
 CONFIG_NAME = "dsv3"
 
 
-# Pure-write HBM stream (torch fill_ of 4 GiB, CUDA events) measured on this machine's B200s:
-# the ceiling of an output-dominated kernel such as the weight-gradient GEMM.
-WRITE_ONLY_GBS = 3911.0
+# Pure-write HBM stream measured on this machine's B200s with TMA stores of 32-row x 128-byte
+# boxes into a 4 GiB [rows, 4096-byte] matrix (the weight-gradient epilogue's pattern; plain
+# coalesced 16-byte stores reach ~6300 GB/s): the ceiling of an output-dominated kernel.
+WRITE_ONLY_GBS = 5959.0
 
 
 def _peaks():
