@@ -535,8 +535,6 @@ moe_status moe_grouped_gemm_mx(int32_t G, int64_t rows_a, int32_t N, int32_t K,
   P.rows_valid = rows_valid;
   P.sfa = a_s;
   P.sfb = b_s;
-  P.out_f32 = d_out;
-  P.ld_out = N;
   P.status = at<int32_t>(ws, 0);
   CUtensorMap tc;
   MOE_TRY(make_out_tmap(&tc, d_out, rows_a, N, false));
@@ -632,8 +630,6 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.rows_valid = counts;
     P.sfa = hs;
     P.sfb = W->wd_s;
-    P.out_f32 = y;
-    P.ld_out = D->d;
     P.status = status;
     CUtensorMap ty;
     MOE_TRY(make_out_tmap(&ty, y, R, D->d, false));
@@ -714,8 +710,6 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.rows_valid = S->counts;
       P.sfa = dsc;
       P.sfb = W->wdT_s;
-      P.out_f32 = gbuf;
-      P.ld_out = f;
       P.status = status;
       MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg, P, sms, st)));
     }
@@ -752,8 +746,6 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.rows_valid = S->counts;
       P.sfa = dgu_s;
       P.sfb = W->wguT_s;
-      P.out_f32 = dxa;
-      P.ld_out = d;
       P.status = status;
       CUtensorMap tx;
       MOE_TRY(make_out_tmap(&tx, dxa, R, d, false));

@@ -22,7 +22,6 @@
 // that a weight tile is read from HBM once and re-read by the neighbouring CTAs from L2.
 //
 // Modes (epilogues):
-//   STORE_F32      D in fp32 (per-thread row stores; the generic path).
 //   STORE_F32_TMA  D in fp32 through shared memory and TMA stores (the down projection
 //                  and both dgrad GEMMs of the backward).
 //   GATEUP_SWIGLU  h = silu(g) * u on paired gate/up columns, MXFP8 requantisation of h
@@ -436,16 +435,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         hdst[3] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
         *reinterpret_cast<uint16_t*>(P.hs + umma_scale_offset(row, fb >> 5, f >> 7)) =
             static_cast<uint16_t>(s0 | (s1 << 8));
-      } else {
-        float4* dst = reinterpret_cast<float4*>(P.out_f32 + row * P.ld_out +
-                                                static_cast<int64_t>(ti.j) * BN + 128 * h);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          dst[c] = make_float4(v0[4 * c], v0[4 * c + 1], v0[4 * c + 2], v0[4 * c + 3]);
-          dst[8 + c] = make_float4(v1[4 * c], v1[4 * c + 1], v1[4 * c + 2], v1[4 * c + 3]);
-          dst[16 + c] = make_float4(v2[4 * c], v2[4 * c + 1], v2[4 * c + 2], v2[4 * c + 3]);
-          dst[24 + c] = make_float4(v3[4 * c], v3[4 * c + 1], v3[4 * c + 2], v3[4 * c + 3]);
-        }
       }
     }
   }
@@ -483,8 +472,6 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensor
                                 const CUtensorMap& tmC0, const CUtensorMap& tmC1,
                                 const GemmParams& P, int num_sms, cudaStream_t stream) {
   switch (mode) {
-    case GEMM_STORE_F32:
-      return launch_mode<GEMM_STORE_F32>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_GATEUP_SWIGLU:
       return launch_mode<GEMM_GATEUP_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
     case GEMM_WGRAD_BF16:

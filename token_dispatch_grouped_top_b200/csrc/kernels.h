@@ -143,10 +143,10 @@ cudaError_t launch_swiglu_bwd(const SwigluBwdParams& P, int num_sms, cudaStream_
 
 // Grouped block-scaled GEMM.
 enum GemmMode : int {
-  GEMM_STORE_F32 = 0,      // D fp32 [rows, N] (down projection, dgrad of x, generic)
   GEMM_GATEUP_SWIGLU = 1,  // SwiGLU + MX requant of h, optional bf16 g/u save
   GEMM_WGRAD_BF16 = 3,     // variable K per group (the group's token segment), bf16 out
-  GEMM_STORE_F32_TMA = 4,  // as STORE_F32 through shared memory + TMA stores; writes whole
+  GEMM_STORE_F32_TMA = 4,  // D fp32 [rows, N] through shared memory + TMA stores (down
+                           // projection, both dgrads, the generic entry point); writes whole
                            // 128-row tiles (rows past a group's count get unused values)
 };
 
@@ -161,8 +161,6 @@ struct GemmParams {
   const int32_t* rows_valid;    // [G] nullable
   const uint8_t* sfa;    // UMMA scales of A
   const uint8_t* sfb;    // UMMA scales of B
-  float* out_f32;        // STORE_F32: [rows, N]
-  int64_t ld_out;
   uint8_t* hq;           // GATEUP: [rows, f]
   uint8_t* hs;           // GATEUP: UMMA scales of [rows, f]
   uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16 save of g | u
