@@ -502,18 +502,18 @@ def run_ours(args, case):
 
 
 def sweep(args):
-    """One JSON line per synthetic configuration (forward; backward for the backward config).
+    """One JSON line per synthetic configuration and pass (forward, forward+backward).
     Not the default line: a table for the design notes."""
     import subprocess as sp
-    for name in ("tiny", "mid", "dsv3", "imbalance", "dsv3_bwd"):
-        cmd = [sys.executable, os.path.abspath(__file__), "--config", name, "--steps",
-               str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline"]
-        if name == "dsv3_bwd":
-            cmd += ["--pass", "fwdbwd"]
-        r = sp.run(cmd, capture_output=True, text=True)
-        line = r.stdout.strip().splitlines()[-1] if r.stdout.strip() else json.dumps(
-            {"config": name, "error": r.stderr[-500:]})
-        print(line, flush=True)
+    for name in ("tiny", "mid", "dsv3", "imbalance"):
+        for pass_ in ("fwd", "fwdbwd"):
+            cmd = [sys.executable, os.path.abspath(__file__), "--config", name, "--steps",
+                   str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline",
+                   "--pass", pass_]
+            r = sp.run(cmd, capture_output=True, text=True)
+            line = r.stdout.strip().splitlines()[-1] if r.stdout.strip() else json.dumps(
+                {"config": name, "pass": pass_, "error": r.stderr[-500:]})
+            print(line, flush=True)
 
 
 def main():

@@ -8,7 +8,8 @@
 //
 // Problem: for group g (an expert) with rows [128*prefix[g], 128*prefix[g+1]) of A,
 //   D[r, n] = sum_k A[r, k] * B[g*N + n, k]      (A, B K-major E4M3, UMMA scales)
-// Tile 128 x 256 x 128 (rows x cols x K per stage), 4-stage TMA pipeline.
+// Tile 128 x 256 x 128 (rows x cols x K per stage), 4-stage TMA pipeline (3 stages in the
+// TMA-store modes, whose output staging buffers take 64 KB of shared memory).
 //
 // Warp roles (320 threads, one CTA per SM, persistent over a static round-robin tile list
 // that is derived on the device from the per-expert tile prefix -- no host round trip):
