@@ -72,6 +72,7 @@ struct GemmSmemT {
   uint64_t empty[ST];
   uint64_t tmem_full;
   uint64_t tmem_empty;
+  uint64_t tmem_empty_hi;  // WGRAD: columns 128..255 drained (tmem_empty: 0..127)
   uint32_t tmem_base;
   int abort_flag;
   int prefix[kMaxG + 1];
@@ -183,6 +184,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(smem_u32(&S.tmem_full), 1);
     mbar_init(smem_u32(&S.tmem_empty), kEpiWarps);
+    mbar_init(smem_u32(&S.tmem_empty_hi), kEpiWarps);
     S.abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmA);
@@ -239,42 +241,87 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(smem_u32(&S.tmem_empty), acc_phase ^ 1u, abort_flag, P.status)) break;
         tc_fence_after();
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(&S.full[stage]), phase, abort_flag, P.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sf = tbase + kSfCol + 16u * stage;
-          tmem_cp_scales(sf, sdesc_scale_chunk(smem_u32(S.sfa[stage])));
-          tmem_cp_scales(sf + 4, sdesc_scale_chunk(smem_u32(S.sfb[stage])));
-          tmem_cp_scales(sf + 8, sdesc_scale_chunk(smem_u32(S.sfb[stage]) + 512));
-          const uint32_t a0 = smem_u32(S.a[stage]), b0 = smem_u32(S.b[stage]);
-          if (swapped) {
-            // D0[w, t] = sum_k B[w, k] A[t, k] for weight rows w < 128, D1 for rows 128..255
-#pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk) {
-              const uint32_t id = idesc_sw | (static_cast<uint32_t>(kk) << 29) |
-                                  (static_cast<uint32_t>(kk) << 4);
-              const uint64_t bt = sdesc_k_sw128(a0 + 32u * kk);
-              mma_mxf8(tbase + kAccCol, sdesc_k_sw128(b0 + 32u * kk), bt, id,
-                       (kb | kk) != 0 ? 1u : 0u, sf + 4, sf);
-              mma_mxf8(tbase + kAccCol + 128, sdesc_k_sw128(b0 + 128u * 128u + 32u * kk), bt, id,
-                       (kb | kk) != 0 ? 1u : 0u, sf + 8, sf);
+        if (MODE == GEMM_WGRAD_BF16) {
+          // Two N = 128 MMAs per K step, columns 0..127 first: the epilogue releases that
+          // half before it drains columns 128..255, so the next tile starts earlier.
+          const uint32_t idesc_h = idesc_mxf8_e4m3(BM, BN / 2);
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait(smem_u32(&S.full[stage]), phase, abort_flag, P.status)) {
+              ok = false;
+              break;
             }
-          } else {
+            tc_fence_after();
+            const uint32_t sf = tbase + kSfCol + 16u * stage;
+            tmem_cp_scales(sf, sdesc_scale_chunk(smem_u32(S.sfa[stage])));
+            tmem_cp_scales(sf + 4, sdesc_scale_chunk(smem_u32(S.sfb[stage])));
+            tmem_cp_scales(sf + 8, sdesc_scale_chunk(smem_u32(S.sfb[stage]) + 512));
+            const uint32_t a0 = smem_u32(S.a[stage]), b0 = smem_u32(S.b[stage]);
 #pragma unroll
             for (int kk = 0; kk < BK / 32; ++kk) {
-              const uint32_t id = idesc | (static_cast<uint32_t>(kk) << 29) |
+              const uint32_t id = idesc_h | (static_cast<uint32_t>(kk) << 29) |
                                   (static_cast<uint32_t>(kk) << 4);
               mma_mxf8(tbase + kAccCol, sdesc_k_sw128(a0 + 32u * kk),
                        sdesc_k_sw128(b0 + 32u * kk), id, (kb | kk) != 0 ? 1u : 0u, sf, sf + 4);
             }
+            if (kb == 0) {
+              if (!mbar_wait(smem_u32(&S.tmem_empty_hi), acc_phase ^ 1u, abort_flag, P.status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk) {
+              const uint32_t id = idesc_h | (static_cast<uint32_t>(kk) << 29) |
+                                  (static_cast<uint32_t>(kk) << 4);
+              mma_mxf8(tbase + kAccCol + BN / 2, sdesc_k_sw128(a0 + 32u * kk),
+                       sdesc_k_sw128(b0 + 128u * 128u + 32u * kk), id, (kb | kk) != 0 ? 1u : 0u,
+                       sf, sf + 8);
+            }
+            mma_commit(smem_u32(&S.empty[stage]));
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          mma_commit(smem_u32(&S.empty[stage]));
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+        } else {
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait(smem_u32(&S.full[stage]), phase, abort_flag, P.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sf = tbase + kSfCol + 16u * stage;
+            tmem_cp_scales(sf, sdesc_scale_chunk(smem_u32(S.sfa[stage])));
+            tmem_cp_scales(sf + 4, sdesc_scale_chunk(smem_u32(S.sfb[stage])));
+            tmem_cp_scales(sf + 8, sdesc_scale_chunk(smem_u32(S.sfb[stage]) + 512));
+            const uint32_t a0 = smem_u32(S.a[stage]), b0 = smem_u32(S.b[stage]);
+            if (swapped) {
+              // D0[w, t] = sum_k B[w, k] A[t, k] for weight rows w < 128, D1 for rows 128..255
+#pragma unroll
+              for (int kk = 0; kk < BK / 32; ++kk) {
+                const uint32_t id = idesc_sw | (static_cast<uint32_t>(kk) << 29) |
+                                    (static_cast<uint32_t>(kk) << 4);
+                const uint64_t bt = sdesc_k_sw128(a0 + 32u * kk);
+                mma_mxf8(tbase + kAccCol, sdesc_k_sw128(b0 + 32u * kk), bt, id,
+                         (kb | kk) != 0 ? 1u : 0u, sf + 4, sf);
+                mma_mxf8(tbase + kAccCol + 128, sdesc_k_sw128(b0 + 128u * 128u + 32u * kk), bt, id,
+                         (kb | kk) != 0 ? 1u : 0u, sf + 8, sf);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < BK / 32; ++kk) {
+                const uint32_t id = idesc | (static_cast<uint32_t>(kk) << 29) |
+                                    (static_cast<uint32_t>(kk) << 4);
+                mma_mxf8(tbase + kAccCol, sdesc_k_sw128(a0 + 32u * kk),
+                         sdesc_k_sw128(b0 + 32u * kk), id, (kb | kk) != 0 ? 1u : 0u, sf, sf + 4);
+              }
+            }
+            mma_commit(smem_u32(&S.empty[stage]));
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
         if (!ok) break;
@@ -305,6 +352,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait(smem_u32(&S.tmem_full), acc_phase, abort_flag, P.status)) break;
       tc_fence_after();
       const uint32_t taddr = tbase + kAccCol + (static_cast<uint32_t>(32 * q) << 16);
+      if (MODE == GEMM_WGRAD_BF16) {
+        // columns 64h..64h+63 of each 128-column half; the lower half is released first
+        float v0[32], v1[32], v2[32], v3[32];
+        tmem_ld32(taddr + 64 * h, v0);
+        tmem_ld32(taddr + 64 * h + 32, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S.tmem_empty));
+        tmem_ld32(taddr + 128 + 64 * h, v2);
+        tmem_ld32(taddr + 128 + 64 * h + 32, v3);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S.tmem_empty_hi));
+        acc_phase ^= 1u;
+        const int32_t y = static_cast<int32_t>(ti.g * P.M + ti.a_row0 + 32 * q);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int n0 = ti.j * BN + 128 * half + 64 * h;  // 64 bf16 columns = one chunk
+          const bool first = n0 < P.split;
+          const float* va = half == 0 ? v0 : v2;
+          const float* vb = half == 0 ? v1 : v3;
+          uint4 r16[8];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            r16[c] = pack_bf16x8(va + 8 * c);
+            r16[4 + c] = pack_bf16x8(vb + 8 * c);
+          }
+          stage_and_store(S.stg[2 * (warp - 2) + stg_buf], r16, first ? &tmC0 : &tmC1,
+                          first ? n0 : n0 - P.split, y, lane);
+          stg_buf ^= 1;
+        }
+        continue;
+      }
       if (ModeCfg<MODE>::kSwapTail && ti.rows < BM) {
         // transposed accumulators: lane = weight row (feature), column = token
         const int tok0 = 64 * h;
@@ -363,30 +445,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       acc_phase ^= 1u;
 
       const int m = 32 * q + lane;
-      if (MODE == GEMM_WGRAD_BF16) {
-        // bf16 rows of 128 columns: two 64-column chunks through the staging buffers
-        const int n0 = ti.j * BN + 128 * h;
-        const bool first = n0 < P.split;
-        const CUtensorMap* tm = first ? &tmC0 : &tmC1;
-        const int x0 = first ? n0 : n0 - P.split;
-        const int32_t y = static_cast<int32_t>(ti.g * P.M + ti.a_row0 + 32 * q);
-        uint4 r16[8];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          r16[c] = pack_bf16x8(v0 + 8 * c);
-          r16[4 + c] = pack_bf16x8(v1 + 8 * c);
-        }
-        stage_and_store(S.stg[2 * (warp - 2) + stg_buf], r16, tm, x0, y, lane);
-        stg_buf ^= 1;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          r16[c] = pack_bf16x8(v2 + 8 * c);
-          r16[4 + c] = pack_bf16x8(v3 + 8 * c);
-        }
-        stage_and_store(S.stg[2 * (warp - 2) + stg_buf], r16, tm, x0 + 64, y, lane);
-        stg_buf ^= 1;
-        continue;
-      }
       if (MODE == GEMM_STORE_F32_TMA) {
         // fp32 rows of 128 columns: four 32-column chunks; whole 32-row boxes are written
         const int32_t x0 = ti.j * BN + 128 * h;
