@@ -114,6 +114,22 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+def max_over_ranks(ms: float, device, world: int) -> float:
+    """The slowest rank's time: every rank contributes its own device-timed milliseconds
+    (one all-reduce MAX over the process group; a no-op on one rank)."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: the tokens every rank processed over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms * 1e-3)
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -327,10 +343,7 @@ def run_ours(args, case):
     moe.profile_enable(False)
     stages = moe.profile_collect()
     ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev, world)
     status = moe.device_status(ws) | (moe.device_status(wsb) if bwd else 0)
 
     # end to end through the public API with host buffers: every step copies its inputs
@@ -395,10 +408,7 @@ def run_ours(args, case):
     e1.record(stream)
     barrier()
     ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, dev, world)
 
     peaks = _peaks()
     A = case.T * case.k
@@ -462,7 +472,7 @@ def run_ours(args, case):
                                  f"streams on this pool measured {WRITE_ONLY_GBS:.0f} GB/s",
                     "frac_of_write_only": w["gbs"] / WRITE_ONLY_GBS}
     ms_step = ms / args.steps
-    value = world * case.T * args.steps / (ms * 1e-3)
+    value = job_tokens_per_s(world, case.T, args.steps, ms)
     fwd_ms = sum(v["ms_per_launch"] for k, v in stage_info.items() if not k.startswith("bwd"))
     bwd_ms = sum(v["ms_per_launch"] for k, v in stage_info.items() if k.startswith("bwd"))
     layer_flops = sum(fl[k] for k in fl if bwd or not k.startswith("bwd"))
@@ -487,7 +497,7 @@ def run_ours(args, case):
         "stages": stage_info,
         "gpu_launches": launches,
         "device_status": status,
-        "e2e": {"value": world * case.T * args.steps / (ms_e2e * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(world, case.T, args.steps, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
         "padded_rows": moe.padded_rows(dims),
