@@ -82,7 +82,9 @@ typedef struct {
   uint8_t *wguT_s;
 } moe_weights;
 
-/* Forward state kept for the backward pass (all device buffers, caller-owned). */
+/* Forward state kept for the backward pass (all device buffers, caller-owned).  With no
+ * tokens (T == 0) the token-sized arrays topk_idx, topk_w, perm and inv_perm hold nothing
+ * and may be NULL. */
 typedef struct {
   int32_t *topk_idx;     /* [T,k]  expert of assignment a                                */
   float   *topk_w;       /* [T,k]  combine weight                                       */

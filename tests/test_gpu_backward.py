@@ -106,3 +106,32 @@ def test_backward_mid_full(moe):
 def test_backward_dsv3_sampled(moe):
     case = synth.CONFIGS["dsv3_bwd"]
     _check(moe, case, tokens=np.array([1234]), experts=None)
+
+
+def test_backward_edge_cases(moe):
+    # E = 1 (dense layer), k = E with the sigmoid score, a single token
+    for case in [synth.MoeCase("b_e1", 130, 256, 256, 1, 1, 0, "none", seed=11),
+                 synth.MoeCase("b_kE", 77, 256, 256, 4, 4, 1, "normal0.5", seed=12),
+                 synth.MoeCase("b_t1", 1, 256, 512, 8, 2, 0, "none", seed=13)]:
+        _check(moe, case)
+
+
+def test_backward_no_tokens(moe):
+    # T = 0: nothing to route; every expert is empty and gets an all-zero weight gradient
+    import torch
+    case = synth.MoeCase("b_t0", 0, 256, 256, 4, 2, 0, "none", seed=14)
+    dims = moe.Dims(case.T, case.d, case.f, case.E, case.k, case.score_fn)
+    wg, wu, wd = synth.expert_weights_torch(case, "cuda")
+    pw = moe.prepare_weights(wg, wu, wd, dims, with_backward=True)
+    x = torch.empty((0, case.d), dtype=torch.bfloat16, device="cuda")
+    lg = torch.empty((0, case.E), dtype=torch.float32, device="cuda")
+    wsf = moe.workspace(dims, moe.OP_FORWARD)
+    out, saved = moe.forward(x, lg, pw, save=True, ws=wsf)
+    wsb = moe.workspace(dims, moe.OP_BACKWARD)
+    grads = moe.backward(torch.empty((0, case.d), dtype=torch.bfloat16, device="cuda"), pw,
+                         saved, ws=wsb)
+    torch.cuda.synchronize()
+    assert moe.device_status(wsf) == 0 and moe.device_status(wsb) == 0
+    assert tuple(out.shape) == (0, case.d) and tuple(grads["dx"].shape) == (0, case.d)
+    for name in ("dWg", "dWu", "dWd"):
+        assert not torch.any(grads[name].float() != 0), name

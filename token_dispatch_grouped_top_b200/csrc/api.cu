@@ -548,8 +548,10 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
   MOE_TRY(check_dims(D));
   if (!W || !ws || (D->T > 0 && (!x || !logits || !out))) return MOE_ERR_INVALID_ARG;
   if (!W->wgu_q || !W->wgu_s || !W->wd_q || !W->wd_s) return MOE_ERR_INVALID_ARG;
-  if (saved && (!saved->topk_idx || !saved->topk_w || !saved->counts || !saved->offsets ||
-                !saved->perm || !saved->inv_perm || !saved->pad_offsets || !saved->xq ||
+  // the token-sized arrays (T*k entries) may be null when there are no tokens
+  if (saved && ((D->T > 0 && (!saved->topk_idx || !saved->topk_w || !saved->perm ||
+                              !saved->inv_perm)) ||
+                !saved->counts || !saved->offsets || !saved->pad_offsets || !saved->xq ||
                 !saved->xs || !saved->hq || !saved->hs || !saved->gu))
     return MOE_ERR_INVALID_ARG;
   if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
@@ -662,8 +664,9 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
   MOE_TRY(check_dims(D));
   if (!W || !S || !ws || !dWg || !dWu || !dWd) return MOE_ERR_INVALID_ARG;
   if (!W->wdT_q || !W->wdT_s || !W->wguT_q || !W->wguT_s) return MOE_ERR_INVALID_ARG;
-  if (!S->topk_idx || !S->topk_w || !S->counts || !S->offsets || !S->perm || !S->inv_perm ||
-      !S->pad_offsets || !S->xq || !S->xs || !S->hq || !S->hs || !S->gu)
+  if ((D->T > 0 && (!S->topk_idx || !S->topk_w || !S->perm || !S->inv_perm)) ||
+      !S->counts || !S->offsets || !S->pad_offsets || !S->xq || !S->xs || !S->hq || !S->hs ||
+      !S->gu)
     return MOE_ERR_INVALID_ARG;
   if (D->T > 0 && (!dout || !dx || !dw_route)) return MOE_ERR_INVALID_ARG;
   if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
