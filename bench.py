@@ -130,6 +130,58 @@ def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, ms: float) ->
     return world * tokens_per_rank * steps / (ms * 1e-3)
 
 
+def layer_summary(case, stage_ms: dict, ms_step: float, peaks: dict, bwd: bool) -> dict:
+    """Whole-layer roofline of one step: algorithmic FLOPs and HBM bytes (MX bytes include
+    the 1/32 scale overhead; activations counted for the A = T*k assignments, not the
+    padded rows; weights read once), t_roof = max(FLOPs / P_mxfp8, bytes / BW_copy), and the
+    fraction of each resource the measured step reaches.  Also the aggregate HBM fraction
+    of the data-movement kernels (routing, dispatch, combine; and their backward twins)."""
+    T, d, f, E, k = case.T, case.d, case.f, case.E, case.k
+    A = T * k
+    mx = 1 + 1 / 32
+    by = {
+        "route": 4 * T * E + 8 * A + 8 * A,
+        "permute": 2 * T * d + A * d * mx,
+        "gateup": 2 * E * f * d * mx + A * d * mx + A * f * mx + (4 * A * f if bwd else 0),
+        "down": E * d * f * mx + A * f * mx + 4 * A * d,
+        "combine": 4 * A * d + 2 * T * d,
+    }
+    fl = {"gateup": 4.0 * A * d * f, "down": 2.0 * A * d * f}
+    if bwd:
+        by.update({
+            "bwd_dout": 2 * T * d + A * d * mx,
+            "bwd_dgrad_down": E * f * d * mx + A * d * mx + 4 * A * f,
+            "bwd_swiglu": A * f * (4 + 4 + 1 + 2) * (1 + 1 / 64),
+            "bwd_dgrad_gateup": 2 * E * d * f * mx + 2 * A * f * mx + 4 * A * d,
+            "bwd_dx": 4 * A * d + 2 * T * d,
+            "bwd_transpose": 2 * A * (2 * d + 3 * f) * mx,
+            "bwd_wgrad": 2 * E * 3 * d * f + A * (2 * d + 3 * f) * mx,
+        })
+        fl.update({"bwd_dgrad_down": 2.0 * A * d * f, "bwd_dgrad_gateup": 4.0 * A * d * f,
+                   "bwd_wgrad": 6.0 * A * d * f})
+    flops, nbytes = sum(fl.values()), sum(by.values())
+    p_mx, bw = 2.0 * peaks["bf16"] * 1e12, peaks["hbm"] * 1e9
+    t_roof = max(flops / p_mx, nbytes / bw)
+    sec = ms_step * 1e-3
+    moves = [n for n in ("route", "permute", "combine", "bwd_dout", "bwd_dx") if n in by]
+    mv_ms = sum(stage_ms.get(n, 0.0) for n in moves)
+    mv_bytes = sum(by[n] for n in moves if n in stage_ms)
+    return {"flops": flops, "bytes": nbytes, "t_roof_ms": t_roof * 1e3,
+            "bound": "tensor" if flops / p_mx >= nbytes / bw else "hbm",
+            "frac_of_roof": t_roof / sec, "tensor_frac": flops / sec / p_mx,
+            "hbm_frac": nbytes / sec / bw,
+            "data_movement_hbm_frac": (mv_bytes / (mv_ms * 1e-3) / bw) if mv_ms > 0 else None,
+            "data_movement_kernels": moves}
+
+
+def _safe_layer_summary(case, stage_info, ms_step, peaks, bwd):
+    try:
+        return layer_summary(case, {n: v["ms_per_launch"] for n, v in stage_info.items()},
+                             ms_step, peaks, bwd)
+    except Exception as e:  # reporting only: never lose the benchmark line over it
+        return {"error": repr(e)}
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -492,6 +544,7 @@ def run_ours(args, case):
         "fwd_tokens_per_s": world * case.T / (fwd_ms * 1e-3),
         "bwd_tokens_per_s": world * case.T / (bwd_ms * 1e-3) if bwd else None,
         "layer_tflops": layer_flops / (ms_step * 1e-3) / 1e12,
+        "layer_roofline": _safe_layer_summary(case, stage_info, ms_step, peaks, bwd),
         "layer_frac_mxfp8": layer_flops / (ms_step * 1e-3) / 1e12 / mx_peak,
         "weights_gbs_fwd": w_bytes / (fwd_ms * 1e-3) / 1e9,
         "stages": stage_info,

@@ -55,3 +55,32 @@ def test_oracle_sample_is_bounded():
     assert len(chosen) == 2
     assert sum(counts[e] for e in chosen) <= 1024      # a pass stays a few seconds
     assert hasattr(bench, "OracleSample") and hasattr(bench, "cpu_baseline")
+
+
+def test_layer_summary_closed_form():
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    case = synth.CONFIGS["dsv3"]
+    A = case.T * case.k
+    peaks = {"bf16": 1000.0, "hbm": 5000.0}          # 2 PFLOP/s MXFP8, 5 TB/s
+    fwd_stages = {"route": 0.05, "permute": 0.2, "gateup": 2.0, "down": 1.5, "combine": 0.3}
+    r = bench.layer_summary(case, fwd_stages, 4.05, peaks, bwd=False)
+    assert r["flops"] == pytest.approx(6.0 * A * case.d * case.f)
+    weights = 3 * case.E * case.d * case.f * (1 + 1 / 32)
+    assert r["bytes"] > weights                       # weights read once, plus activations
+    t_fl, t_by = r["flops"] / 2e15, r["bytes"] / 5e12
+    assert r["t_roof_ms"] == pytest.approx(1e3 * max(t_fl, t_by))
+    assert r["bound"] == ("tensor" if t_fl >= t_by else "hbm")
+    assert r["tensor_frac"] == pytest.approx(r["flops"] / 4.05e-3 / 2e15)
+    assert r["frac_of_roof"] == pytest.approx(r["t_roof_ms"] / 4.05)
+    mv = (4 * case.T * case.E + 16 * A) + (2 * case.T * case.d + A * case.d * (1 + 1 / 32)) + \
+        (4 * A * case.d + 2 * case.T * case.d)
+    assert r["data_movement_hbm_frac"] == pytest.approx(mv / 0.55e-3 / 5e12)
+    bwd_stages = dict(fwd_stages, bwd_dout=0.2, bwd_dgrad_down=1.3, bwd_swiglu=0.4,
+                      bwd_dgrad_gateup=2.7, bwd_dx=0.3, bwd_transpose=1.0, bwd_wgrad=6.2)
+    rb = bench.layer_summary(case, bwd_stages, 16.6, peaks, bwd=True)
+    assert rb["flops"] == pytest.approx(18.0 * A * case.d * case.f)
+    # the weight gradients' bf16 output alone: 2 bytes x E x 3 x d x f
+    assert rb["bytes"] - r["bytes"] > 2 * case.E * 3 * case.d * case.f
+    assert rb["bound"] == "hbm"
