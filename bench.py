@@ -257,6 +257,17 @@ class OracleSample:
                 f"{passes} pass(es), {seconds:.1f} s timed")
 
 
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def _threads():
     try:
         from threadpoolctl import threadpool_info
@@ -276,7 +287,7 @@ def cpu_baseline(case, budget_s: float = 15.0, with_bwd: bool = False):
     value = (sample.n_rows / case.k) * passes / total
     return {"value": value, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
             "sample": sample.describe(total, passes),
-            "host_cores_visible": len(os.sched_getaffinity(0))}
+            "host_cores_visible": len(os.sched_getaffinity(0)), "host_cpu": _cpu_model()}
 
 
 def run_reference(args, case):
@@ -297,7 +308,8 @@ def run_reference(args, case):
         vals.append((sample.n_rows / case.k) / s)
     wall = time.perf_counter() - t0
     value = statistics.median(vals)
-    info = {"cores": _threads(), "sample": sample.describe(secs, args.steps)}
+    info = {"cores": _threads(), "sample": sample.describe(secs, args.steps),
+            "host_cpu": _cpu_model()}
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * case.T / value, "higher_is_better": True, "scaling": "weak",
@@ -307,7 +319,7 @@ def run_reference(args, case):
                        "T": case.T, "d": case.d, "f": case.f, "E": case.E, "k": case.k},
             "impl": "reference",
             "cpu_baseline": {"kind": "oracle", "cores": info["cores"], "sample": info["sample"],
-                             "value": value, "unit": "tokens/s"},
+                             "value": value, "unit": "tokens/s", "host_cpu": info["host_cpu"]},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
             "wall_s": wall}
