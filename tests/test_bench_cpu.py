@@ -84,3 +84,14 @@ def test_layer_summary_closed_form():
     # the weight gradients' bf16 output alone: 2 bytes x E x 3 x d x f
     assert rb["bytes"] - r["bytes"] > 2 * case.E * 3 * case.d * case.f
     assert rb["bound"] == "hbm"
+
+
+@pytest.mark.parametrize("with_bwd", [False, True])
+def test_cpu_baseline_fields(with_bwd):
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    r = bench.cpu_baseline(synth.CONFIGS["tiny"], budget_s=0.2, with_bwd=with_bwd)
+    assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
+    assert r["cores"] >= 1 and r["host_cores_visible"] >= 1 and r["host_cpu"]
+    assert ("backward" in r["sample"]) == with_bwd
