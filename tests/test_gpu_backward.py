@@ -135,3 +135,27 @@ def test_backward_no_tokens(moe):
     assert tuple(out.shape) == (0, case.d) and tuple(grads["dx"].shape) == (0, case.d)
     for name in ("dWg", "dWu", "dWd"):
         assert not torch.any(grads[name].float() != 0), name
+
+
+def test_backward_latches_bounds_error_on_corrupted_state(moe):
+    # Fault detection without a fault: an out-of-range expert id in the saved routing
+    # state is caught by the dX combine's index check (before any access), latched as
+    # MOE_ERR_DEVICE_BOUNDS (7) in the workspace and read back; the context stays usable.
+    import torch
+    case = synth.MoeCase("b_bad", 300, 256, 512, 8, 2, 0, "none", seed=15)
+    dims = moe.Dims(case.T, case.d, case.f, case.E, case.k, case.score_fn)
+    wg, wu, wd = synth.expert_weights_torch(case, "cuda")
+    pw = moe.prepare_weights(wg, wu, wd, dims, with_backward=True)
+    x = bits_to_bf16_tensor(synth.make_x(case), "cuda")
+    lg = torch.from_numpy(synth.make_logits(case)).cuda()
+    wsf = moe.workspace(dims, moe.OP_FORWARD)
+    _, saved = moe.forward(x, lg, pw, save=True, ws=wsf)
+    assert moe.device_status(wsf) == 0
+    saved.bufs["topk_idx"][5] = case.E + 5
+    wsb = moe.workspace(dims, moe.OP_BACKWARD)
+    moe.backward(bits_to_bf16_tensor(synth.make_dout(case), "cuda"), pw, saved, ws=wsb)
+    assert moe.device_status(wsb) == 7
+    assert moe.device_status(wsb) == 0            # reading clears the latched word
+    y, _ = moe.forward(x, lg, pw, ws=wsf)         # the context is still usable
+    torch.cuda.synchronize()
+    assert moe.device_status(wsf) == 0
