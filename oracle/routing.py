@@ -59,6 +59,35 @@ def routing_weights(logits: np.ndarray, idx: np.ndarray, score_fn: int) -> np.nd
     raise ValueError(score_fn)
 
 
+def routing_weights_backward(logits: np.ndarray, idx: np.ndarray, dw: np.ndarray,
+                             score_fn: int) -> np.ndarray:
+    """d(loss)/d(logits) [T, E] in fp64 from d(loss)/d(combine weights) ``dw`` [T, k].
+
+    The top-k selection is piecewise constant in the logits, so only the k selected
+    logits of a token receive a gradient (the others get exactly zero); through the
+    weights it is the chain rule of the two definitions above:
+      softmax-top-k:  w = softmax(l_sel)         -> dl_i = w_i (dw_i - sum_j w_j dw_j)
+      sigmoid-renorm: w = s / sum(s), s = sig(l) -> ds_i = (dw_i - sum_j w_j dw_j) / sum(s),
+                                                     dl_i = ds_i s_i (1 - s_i)
+    """
+    logits = np.asarray(logits, np.float64)
+    idx = idx.astype(np.int64)
+    dw = np.asarray(dw, np.float64)
+    w = routing_weights(logits, idx, score_fn)
+    centred = dw - np.sum(w * dw, axis=1, keepdims=True)
+    if score_fn == SCORE_SOFTMAX_TOPK:
+        dsel = w * centred
+    elif score_fn == SCORE_SIGMOID_RENORM:
+        sel = np.take_along_axis(logits, idx, axis=1)
+        s = 1.0 / (1.0 + np.exp(-sel))
+        dsel = centred / s.sum(axis=1, keepdims=True) * s * (1.0 - s)
+    else:
+        raise ValueError(score_fn)
+    out = np.zeros_like(logits)
+    np.put_along_axis(out, idx, dsel, axis=1)
+    return out
+
+
 def route(logits: np.ndarray, k: int, score_fn: int):
     """Top-k indices [T,k] int32 and weights [T,k] float64."""
     idx = topk_select(logits, k)

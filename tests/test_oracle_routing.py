@@ -117,3 +117,84 @@ def test_imbalance_config_load_pattern():
     assert (counts == 0).sum() == 16
     share = np.sort(counts)[-4:].sum() / idx.size
     assert 0.4 < share < 0.55
+
+
+# ---------------------------------------------------------------------------------------
+# Router backward: d(logits) from d(combine weights)
+# ---------------------------------------------------------------------------------------
+def _spread_logits(rng, T, E):
+    # distinct logits at least 0.05 apart inside each row, so a 1e-6 perturbation never
+    # changes the top-k set
+    base = rng.permutation(np.arange(E, dtype=np.float64))[None, :].repeat(T, axis=0)
+    return 0.05 * base + 0.01 * rng.random((T, E)) + rng.standard_normal((T, 1))
+
+
+@pytest.mark.parametrize("score", [rt.SCORE_SOFTMAX_TOPK, rt.SCORE_SIGMOID_RENORM])
+@pytest.mark.parametrize("k", [1, 2, 5])
+def test_router_backward_central_differences(score, k):
+    rng = np.random.default_rng(100 + 10 * k + score)
+    T, E = 6, 9
+    logits = _spread_logits(rng, T, E)
+    idx = rt.topk_select(logits.astype(np.float32), k)
+    dw = rng.standard_normal((T, k))
+    got = rt.routing_weights_backward(logits, idx, dw, score)
+
+    def loss(lg):
+        return float(np.sum(dw * rt.routing_weights(lg, idx, score)))
+
+    eps = 1e-6
+    fd = np.zeros_like(logits)
+    for t in range(T):
+        for e in range(E):
+            lp, lm = logits.copy(), logits.copy()
+            lp[t, e] += eps
+            lm[t, e] -= eps
+            # the selection is held fixed (it does not change under these perturbations)
+            assert np.array_equal(rt.topk_select(lp.astype(np.float32), k), idx)
+            fd[t, e] = (loss(lp) - loss(lm)) / (2 * eps)
+    np.testing.assert_allclose(got, fd, rtol=1e-6, atol=1e-9)
+
+
+@pytest.mark.parametrize("score", [rt.SCORE_SOFTMAX_TOPK, rt.SCORE_SIGMOID_RENORM])
+def test_router_backward_matches_torch_autograd(score):
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(7 + score)
+    T, E, k = 16, 12, 4
+    logits = rng.standard_normal((T, E)) * 2.0
+    idx = rt.topk_select(logits.astype(np.float32), k)
+    dw = rng.standard_normal((T, k))
+    lt = torch.tensor(logits, dtype=torch.float64, requires_grad=True)
+    sel = torch.gather(lt, 1, torch.tensor(idx, dtype=torch.int64))
+    if score == rt.SCORE_SOFTMAX_TOPK:
+        w = torch.softmax(sel, dim=1)
+    else:
+        s = torch.sigmoid(sel)
+        w = s / s.sum(dim=1, keepdim=True)
+    w.backward(torch.tensor(dw))
+    np.testing.assert_allclose(rt.routing_weights_backward(logits, idx, dw, score),
+                               lt.grad.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_router_backward_invariants():
+    rng = np.random.default_rng(3)
+    T, E, k = 32, 10, 3
+    logits = rng.standard_normal((T, E))
+    idx = rt.topk_select(logits.astype(np.float32), k)
+    dw = rng.standard_normal((T, k))
+    for score in (rt.SCORE_SOFTMAX_TOPK, rt.SCORE_SIGMOID_RENORM):
+        g = rt.routing_weights_backward(logits, idx, dw, score)
+        mask = np.zeros((T, E), bool)
+        np.put_along_axis(mask, idx.astype(np.int64), True, axis=1)
+        assert np.all(g[~mask] == 0.0)                # unselected experts: no gradient
+    # softmax over the selected logits is shift-invariant: each row's gradient sums to 0
+    g = rt.routing_weights_backward(logits, idx, dw, rt.SCORE_SOFTMAX_TOPK)
+    np.testing.assert_allclose(g.sum(axis=1), 0.0, atol=1e-14)
+    # a constant d(weights) changes nothing (the weights always sum to one)
+    for score in (rt.SCORE_SOFTMAX_TOPK, rt.SCORE_SIGMOID_RENORM):
+        g = rt.routing_weights_backward(logits, idx, np.full((T, k), 0.7), score)
+        np.testing.assert_allclose(g, 0.0, atol=1e-15)
+    # k = 1: the single weight is identically one
+    idx1 = rt.topk_select(logits.astype(np.float32), 1)
+    for score in (rt.SCORE_SOFTMAX_TOPK, rt.SCORE_SIGMOID_RENORM):
+        assert np.all(rt.routing_weights_backward(logits, idx1, rng.standard_normal((T, 1)),
+                                                  score) == 0.0)
