@@ -19,7 +19,7 @@
  *     latched into a status word inside the workspace and read back with
  *     moe_get_device_status(); device code never traps.
  *   - Shapes: d % 256 == 0, f % 256 == 0, 1 <= k <= min(E, 32), 1 <= E <= 1024, T >= 0,
- *     T*k < 2^31.  Pointers must be 16-byte aligned; workspaces 256-byte aligned, and
+ *     T*k + 127*E + 127 < 2^31 (the padded row count fits int32).  Pointers must be 16-byte aligned; workspaces 256-byte aligned, and
  *     the first 256 bytes of a workspace must be zero when it is first used (they hold
  *     the latched device status).
  *

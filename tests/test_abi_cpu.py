@@ -57,7 +57,9 @@ def test_sizes(lib):
 
 @pytest.mark.parametrize("bad,code", [
     (dict(d=200), 2), (dict(f=384), 2), (dict(k=33, E=64), 2), (dict(E=1025), 2),
-    (dict(k=9, E=8), 2), (dict(T=-1), 1), (dict(s=3), 1), (dict(E=0), 1)])
+    (dict(k=9, E=8), 2), (dict(T=-1), 1), (dict(s=3), 1), (dict(E=0), 1),
+    # T*k below 2^31 but the padded row count (T*k + 127*E, rounded up) is not
+    (dict(T=(2**31 - 1024 * 127) // 2, k=2, E=1024), 2)])
 def test_dims_rejected_before_any_launch(lib, bad, code):
     args = dict(T=16, d=256, f=256, E=8, k=2, s=0)
     args.update(bad)

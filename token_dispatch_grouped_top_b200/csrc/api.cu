@@ -28,7 +28,9 @@ moe_status check_dims(const moe_dims* D) {
     return MOE_ERR_INVALID_ARG;
   if (D->E > 1024 || D->k > D->E || D->k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (D->d % 256 || D->f % 256) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (D->T * D->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  // row indices of the padded expert-contiguous buffers (and their offsets) are int32
+  if (D->T * D->k + static_cast<int64_t>(D->E) * 127 + 127 >= (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
 
