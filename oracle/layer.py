@@ -164,6 +164,37 @@ def forward(x_bits, logits, k, score_fn, E, weights_fn, tokens=None, keep=False,
     return res
 
 
+def forward_bf16(x_bits, logits, k, score_fn, E, weights_fn, round_h=True):
+    """Oracle forward of the layer's BF16 variant (no MX quantisation).
+
+    Reading (the pages report BF16 results beside MXFP8 ones and say nothing more): the
+    same layer with bf16 operands throughout -- x and the expert weights as given (bf16
+    values), each GEMM accumulated exactly here (fp32 on the device), and the SwiGLU output
+    rounded to bf16, the operand dtype of the down GEMM:
+        g = x Wg, u = x Wu, h = bf16(silu(g) * u), y = h Wd, out_t = sum_j w[t,j] y.
+    ``round_h=False`` drops that rounding (the structure pin against forward_exact).
+    Returns dict with idx, w and out [T,d] (fp64, before the final bf16 rounding).
+    """
+    T, d = x_bits.shape
+    idx, w = rt.route(logits, k, score_fn)
+    counts, offsets, perm, inv = rt.layout(idx, E)
+    x = bf16_bits_to_f64(x_bits)
+    out = np.zeros((T, d), np.float64)
+    wflat = w.reshape(-1)
+    for e in range(E):
+        rows = perm[offsets[e]:offsets[e + 1]]
+        if rows.size == 0:
+            continue
+        t = rows // k
+        wg, wu, wd = weights_fn(e)
+        g, u = x[t] @ wg, x[t] @ wu
+        h = g * sigmoid(g) * u
+        if round_h:
+            h = bf16_round(h)
+        np.add.at(out, t, wflat[rows][:, None] * (h @ wd))
+    return dict(idx=idx, w=w, out=out)
+
+
 def backward(x_bits, logits, dout_bits, k, score_fn, E, weights_fn, experts=None,
              want_dx=True, exact=False, prepared=None):
     """Oracle backward (quantised reading, see module docstring).

@@ -253,3 +253,71 @@ def test_weight_gradient_sensitivity(monkeypatch):
     assert 0 < n_out <= 1e-4 * n_el            # flips happen, and they are rare
     r = np.sqrt(np.mean(ref["dx"] ** 2))
     assert np.max(np.abs(got["dx"] - ref["dx"])) <= 3e-2 * r
+
+
+# ---------------------------------------------------------------------------------------
+# BF16 variant of the layer (no MX quantisation)
+# ---------------------------------------------------------------------------------------
+def _brute_forward_bf16(x_bits, logits, k, score_fn, wfn):
+    """Per-token, per-slot loop: bf16 operands, h rounded to bf16 between the GEMMs."""
+    x = L.bf16_bits_to_f64(x_bits)
+    T, d = x.shape
+    out = np.zeros((T, d))
+    for t in range(T):
+        order = sorted(range(logits.shape[1]), key=lambda e: (-float(logits[t, e]), e))[:k]
+        sel = np.array([float(logits[t, e]) for e in order])
+        if score_fn == 0:
+            w = np.exp(sel - sel.max()); w /= w.sum()
+        else:
+            s = 1 / (1 + np.exp(-sel)); w = s / s.sum()
+        for j, e in enumerate(order):
+            Wg, Wu, Wd = wfn(e)
+            g, u = x[t] @ Wg, x[t] @ Wu
+            h = L.bf16_round(g / (1 + np.exp(-g)) * u)
+            out[t] += w[j] * (h @ Wd)
+    return out
+
+
+@pytest.mark.parametrize("score,bias", [(0, "none"), (1, "normal0.5")])
+def test_bf16_variant_matches_bruteforce(score, bias):
+    case = _case(score=score, bias=bias, seed=21)
+    x, lg, wfn = _inputs(case)
+    got = L.forward_bf16(x, lg, case.k, case.score_fn, case.E, wfn)["out"]
+    np.testing.assert_allclose(got, _brute_forward_bf16(x, lg, case.k, case.score_fn, wfn),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_bf16_variant_structure_and_rounding_bound():
+    case = _case(seed=22)
+    x, lg, wfn = _inputs(case)
+    idx, w = rt.route(lg, case.k, case.score_fn)
+    weights = [wfn(e) for e in range(case.E)]
+    exact = L.forward_exact(L.bf16_bits_to_f64(x), idx, w, weights)
+    # without the h rounding the variant is the exact layer
+    unrounded = L.forward_bf16(x, lg, case.k, case.score_fn, case.E, wfn, round_h=False)["out"]
+    np.testing.assert_allclose(unrounded, exact, rtol=1e-12, atol=1e-12)
+    # with it, each h element moves by at most half a bf16 quantum (2^-9 relative), so
+    # |out - exact| <= sum_j w_j * 2^-9 * |h_j| @ |Wd|, elementwise
+    got = L.forward_bf16(x, lg, case.k, case.score_fn, case.E, wfn)["out"]
+    xf = L.bf16_bits_to_f64(x)
+    bound = np.zeros_like(exact)
+    for t in range(case.T):
+        for j in range(case.k):
+            Wg, Wu, Wd = weights[int(idx[t, j])]
+            g, u = xf[t] @ Wg, xf[t] @ Wu
+            h = g * L.sigmoid(g) * u
+            bound[t] += w[t, j] * (2.0 ** -9 * np.abs(h)) @ np.abs(Wd)
+    assert np.all(np.abs(got - exact) <= bound * (1 + 1e-9) + 1e-300)
+    assert np.any(got != exact)                   # the rounding is real
+
+
+def test_bf16_variant_k1_is_unpermute():
+    case = _case(k=1, seed=23)
+    x, lg, wfn = _inputs(case)
+    r = L.forward_bf16(x, lg, 1, case.score_fn, case.E, wfn)
+    xf = L.bf16_bits_to_f64(x)
+    for t in range(case.T):
+        Wg, Wu, Wd = wfn(int(r["idx"][t, 0]))
+        g, u = xf[t] @ Wg, xf[t] @ Wu
+        np.testing.assert_allclose(r["out"][t], L.bf16_round(g * L.sigmoid(g) * u) @ Wd,
+                                   rtol=1e-12, atol=1e-12)
