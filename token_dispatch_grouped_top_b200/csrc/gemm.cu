@@ -145,19 +145,6 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
 // Relative error ~1e-6 (large |x|: e^-x -> 0 or inf gives exactly 1 or 0).
 __device__ __forceinline__ float sigmoid_fast(float x) { return __frcp_rn(1.f + __expf(-x)); }
 
-// E4M3 byte -> fp32, exact (normal: (1 + m/8) 2^(e-7); subnormal: m 2^-9).
-__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
-  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
-  const float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20))
-                    : static_cast<float>(m) * 0.001953125f;
-  return (c & 0x80u) ? -v : v;
-}
-
-// E8M0 byte -> 2^(b-127) as fp32 (2^-127 is subnormal).
-__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
-  return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
-}
-
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
