@@ -88,7 +88,14 @@ def test_status_strings(lib):
 
 def test_wave_rule_reproduces_minibatch_figure(lib):
     """Two full waves of 128x256 tiles on 148 SMs for the gate/up GEMM (N = 2*2048) need
-    2368 tokens -- the article's minimum minibatch at hidden 7168 / intermediate 2048."""
-    assert lib.moe_min_tokens_for_waves(148, 2, 128, 256, 2 * 2048) == 2368
+    2368 tokens -- the article's minimum minibatch at hidden 7168 / intermediate 2048
+    (the printed value and its citation: tests/golden/minibatch_waves.txt)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "minibatch_waves.txt")
+    g = dict(line.strip().split("=") for line in open(path)
+             if line.strip() and not line.startswith("#"))
+    g = {key: int(v) for key, v in g.items()}
+    assert lib.moe_min_tokens_for_waves(g["sms"], g["waves"], g["tile_m"], g["tile_n"],
+                                        2 * g["intermediate"]) == g["min_tokens"]
     assert lib.moe_min_tokens_for_waves(148, 1, 128, 256, 2 * 2048) == 1184
     assert lib.moe_min_tokens_for_waves(0, 1, 128, 256, 4096) == -1
