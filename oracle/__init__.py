@@ -17,7 +17,9 @@ brute force (see ``tests/test_oracle_*.py``), not by numbers from the pages.
 
 Modules
   mxfp8   -- OCP MX E4M3 / E8M0 block quantiser, bit-exact, along the last axis.
-  routing -- top-k routing, routing weights, per-expert layout (counts, offsets, perm).
-  layer   -- expert FFN forward / backward on MX-quantised operands, one expert at a time.
+  routing -- top-k routing, routing weights and their backward to the logits, per-expert
+             layout (counts, offsets, perm).
+  layer   -- expert FFN forward / backward on MX-quantised operands, one expert at a time;
+             the layer's BF16 variant (no MX) forward.
 """
 from . import mxfp8, routing, layer  # noqa: F401
