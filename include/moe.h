@@ -19,9 +19,9 @@
  *     latched into a status word inside the workspace and read back with
  *     moe_get_device_status(); device code never traps.
  *   - Shapes: d % 256 == 0, f % 256 == 0, 1 <= k <= min(E, 32), 1 <= E <= 1024, T >= 0,
- *     T*k + 127*E + 127 < 2^31 (the padded row count fits int32).  Pointers must be 16-byte aligned; workspaces 256-byte aligned, and
- *     the first 256 bytes of a workspace must be zero when it is first used (they hold
- *     the latched device status).
+ *     T*k + 127*E + 127 < 2^31 (the padded row count fits int32).  Pointers must be
+ *     16-byte aligned; workspaces 256-byte aligned, and the first 256 bytes of a
+ *     workspace must be zero when it is first used (they hold the latched device status).
  *
  * Notation: T tokens, d hidden size, f expert intermediate size, E experts, k experts per
  * token, A = T*k assignments with id a = t*k + j (j = rank of the expert among the
@@ -125,8 +125,9 @@ const char* moe_status_string(moe_status s);
  * Article lead and §01 (router picks experts per token; count tokens per expert, decide
  * placement, keep each expert's tokens contiguous).
  * logits [T,E] fp32 -> topk_idx [T,k] (top-k by logit, ties to the lower expert index,
- * slot j = rank), topk_w [T,k] (softmax over the k selected logits, or sigmoid scores
- * renormalised over the k selected), counts [E], offsets [E+1], perm [A] (stable:
+ * slot j = rank; a NaN logit ranks as -inf, so every index is a valid expert),
+ * topk_w [T,k] (softmax over the k selected logits, or sigmoid scores renormalised over
+ * the k selected), counts [E], offsets [E+1], perm [A] (stable:
  * ascending token inside each expert), inv_perm [A].  Indices are exact; weights fp32.
  * pad_offsets [E+1] (nullable): padded segment starts.  ws: moe_workspace_bytes(ROUTE). */
 moe_status moe_route_layout(const moe_dims* dims, const float* logits, int32_t* topk_idx,
@@ -142,15 +143,17 @@ moe_status moe_route_layout(const moe_dims* dims, const float* logits, int32_t* 
  * and results as moe_route_layout, but the scratch lives in a fixed 8 MiB array inside
  * the library (held by every GPU that loads the library until the process exits);
  * nothing is allocated and no workspace is passed.
- *  - Problems whose scratch exceeds 8 MiB return MOE_ERR_UNSUPPORTED_SHAPE before any
+ *  - The shape rules, pointer checks and device check are those of moe_route_layout.
+ *    Problems whose scratch exceeds 8 MiB return MOE_ERR_UNSUPPORTED_SHAPE before any
  *    launch.  The scratch is 256 + 4*nt + 8*nt*E + 4*T*k + 4*(E+1) bytes (each term
  *    rounded up to 256) with nt = ceil(T/64): e.g. E = 256, k = 8 fits T <= 130896.
- *  - The first call on a device looks up the array's device address for that device
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress; it allocates nothing), so a device reset is picked up; make
+ *    the first call on a device before any stream capture.
  *  - Every call shares the one array: calls whose executions overlap on the GPU race on
  *    it and give wrong results.  Each call clears the parts that must start at zero.
- *  - status (nullable, device int32, zeroed by the caller): device-side errors are
- *    latched there (first error wins) instead of in a workspace. */
+ *  - status (device int32, zeroed by the caller; required when T > 0): device-side
+ *    errors are latched there (first error wins) instead of in a workspace. */
 moe_status moe_route_layout_noalloc(const moe_dims* dims, const float* logits,
                                     int32_t* topk_idx, float* topk_w, int32_t* counts,
                                     int32_t* offsets, int32_t* perm, int32_t* inv_perm,

@@ -24,12 +24,23 @@ SCORE_SOFTMAX_TOPK = 0
 SCORE_SIGMOID_RENORM = 1
 
 
+def rank_keys(logits: np.ndarray, dtype=np.float32) -> np.ndarray:
+    """The logits as ranking keys: a NaN logit ranks as -inf (the lowest key).
+
+    Reading: the pages say nothing about invalid router outputs; a NaN must not be chosen
+    ahead of any number, and when a row has fewer than k numbers the NaN experts are
+    taken like -inf ones, lower index first.  The same keys feed the weights.
+    """
+    a = np.asarray(logits, dtype=dtype)
+    return np.where(np.isnan(a), a.dtype.type(-np.inf), a)
+
+
 def topk_select(logits: np.ndarray, k: int) -> np.ndarray:
     """Indices [T, k] of the k largest logits per row, ties broken by the lower index.
 
     A stable ascending sort of -logit keeps equal keys in index order.
     """
-    logits = np.asarray(logits, dtype=np.float32)
+    logits = rank_keys(logits)
     order = np.argsort(-logits, axis=1, kind="stable")
     return order[:, :k].astype(np.int32)
 
@@ -37,7 +48,7 @@ def topk_select(logits: np.ndarray, k: int) -> np.ndarray:
 def topk_select_bruteforce(logits: np.ndarray, k: int) -> np.ndarray:
     """Per-token Python sort by the key (-logit, expert)."""
     out = []
-    for row in np.asarray(logits, dtype=np.float32):
+    for row in rank_keys(logits):
         keyed = sorted(range(row.shape[0]), key=lambda e: (-float(row[e]), e))
         out.append(keyed[:k])
     return np.array(out, dtype=np.int32).reshape(len(out), k)
@@ -49,7 +60,7 @@ def routing_weights(logits: np.ndarray, idx: np.ndarray, score_fn: int) -> np.nd
     softmax-top-k: softmax over the k selected logits (max subtracted).
     sigmoid-renorm: s = 1 / (1 + exp(-logit)) for the selected experts, w = s / sum(s).
     """
-    sel = np.take_along_axis(np.asarray(logits, np.float64), idx.astype(np.int64), axis=1)
+    sel = np.take_along_axis(rank_keys(logits, np.float64), idx.astype(np.int64), axis=1)
     if score_fn == SCORE_SOFTMAX_TOPK:
         z = np.exp(sel - sel.max(axis=1, keepdims=True))
         return z / z.sum(axis=1, keepdims=True)

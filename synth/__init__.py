@@ -221,5 +221,16 @@ def expert_weights_torch(case: MoeCase, device, experts=None):
     return tuple(outs)
 
 
+def expert_weights_uploaded(case: MoeCase, device):
+    """The same weights as :func:`expert_weights_torch`, drawn on the host with NumPy and
+    uploaded with one copy per matrix (for small cases: no device-side generator kernels)."""
+    import torch
+    outs = []
+    for which in (_WG, _WU, _WD):
+        bits = np.stack([expert_weight_bits(case, e, which) for e in range(case.E)])
+        outs.append(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device))
+    return tuple(outs)
+
+
 def case_by_name(name: str, **overrides) -> MoeCase:
     return CONFIGS[name].replace(**overrides) if overrides else CONFIGS[name]

@@ -63,6 +63,33 @@ def test_route_all_tokens_one_expert_and_empty_batch(moe):
     assert not to_np(res["counts"]).any() and not to_np(res["offsets"]).any()
 
 
+@pytest.mark.parametrize("score", [0, 1])
+def test_route_nan_logits_rank_as_minus_infinity(moe, score):
+    # Rows with a few NaN logits, rows with fewer than k numbers and all-NaN rows: every
+    # index stays a valid expert (the oracle's reading: a NaN ranks as -inf) and no device
+    # error is latched.  Weights of rows that had to take -inf experts may be NaN on both
+    # sides (0/0); they must be NaN at the same places and close elsewhere.
+    import torch
+    T, E, k = 300, 40, 6
+    rng = np.random.default_rng(17 + score)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    lg[rng.random((T, E)) < 0.1] = np.nan
+    lg[::7, 3:] = np.nan                    # only 3 numbers left in these rows
+    lg[::11] = np.nan                       # nothing but NaN
+    lg[5, :10] = -np.inf
+    res = moe.route_layout(torch.from_numpy(lg).cuda(), k, score)
+    assert moe.device_status(res["ws"]) == 0
+    idx, w = ort.route(lg, k, score)
+    counts, offsets, perm, inv = ort.layout(idx, E)
+    assert np.array_equal(to_np(res["idx"]), idx)
+    gw = to_np(res["w"]).astype(np.float64)
+    assert np.array_equal(np.isnan(gw), np.isnan(w))
+    ok = ~np.isnan(w)
+    assert np.max(np.abs(gw[ok] - w[ok])) <= 2e-6
+    for key, want in (("counts", counts), ("offsets", offsets), ("perm", perm), ("inv", inv)):
+        assert np.array_equal(to_np(res[key]), want), key
+
+
 def test_route_deterministic(moe):
     import torch
     case = synth.CONFIGS["imbalance"]

@@ -198,3 +198,21 @@ def test_router_backward_invariants():
     for score in (rt.SCORE_SOFTMAX_TOPK, rt.SCORE_SIGMOID_RENORM):
         assert np.all(rt.routing_weights_backward(logits, idx1, rng.standard_normal((T, 1)),
                                                   score) == 0.0)
+
+
+def test_nan_logits_rank_as_minus_infinity():
+    # Reading for invalid router outputs: a NaN ranks as -inf; -inf keys (NaN or not) are
+    # taken in index order once the numbers run out.  Expected indices written by hand.
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+    lg = np.array([[nan, 1.0, nan, -inf, 0.5],
+                   [nan, nan, nan, nan, nan],
+                   [-inf, nan, 2.0, nan, -inf]], np.float32)
+    idx = rt.topk_select(lg, 4)
+    assert idx[0].tolist() == [1, 4, 0, 2]
+    assert idx[1].tolist() == [0, 1, 2, 3]
+    assert idx[2].tolist() == [2, 0, 1, 3]
+    assert np.array_equal(idx, rt.topk_select_bruteforce(lg, 4))
+    # a finite row's weights do not see the NaN experts that were not selected
+    w = rt.routing_weights(lg[:1], np.array([[1, 4]]), rt.SCORE_SOFTMAX_TOPK)
+    assert np.allclose(w, [[1 / (1 + np.exp(-0.5)), np.exp(-0.5) / (1 + np.exp(-0.5))]],
+                       rtol=1e-15)

@@ -14,6 +14,9 @@ def test_weight_generators_agree_on_cpu():
             ref = synth.expert_weight_bits(case, e, which)
             got = t[e].contiguous().view(torch.int16).numpy().view(np.uint16)
             assert np.array_equal(got, ref)
+    up = synth.expert_weights_uploaded(case, "cpu")
+    for a, b in zip(up, (wg, wu, wd)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
 def test_weight_statistics():

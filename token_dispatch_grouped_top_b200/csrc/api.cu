@@ -13,10 +13,7 @@
 
 using namespace moe;
 
-namespace {
-
-constexpr int64_t kAlign = 256;
-inline int64_t align_up(int64_t x, int64_t a = kAlign) { return (x + a - 1) / a * a; }
+namespace moe {
 
 // ---------------------------------------------------------------------------------------
 // argument checks (pure host logic, no CUDA call)
@@ -33,9 +30,6 @@ moe_status check_dims(const moe_dims* D) {
     return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
-
-inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
 // ---------------------------------------------------------------------------------------
 // device properties
@@ -58,6 +52,16 @@ moe_status device_sms(int* num_sms) {
   *num_sms = sms;
   return MOE_OK;
 }
+
+}  // namespace moe
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+constexpr int64_t kAlign = 256;
+inline int64_t align_up(int64_t x, int64_t a = kAlign) { return (x + a - 1) / a * a; }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -401,6 +405,11 @@ moe_status moe_route_layout(const moe_dims* D, const float* logits, int32_t* top
                                                   !inv_perm)))
     return MOE_ERR_INVALID_ARG;
   if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  {
+    const void* ptrs[] = {logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, pad_offsets};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
   const WsLayout L = ws_layout(D, MOE_OP_ROUTE);
   if (ws_bytes < static_cast<size_t>(L.total)) return MOE_ERR_WORKSPACE_TOO_SMALL;
   int sms = 0;

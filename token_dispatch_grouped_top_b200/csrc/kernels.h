@@ -5,7 +5,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
+
+// Host-side checks shared by the entry points (api.cu): the shape rules of moe.h (no
+// CUDA call), and the current device's SM count (MOE_ERR_NO_DEVICE unless sm_100).
+moe_status check_dims(const moe_dims* D);
+moe_status device_sms(int* num_sms);
 
 struct RouteParams {
   const float* logits;

@@ -78,7 +78,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_rank_kernel(RouteParams P
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        v[u][i] = (tv && e < E) ? row[e] : -INFINITY;
+        // A NaN logit ranks as -inf: the comparisons below then always find k valid
+        // experts (ties, -inf included, go to the lower index).
+        const float lv = (tv && e < E) ? row[e] : -INFINITY;
+        v[u][i] = lv != lv ? -INFINITY : lv;
         if (e >= E) removed[u] |= 1u << i;
       }
       sel_v[u] = 0.f;
@@ -114,6 +117,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_rank_kernel(RouteParams P
       }
 #pragma unroll
       for (int u = 0; u < kTPW; ++u) {
+        if (be[u] < 0 || be[u] >= E) {  // cannot happen with finite or -inf keys; never index with it
+          if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+          be[u] = 0;
+        }
         if ((be[u] & 31) == lane) removed[u] |= 1u << (be[u] >> 5);
         if (lane == j) {
           sel_v[u] = bv[u];

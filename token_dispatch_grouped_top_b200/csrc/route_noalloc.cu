@@ -13,15 +13,17 @@
 //    library holds it until the process exits.
 //  - Problems whose scratch exceeds kScratchBytes are rejected (MOE_ERR_UNSUPPORTED_SHAPE)
 //    before anything is launched.
-//  - The first call on a device looks the array's device address up (once per device,
-//    with that device current); make that first call before any stream capture.
+//  - Every call looks the array's device address up for the current device
+//    (cudaGetSymbolAddress: no allocation, no synchronisation), so a context that was torn
+//    down and re-created (cudaDeviceReset) is picked up; make the first call on a device
+//    before any stream capture, since that lookup may load the library's module.
 //  - All calls share the one array.  Each call clears the parts that must start at zero
 //    (counters and lookback flags); calls whose executions overlap on the GPU (different
 //    streams, or different host threads) race on the array and give wrong results.
+//  - The same shape rules and device check as moe_route_layout apply; device-side errors
+//    are latched into the caller's status word, which is therefore required.
 //  - No cudaMalloc, cudaFree or allocating library routine is called.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "../../include/moe.h"
 #include "kernels.h"
@@ -54,27 +56,18 @@ ScratchLayout scratch_layout(const moe_dims* D) {
   return L;
 }
 
-// device address of the array, looked up once per device
+// device address of the array for the current device (looked up on every call)
 uint8_t* scratch_ptr(moe_status* st) {
-  static std::mutex mu;
-  static uint8_t* ptrs[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    *st = MOE_ERR_NO_DEVICE;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) {
+    *st = MOE_ERR_CUDA;
     return nullptr;
   }
-  std::lock_guard<std::mutex> g(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) {
-      *st = MOE_ERR_CUDA;
-      return nullptr;
-    }
-    ptrs[dev] = static_cast<uint8_t*>(p);
-  }
   *st = MOE_OK;
-  return ptrs[dev];
+  return static_cast<uint8_t*>(p);
 }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -83,24 +76,25 @@ extern "C" moe_status moe_route_layout_noalloc(const moe_dims* D, const float* l
                                                int32_t* offsets, int32_t* perm, int32_t* inv_perm,
                                                int32_t* pad_offsets, int32_t* status,
                                                void* stream) {
-  if (!D || D->T < 0 || D->d <= 0 || D->f <= 0 || D->E <= 0 || D->k <= 0 ||
-      (D->score_fn != MOE_SCORE_SOFTMAX_TOPK && D->score_fn != MOE_SCORE_SIGMOID_RENORM))
-    return MOE_ERR_INVALID_ARG;
-  if (D->E > 1024 || D->k > D->E || D->k > 32 || D->T * D->k >= (int64_t(1) << 31))
-    return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (!counts || !offsets || (D->T > 0 && (!logits || !topk_idx || !topk_w || !perm ||
-                                           !inv_perm)))
-    return MOE_ERR_INVALID_ARG;
+  const moe_status dim_ok = moe::check_dims(D);
+  if (dim_ok != MOE_OK) return dim_ok;
   const ScratchLayout L = scratch_layout(D);
   if (L.total > kScratchBytes) return MOE_ERR_UNSUPPORTED_SHAPE;
-
+  if (!counts || !offsets || (D->T > 0 && (!logits || !topk_idx || !topk_w || !perm ||
+                                           !inv_perm || !status)))
+    return MOE_ERR_INVALID_ARG;
+  {
+    const void* ptrs[] = {logits, topk_idx, topk_w, counts, offsets, perm, inv_perm,
+                          pad_offsets, status};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  int sms = 0;
+  const moe_status dev_ok = moe::device_sms(&sms);
+  if (dev_ok != MOE_OK) return dev_ok;
   moe_status st = MOE_OK;
   uint8_t* base = scratch_ptr(&st);
   if (st != MOE_OK) return st;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return MOE_ERR_NO_DEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* mtile = reinterpret_cast<int32_t*>(base + L.mtile);
   if (D->T == 0) {
