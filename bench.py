@@ -130,12 +130,11 @@ def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, ms: float) ->
     return world * tokens_per_rank * steps / (ms * 1e-3)
 
 
-def layer_summary(case, stage_ms: dict, ms_step: float, peaks: dict, bwd: bool) -> dict:
-    """Whole-layer roofline of one step: algorithmic FLOPs and HBM bytes (MX bytes include
-    the 1/32 scale overhead; activations counted for the A = T*k assignments, not the
-    padded rows; weights read once), t_roof = max(FLOPs / P_mxfp8, bytes / BW_copy), and the
-    fraction of each resource the measured step reaches.  Also the aggregate HBM fraction
-    of the data-movement kernels (routing, dispatch, combine; and their backward twins)."""
+def algorithmic_bytes(case, bwd: bool) -> dict:
+    """Bytes each stage must move by the method (the survey's per-unit figures times the
+    units of one step): MX bytes include the 1/32 scale overhead, activations count the
+    A = T*k assignments (no tile padding), expert outputs and input gradients per
+    assignment are bf16, weights are read once."""
     T, d, f, E, k = case.T, case.d, case.f, case.E, case.k
     A = T * k
     mx = 1 + 1 / 32
@@ -143,35 +142,80 @@ def layer_summary(case, stage_ms: dict, ms_step: float, peaks: dict, bwd: bool) 
         "route": 4 * T * E + 8 * A + 8 * A,
         "permute": 2 * T * d + A * d * mx,
         "gateup": 2 * E * f * d * mx + A * d * mx + A * f * mx + (4 * A * f if bwd else 0),
-        "down": E * d * f * mx + A * f * mx + 4 * A * d,
-        "combine": 4 * A * d + 2 * T * d,
+        "down": E * d * f * mx + A * f * mx + 2 * A * d,
+        "combine": 2 * A * d + 2 * T * d,
     }
-    fl = {"gateup": 4.0 * A * d * f, "down": 2.0 * A * d * f}
     if bwd:
         by.update({
             "bwd_dout": 2 * T * d + A * d * mx,
-            "bwd_dgrad_down": E * f * d * mx + A * d * mx + 4 * A * f,
-            "bwd_swiglu": A * f * (4 + 4 + 1 + 2) * (1 + 1 / 64),
-            "bwd_dgrad_gateup": 2 * E * d * f * mx + 2 * A * f * mx + 4 * A * d,
-            "bwd_dx": 4 * A * d + 2 * T * d,
+            "bwd_dgrad_down": E * f * d * mx + A * d * mx + 2 * A * f,
+            # G and the saved g|u read, h^ read, [dg|du]^ written, per assignment row
+            "bwd_swiglu": A * f * (2 + 4 + 3 * mx),
+            "bwd_dgrad_gateup": 2 * E * d * f * mx + 2 * A * f * mx + 2 * A * d,
+            "bwd_dx": 2 * A * d + 2 * T * d,
             "bwd_transpose": 2 * A * (2 * d + 3 * f) * mx,
             "bwd_wgrad": 2 * E * 3 * d * f + A * (2 * d + 3 * f) * mx,
         })
+    return by
+
+
+def implementation_bytes(case, bwd: bool, rows_used: int, rows_out: int) -> dict:
+    """Bytes the kernels actually move where they differ from the algorithmic count:
+    fp32 expert outputs / dgrad results, and the tile-padded rows (``rows_used``: rows
+    inside some expert segment; ``rows_out``: rows an fp32-output GEMM writes)."""
+    T, d, f, k = case.T, case.d, case.f, case.k
+    A = T * k
+    mx = 1 + 1 / 32
+    alg = algorithmic_bytes(case, bwd)
+    impl = dict(alg)
+    impl["down"] = alg["down"] - 2 * A * d + 4 * rows_out * d
+    impl["combine"] = 4 * A * d + 2 * T * d
+    if bwd:
+        impl["bwd_dgrad_down"] = alg["bwd_dgrad_down"] - 2 * A * f + 4 * rows_out * f
+        impl["bwd_swiglu"] = A * f * (4 + 4 + 3 * mx)
+        impl["bwd_dgrad_gateup"] = alg["bwd_dgrad_gateup"] - 2 * A * d + 4 * rows_out * d
+        impl["bwd_dx"] = 4 * A * d + 2 * T * d
+        impl["bwd_transpose"] = 2 * rows_used * (2 * d + 3 * f) * mx
+        impl["bwd_wgrad"] = 2 * case.E * 3 * d * f + rows_used * (2 * d + 3 * f) * mx
+    return impl
+
+
+def layer_flops(case, bwd: bool) -> dict:
+    A, d, f = case.T * case.k, case.d, case.f
+    fl = {"gateup": 4.0 * A * d * f, "down": 2.0 * A * d * f}
+    if bwd:
         fl.update({"bwd_dgrad_down": 2.0 * A * d * f, "bwd_dgrad_gateup": 4.0 * A * d * f,
                    "bwd_wgrad": 6.0 * A * d * f})
+    return fl
+
+
+DATA_MOVEMENT = ("route", "permute", "combine", "bwd_dout", "bwd_dx")
+
+
+def layer_summary(case, stage_ms: dict, ms_step: float, peaks: dict, bwd: bool) -> dict:
+    """Whole-layer roofline of one step: algorithmic FLOPs and HBM bytes
+    (:func:`algorithmic_bytes`), t_roof = max(FLOPs / P_mxfp8, bytes / BW_copy), and the
+    fraction of each resource the measured step reaches.  Also the aggregate HBM fraction
+    (sum of bytes over sum of times) of the data-movement kernels: routing, dispatch and
+    combine (forward) and, with the backward, its dispatch and combine twins."""
+    by, fl = algorithmic_bytes(case, bwd), layer_flops(case, bwd)
     flops, nbytes = sum(fl.values()), sum(by.values())
     p_mx, bw = 2.0 * peaks["bf16"] * 1e12, peaks["hbm"] * 1e9
     t_roof = max(flops / p_mx, nbytes / bw)
     sec = ms_step * 1e-3
-    moves = [n for n in ("route", "permute", "combine", "bwd_dout", "bwd_dx") if n in by]
-    mv_ms = sum(stage_ms.get(n, 0.0) for n in moves)
-    mv_bytes = sum(by[n] for n in moves if n in stage_ms)
+
+    def agg(names):
+        ms = sum(stage_ms.get(n, 0.0) for n in names)
+        b = sum(by[n] for n in names if n in stage_ms)
+        return (b / (ms * 1e-3) / bw) if ms > 0 else None
+    fwd_moves = [n for n in DATA_MOVEMENT if not n.startswith("bwd") and n in by]
+    moves = [n for n in DATA_MOVEMENT if n in by]
     return {"flops": flops, "bytes": nbytes, "t_roof_ms": t_roof * 1e3,
             "bound": "tensor" if flops / p_mx >= nbytes / bw else "hbm",
             "frac_of_roof": t_roof / sec, "tensor_frac": flops / sec / p_mx,
             "hbm_frac": nbytes / sec / bw,
-            "data_movement_hbm_frac": (mv_bytes / (mv_ms * 1e-3) / bw) if mv_ms > 0 else None,
-            "data_movement_kernels": moves}
+            "route_permute_combine_hbm_frac": agg(fwd_moves),
+            "data_movement_hbm_frac": agg(moves), "data_movement_kernels": moves}
 
 
 def _safe_layer_summary(case, stage_info, ms_step, peaks, bwd):
@@ -474,31 +518,42 @@ def run_ours(args, case):
     ms_e2e = e0.elapsed_time(e1)
     ms_e2e = max_over_ranks(ms_e2e, dev, world)
 
+    # the forward alone (inference: nothing saved for a backward), timed on its own
+    fwd_only = None
+    if bwd:
+        for _ in range(args.warmup):
+            moe.forward(x, logits, pw, ws=ws, out=out)
+        moe.profile_collect()
+        moe.profile_enable(True)
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            moe.forward(x, logits, pw, ws=ws, out=out)
+        f1.record(stream)
+        barrier()
+        moe.profile_enable(False)
+        fwd_stages = moe.profile_collect()
+        fwd_ms = max_over_ranks(f0.elapsed_time(f1), dev, world)
+        status |= moe.device_status(ws)
+        fwd_only = {"ms_per_step": fwd_ms / args.steps,
+                    "tokens_per_s": job_tokens_per_s(world, case.T, args.steps, fwd_ms),
+                    "stages_ms": {n: t / max(c, 1) for n, (t, c) in fwd_stages.items()}}
+
     peaks = _peaks()
     A = case.T * case.k
     mx_peak = 2.0 * peaks["bf16"]                      # MXFP8 dense = 2 x bf16 (nominal ratio)
-    fl = {"gateup": 4.0 * A * case.d * case.f, "down": 2.0 * A * case.d * case.f,
-          "bwd_dgrad_down": 2.0 * A * case.d * case.f,
-          "bwd_dgrad_gateup": 4.0 * A * case.d * case.f,
-          "bwd_wgrad": 6.0 * A * case.d * case.f}
+    fl = layer_flops(case, True)
     cd = dims.c()
     lib = moe.load()
     w_bytes = sum(lib.moe_weights_bytes(ctypes.byref(cd), i) for i in range(4))
-    alg_bytes = {
-        "route": 4 * case.T * case.E + 8 * A + 8 * A,
-        "permute": 2 * case.T * case.d + A * case.d * (1 + 1 / 32),
-        "combine": 4 * A * case.d + 2 * case.T * case.d,
-        "bwd_dout": 2 * case.T * case.d + A * case.d * (1 + 1 / 32),
-        "bwd_dx": 4 * A * case.d + 2 * case.T * case.d,
-        # G fp32 + saved g|u bf16 + h MX read, dg|du MX written, per assignment row
-        "bwd_swiglu": A * case.f * (4 + 4 + 1 + 2) * (1 + 1 / 64),
-    }
-    if bwd:
-        # rows inside some expert segment (the transposes and the wgrad K ranges cover these)
-        r_used = int(saved.bufs["pad_offsets"][case.E].item())
-        cols = 2 * case.d + 3 * case.f      # x^, w*dout^ (d), h^ (f), [dg|du]^ (2f)
-        alg_bytes["bwd_transpose"] = 2 * r_used * cols * (1 + 1 / 32)
-        alg_bytes["bwd_wgrad"] = 2 * case.E * 3 * case.d * case.f + r_used * cols * (1 + 1 / 32)
+    # rows the kernels touch beyond the A assignments (tile padding), from the layout
+    counts_h = (saved.bufs["counts"] if bwd else moe.workspace_view(
+        ws, dims, moe.OP_FORWARD, "counts", 4 * case.E).view(torch.int32)).cpu().numpy()
+    r_used = int(((counts_h + 127) // 128 * 128).sum())
+    r_out = int((counts_h // 128 * 128 + (counts_h % 128 + 31) // 32 * 32).sum())
+    alg_bytes = algorithmic_bytes(case, bwd)
+    impl_bytes = implementation_bytes(case, bwd, r_used, r_out)
     stage_info = {}
     for name, (tot_ms, n) in stages.items():
         s = {"ms_per_launch": tot_ms / max(n, 1), "launches": n}
@@ -506,21 +561,16 @@ def run_ours(args, case):
             s["alg_bytes"] = alg_bytes[name]
             s["gbs"] = alg_bytes[name] / (s["ms_per_launch"] * 1e-3) / 1e9
             s["frac_hbm"] = s["gbs"] / peaks["hbm"]
+            s["overhead_bytes"] = impl_bytes[name] - alg_bytes[name]
         if name in fl:
             s["flops"] = fl[name]
             s["tflops"] = fl[name] / (s["ms_per_launch"] * 1e-3) / 1e12
             s["frac_mxfp8"] = s["tflops"] / mx_peak
         stage_info[name] = s
     g = stage_info.get("gateup", {"ms_per_launch": float("nan"), "tflops": float("nan")})
-    tr = {}
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as fh:
-            tr = json.load(fh)
     roof_gateup = {"bound": "tensor", "kernel": "grouped_gemm_kernel<GATEUP_SWIGLU>",
                    "achieved": g["tflops"], "peak": mx_peak, "unit": "TFLOP/s",
-                   "frac": g["tflops"] / mx_peak,
-                   "traffic": tr.get("gateup_bytes_per_launch") if case.name == "dsv3" else None,
+                   "frac": g["tflops"] / mx_peak, "traffic": None,
                    "peak_note": f"2 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
                                 f"MXFP8:bf16 nominal ratio 2"}
     roofline = roof_gateup
@@ -530,16 +580,21 @@ def run_ours(args, case):
         w = stage_info["bwd_wgrad"]
         roofline = {"bound": "hbm", "kernel": "grouped_gemm_kernel<WGRAD_BF16> (2 launches)",
                     "achieved": w["gbs"], "peak": peaks["hbm"], "unit": "GB/s",
-                    "frac": w["gbs"] / peaks["hbm"],
-                    "traffic": tr.get("wgrad_bytes_per_stage") if case.name == "dsv3" else None,
+                    "frac": w["gbs"] / peaks["hbm"], "traffic": None,
                     "peak_note": f"{peaks['src']} copy bandwidth (read+write); pure-write "
                                  f"streams on this pool measured {WRITE_ONLY_GBS:.0f} GB/s",
                     "frac_of_write_only": w["gbs"] / WRITE_ONLY_GBS}
+    if fwd_only is not None:
+        fwd_only["frac_mxfp8"] = (fl["gateup"] + fl["down"]) / (
+            fwd_only["ms_per_step"] * 1e-3) / 1e12 / mx_peak
+        fwd_only["layer_roofline"] = _safe_layer_summary(
+            case, {n: {"ms_per_launch": v} for n, v in fwd_only["stages_ms"].items()},
+            fwd_only["ms_per_step"], peaks, False)
     ms_step = ms / args.steps
     value = job_tokens_per_s(world, case.T, args.steps, ms)
     fwd_ms = sum(v["ms_per_launch"] for k, v in stage_info.items() if not k.startswith("bwd"))
     bwd_ms = sum(v["ms_per_launch"] for k, v in stage_info.items() if k.startswith("bwd"))
-    layer_flops = sum(fl[k] for k in fl if bwd or not k.startswith("bwd"))
+    step_flops = sum(fl[k] for k in fl if bwd or not k.startswith("bwd"))
     launches = sum(KERNELS_PER_STAGE[k] * v["launches"] for k, v in stage_info.items())
     pass_name = "forward+backward" if bwd else "forward"
     line = {
@@ -555,15 +610,22 @@ def run_ours(args, case):
         "roofline_gateup": roof_gateup,
         "fwd_tokens_per_s": world * case.T / (fwd_ms * 1e-3),
         "bwd_tokens_per_s": world * case.T / (bwd_ms * 1e-3) if bwd else None,
-        "layer_tflops": layer_flops / (ms_step * 1e-3) / 1e12,
+        "layer_tflops": step_flops / (ms_step * 1e-3) / 1e12,
         "layer_roofline": _safe_layer_summary(case, stage_info, ms_step, peaks, bwd),
-        "layer_frac_mxfp8": layer_flops / (ms_step * 1e-3) / 1e12 / mx_peak,
+        "layer_frac_mxfp8": step_flops / (ms_step * 1e-3) / 1e12 / mx_peak,
+        "fwd_frac_mxfp8": (fl["gateup"] + fl["down"]) / (fwd_ms * 1e-3) / 1e12 / mx_peak,
+        "forward_only": fwd_only,
         "weights_gbs_fwd": w_bytes / (fwd_ms * 1e-3) / 1e9,
         "stages": stage_info,
         "gpu_launches": launches,
         "device_status": status,
         "e2e": {"value": job_tokens_per_s(world, case.T, args.steps, ms_e2e), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "per step: x, logits" + (", dOut" if bwd else "") + " copied in from "
+                        "pinned host memory; out" + (", dX, d(router weights)" if bwd else "") +
+                        " copied back" + ("; the weight gradients stay on the device (an "
+                                          "optimizer step consumes them there)" if bwd else "") +
+                        "; copies of step i+1 / i overlap step i's compute on two copy streams"},
         "clocks": clk.summary(),
         "padded_rows": moe.padded_rows(dims),
     }

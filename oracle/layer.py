@@ -196,13 +196,18 @@ def forward_bf16(x_bits, logits, k, score_fn, E, weights_fn, round_h=True):
 
 
 def backward(x_bits, logits, dout_bits, k, score_fn, E, weights_fn, experts=None,
-             want_dx=True, exact=False, prepared=None):
+             want_dx=True, exact=False, prepared=None, plain=False):
     """Oracle backward (quantised reading, see module docstring).
 
     Returns dict with dx [T,d] (fp64, contributions of the processed experts only when
     ``experts`` is given), dw [T,k], and dW = {e: (dWg [d,f], dWu [d,f], dWd [f,d])} for
     the processed experts.  ``prepared``: optional {e: ExpertWeights} whose quantised
     weight views are reused (weight preparation done ahead of time).
+
+    ``plain=True`` swaps in the textbook alternatives of the two readings, for comparison
+    only: the incoming-gradient operands of the weight gradients are quantised along the
+    tokens straight from their unquantised values (bf16 dg, du; w * dOut), and
+    d(combine weight) = <dOut_t, y_a> with the forward's expert output y_a.
     """
     T, d = x_bits.shape
     idx, w = rt.route(logits, k, score_fn)
@@ -230,7 +235,11 @@ def backward(x_bits, logits, dout_bits, k, score_fn, E, weights_fn, experts=None
         gb, ub = _bf(g, exact), _bf(u, exact)                 # saved pre-activations
         wd_k, wgu_k = W.bwd()
         G = dhat[t] @ wd_k.T                                  # [n, f]
-        dw[rows] = np.sum(G * hhat, axis=1)
+        if plain:
+            y = hhat @ W.fwd()[2].T
+            dw[rows] = np.sum(dout[t] * y, axis=1)
+        else:
+            dw[rows] = np.sum(G * hhat, axis=1)
         dh = wflat[rows][:, None] * G
         s = sigmoid(gb)
         dg = dh * ub * s * (1.0 + gb * (1.0 - s))
@@ -239,10 +248,14 @@ def backward(x_bits, logits, dout_bits, k, score_fn, E, weights_fn, experts=None
         if want_dx:
             np.add.at(dx, t, dgu_hat @ wgu_k.T)
         # weight gradients: the data path's MX operands requantised along the tokens
-        dy = wflat[rows][:, None] * dhat[t]
+        if plain:
+            dy = wflat[rows][:, None] * dout[t]
+            DGt, DUt = _tok_fake(_bf(dg, exact), exact), _tok_fake(_bf(du, exact), exact)
+        else:
+            dy = wflat[rows][:, None] * dhat[t]
+            DGt, DUt = _tok_fake(dgu_hat[:, :f], exact), _tok_fake(dgu_hat[:, f:], exact)
         Ht, DYt = _tok_fake(hhat, exact), _tok_fake(dy, exact)
         Xt = _tok_fake(xhat[t], exact)
-        DGt, DUt = _tok_fake(dgu_hat[:, :f], exact), _tok_fake(dgu_hat[:, f:], exact)
         dW[e] = (Xt.T @ DGt, Xt.T @ DUt, Ht.T @ DYt)
     return dict(idx=idx, w=w, counts=counts, offsets=offsets, perm=perm, inv=inv,
                 dx=dx, dw=dw.reshape(T, k), dW=dW)

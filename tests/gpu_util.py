@@ -66,3 +66,72 @@ def padded_rows_of(pad_offsets: np.ndarray, offsets: np.ndarray) -> np.ndarray:
     e = np.searchsorted(offsets, pos, side="right") - 1
     e = np.minimum(e, E - 1)
     return pad_offsets[e] + (pos - offsets[e])
+
+
+def canonical_scales(umma_buf, rows_total: int, K: int, rows) -> np.ndarray:
+    """Canonical [len(rows), K/32] scale bytes of the given rows of a [rows_total, K]
+    matrix whose scales are stored in the UMMA layout (documented in moe.h)."""
+    r = np.asarray(rows, dtype=np.int64)[:, None]
+    kb = np.arange(K // 32, dtype=np.int64)[None, :]
+    off = ((((r >> 7) * (K // 128) + (kb >> 2)) << 9) + ((r & 31) << 4)
+           + (((r & 127) >> 5) << 2) + (kb & 3))
+    return np.asarray(umma_buf, np.uint8)[off]
+
+
+def mx_values(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Dequantised float64 values of MX codes [n, K] with canonical scales [n, K/32]."""
+    from oracle import mxfp8 as omx
+    return omx.e4m3_decode(codes) * np.repeat(omx.e8m0_decode(scales), 32, axis=1)
+
+
+def expert_rows(pad_offsets: np.ndarray, counts: np.ndarray, e: int) -> np.ndarray:
+    """Padded-buffer row indices of expert e's assignments (in segment order)."""
+    return int(pad_offsets[e]) + np.arange(int(counts[e]))
+
+
+def pick_experts(counts: np.ndarray) -> dict:
+    """Experts whose rows exercise the tile edge cases: the most loaded one, one whose last
+    128-row tile holds fewer than 16 rows, one with a multiple of 128 rows, an empty one
+    (each only when the layout has one)."""
+    counts = np.asarray(counts)
+    out = {"hottest": int(np.argmax(counts))}
+    tail = [e for e in range(counts.size) if counts[e] % 128 and counts[e] % 128 < 16]
+    if tail:
+        out["short_last_tile"] = tail[0]
+    full = [e for e in range(counts.size) if counts[e] and counts[e] % 128 == 0]
+    if full:
+        out["multiple_of_128"] = full[0]
+    empty = [e for e in range(counts.size) if counts[e] == 0]
+    if empty:
+        out["empty"] = empty[0]
+    return out
+
+
+def assert_stage_close(got: np.ndarray, ref: np.ndarray, rel: float, what: str):
+    """Stage parity on identical operands: only the kernel's own fp32 arithmetic differs."""
+    err = rel_fro(got, ref)
+    print(f"  {what}: rel_fro {err:.3e}")
+    assert err <= rel, f"{what}: relative Frobenius error {err:.3e} > {rel:.1e}"
+
+
+def assert_codes_near(got_q, got_s, ref_q, ref_s, ref_vals, what: str, max_frac=1e-3):
+    """MX codes computed from fp32 (device) and fp64 (oracle) values of the same quantity:
+    equal except where the value sits on a rounding boundary.  At most ``max_frac`` of the
+    elements may differ; a differing code under an equal scale must be the neighbour of the
+    oracle's and the oracle's value must lie next to the midpoint of the two codes' values
+    (within 1e-4 relative: the fp32 evaluation's error is ~1e-6)."""
+    from oracle import mxfp8 as omx
+    got_q, ref_q = np.asarray(got_q), np.asarray(ref_q)
+    scale_eq = np.repeat(np.asarray(got_s) == np.asarray(ref_s), 32, axis=1)
+    bad = ~((got_q == ref_q) & scale_eq)
+    frac = bad.mean() if bad.size else 0.0
+    print(f"  {what}: {int(bad.sum())} of {bad.size} codes differ")
+    assert frac <= max_frac, f"{what}: {frac:.2e} of the codes differ"
+    sel = bad & scale_eq
+    if sel.any():
+        g, r = got_q[sel].astype(np.int64), ref_q[sel].astype(np.int64)
+        assert np.all(np.abs((g & 0x7F) - (r & 0x7F)) <= 1), what
+        sc = np.repeat(omx.e8m0_decode(np.asarray(ref_s)), 32, axis=1)[sel]
+        v = np.asarray(ref_vals)[sel] / sc
+        mid = 0.5 * (omx.e4m3_decode(got_q[sel]) + omx.e4m3_decode(ref_q[sel]))
+        assert np.all(np.abs(np.abs(v) - np.abs(mid)) <= 1e-4 * np.abs(v) + 1e-30), what

@@ -74,9 +74,16 @@ def test_layer_summary_closed_form():
     assert r["bound"] == ("tensor" if t_fl >= t_by else "hbm")
     assert r["tensor_frac"] == pytest.approx(r["flops"] / 4.05e-3 / 2e15)
     assert r["frac_of_roof"] == pytest.approx(r["t_roof_ms"] / 4.05)
+    # the survey's per-unit bytes: logits + idx/w + perm/inv; x + permuted MX rows; bf16
+    # expert outputs + out
     mv = (4 * case.T * case.E + 16 * A) + (2 * case.T * case.d + A * case.d * (1 + 1 / 32)) + \
-        (4 * A * case.d + 2 * case.T * case.d)
+        (2 * A * case.d + 2 * case.T * case.d)
     assert r["data_movement_hbm_frac"] == pytest.approx(mv / 0.55e-3 / 5e12)
+    assert r["route_permute_combine_hbm_frac"] == pytest.approx(mv / 0.55e-3 / 5e12)
+    impl = bench.implementation_bytes(case, True, rows_used=A + 1000, rows_out=A + 500)
+    alg = bench.algorithmic_bytes(case, True)
+    assert impl["combine"] - alg["combine"] == 2 * A * case.d     # fp32 instead of bf16 rows
+    assert impl["bwd_transpose"] > alg["bwd_transpose"]           # padded rows
     bwd_stages = dict(fwd_stages, bwd_dout=0.2, bwd_dgrad_down=1.3, bwd_swiglu=0.4,
                       bwd_dgrad_gateup=2.7, bwd_dx=0.3, bwd_transpose=1.0, bwd_wgrad=6.2)
     rb = bench.layer_summary(case, bwd_stages, 16.6, peaks, bwd=True)

@@ -1,14 +1,16 @@
-"""GPU parity of the backward pass (S8) against the fp64 oracle on the same quantised operands.
+"""GPU parity of the backward pass (S8) against the fp64 oracle, end to end from the raw
+inputs.
 
 dX and d(routing weights) must reach relative Frobenius error <= 2e-3 and max-abs <=
-3e-2*RMS.  The weight gradients reach relative Frobenius <= 2e-3 per expert matrix; their
-element-wise bound allows for requantisation decisions: the saved g, u (bf16) and dg, du
-(MX along f, then along the tokens) are computed values (fp32 on the GPU, fp64 in the
-oracle), so a value on a rounding boundary can land one code apart, and in a sum over an
-expert's tokens one such code moves an element by up to ~0.1*RMS (the oracle itself does
-this under 1e-6 relative noise).  Elements beyond 3e-2*RMS must be
-rare (<= 1e-4 of all weight-gradient elements) and below 0.25*RMS.  An expert without
-tokens gets an exactly zero weight gradient.
+3e-2*RMS.  The weight gradients reach relative Frobenius <= 2e-3 per expert matrix.  The
+strict element-wise bound for them is checked stage by stage, on identical operands, in
+test_gpu_stage_parity.py; end to end it cannot hold element by element: the saved g, u
+(bf16) and dg, du (MX along f, then along the tokens) are computed values (fp32 on the
+GPU, fp64 in the oracle), so a value on a rounding boundary can land one code apart, and
+in a sum over an expert's tokens one such code moves an element by up to ~0.1*RMS (the
+oracle does the same to itself under 1e-6 relative noise).  As a documented extra, the
+end-to-end elements beyond 3e-2*RMS must be rare (<= 1e-4 of all weight-gradient
+elements) and below 0.25*RMS.  An expert without tokens gets an exactly zero gradient.
 """
 import numpy as np
 import pytest
@@ -69,6 +71,10 @@ def _check(moe, case, tokens=None, experts=None):
     dw = to_np(grads["dw_route"]).astype(np.float64)
     print(f"{case.name} dw_route:")
     assert_close_out(dw[rows], ref["dw"][rows])
+    if experts is not None:           # every assignment of the listed experts
+        sel = np.isin(ref["idx"].ravel(), experts)
+        print(f"{case.name} dw_route of experts {experts} ({int(sel.sum())} assignments):")
+        assert_close_out(dw.ravel()[sel], ref["dw"].ravel()[sel])
     names = ("dWg", "dWu", "dWd")
     n_el = n_out = 0
     worst = 0.0
@@ -103,9 +109,14 @@ def test_backward_mid_full(moe):
     _check(moe, synth.CONFIGS["mid"])
 
 
-def test_backward_dsv3_sampled(moe):
+def test_backward_dsv3_experts(moe):
+    # the tile edge cases of the layout: most loaded expert, a last tile of < 16 rows, a
+    # multiple of 128 rows; dX and d(routing weights) on the tokens routed to them
+    from tests.gpu_util import pick_experts
     case = synth.CONFIGS["dsv3_bwd"]
-    _check(moe, case, tokens=np.array([1234]), experts=None)
+    idx = np.argsort(-synth.make_logits(case), axis=1, kind="stable")[:, :case.k]
+    picks = sorted(set(pick_experts(np.bincount(idx.ravel(), minlength=case.E)).values()))
+    _check(moe, case, tokens=np.array([1234]), experts=picks)
 
 
 def test_backward_edge_cases(moe):

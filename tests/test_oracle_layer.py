@@ -197,6 +197,23 @@ def test_quantised_backward_with_identity_quantisers_is_exact():
             assert np.allclose(res["dW"][e][m], dW[e][m], rtol=1e-11, atol=1e-11)
 
 
+def test_plain_readings_coincide_in_exact_arithmetic():
+    # <G, h> and <dOut, y> are the same number when no operand is quantised, and so are the
+    # two choices of weight-gradient operands: the readings differ only by quantisation
+    case = _case(T=24, d=64, f=64, E=4, k=2, score=1, bias="normal0.5", seed=6)
+    x, lg, wfn = _inputs(case)
+    dout = synth.make_dout(case)
+    a = L.backward(x, lg, dout, case.k, 1, case.E, wfn, exact=True)
+    b = L.backward(x, lg, dout, case.k, 1, case.E, wfn, exact=True, plain=True)
+    assert np.allclose(a["dw"], b["dw"], rtol=1e-11, atol=1e-11)
+    for e in range(case.E):
+        for m in range(3):
+            assert np.allclose(a["dW"][e][m], b["dW"][e][m], rtol=1e-11, atol=1e-11)
+    q = L.backward(x, lg, dout, case.k, 1, case.E, wfn)
+    p = L.backward(x, lg, dout, case.k, 1, case.E, wfn, plain=True)
+    assert not np.allclose(q["dw"], p["dw"], rtol=1e-6, atol=0)   # quantised: they differ
+
+
 def test_quantised_backward_close_to_exact_and_empty_expert_zero():
     case = _case(T=64, d=128, f=64, E=6, k=2, score=0, bias="skew1.5", seed=5)
     x, lg, wfn = _inputs(case)
@@ -215,6 +232,157 @@ def test_quantised_backward_close_to_exact_and_empty_expert_zero():
                 assert not np.any(q["dW"][e][m])
             else:
                 assert rel(q["dW"][e][m], ex["dW"][e][m]) < 0.15
+
+
+def _brute_backward(x_bits, logits, dout_bits, k, score_fn, E, wfn):
+    """Per-token, per-slot loop written from the definitions of the quantised backward:
+    every GEMM operand MX-quantised along that GEMM's reduction axis, the saved g, u in
+    bf16, a straight-through quantiser.  The weight gradients are sums of per-token outer
+    products of operands quantised along the tokens of the expert's segment (blocks of 32
+    rows counted from the segment start, missing rows zero), each block quantised on its
+    own here.  Shares nothing with the oracle but the basic quantiser along a vector."""
+    fq = mx.fake_quantize_mx
+    x = L.bf16_bits_to_f64(x_bits)
+    dout = L.bf16_bits_to_f64(dout_bits)
+    T, d = x.shape
+    dx = np.zeros((T, d))
+    dw = np.zeros((T, k))
+    per_expert = {e: [] for e in range(E)}      # (t, xh, hh, dy, dgu_hat) in token order
+    qcache = {}
+
+    def wq(e):
+        """Expert e's weights quantised once, column by column / row by row as each GEMM
+        reduces: Wg, Wu columns along d; W_down rows along d (dgrad); [Wg|Wu] rows along 2f."""
+        if e not in qcache:
+            Wg, Wu, Wd = wfn(e)
+            Wcat = np.concatenate([Wg, Wu], axis=1)
+            qcache[e] = ([fq(Wg[:, n]) for n in range(Wg.shape[1])],
+                         [fq(Wu[:, n]) for n in range(Wu.shape[1])],
+                         [fq(Wd[i, :]) for i in range(Wd.shape[0])],
+                         [fq(Wcat[r, :]) for r in range(Wcat.shape[0])])
+        return qcache[e]
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-float(logits[t, e]), e))[:k]
+        sel = np.array([float(logits[t, e]) for e in order])
+        if score_fn == 0:
+            w = np.exp(sel - sel.max()); w /= w.sum()
+        else:
+            s = 1 / (1 + np.exp(-sel)); w = s / s.sum()
+        xh = fq(x[t])                            # x along d
+        dh_t = fq(dout[t])                       # dOut along d
+        for j, e in enumerate(order):
+            qg, qu, qd, qcat = wq(e)
+            g = np.array([xh @ c for c in qg])                               # Wg along d
+            u = np.array([xh @ c for c in qu])
+            hh = fq(g / (1 + np.exp(-g)) * u)                             # h along f
+            f = g.size
+            # dgrad of the down projection: K = d, W_down's rows quantised along d
+            G = np.array([dh_t @ r for r in qd])
+            dw[t, j] = G @ hh
+            gb, ub = L.bf16_round(g), L.bf16_round(u)
+            sg = 1 / (1 + np.exp(-gb))
+            dh = w[j] * G
+            dg = dh * ub * sg * (1 + gb * (1 - sg))
+            du = dh * gb * sg
+            dgu = fq(np.concatenate([dg, du]))                               # along 2f
+            dx[t] += np.array([dgu @ r for r in qcat])           # [Wg|Wu] rows along 2f
+            per_expert[e].append((xh, hh, w[j] * dh_t, dgu))
+    dW = {}
+    for e in range(E):
+        Wg, Wu, Wd = wfn(e)
+        f = Wg.shape[1]
+        rows = per_expert[e]
+        dWg, dWu, dWd = np.zeros((d, f)), np.zeros((d, f)), np.zeros((f, d))
+        for b0 in range(0, len(rows), 32):       # blocks of 32 tokens from the segment start
+            blk = rows[b0:b0 + 32]
+            pad = 32 - len(blk)
+
+            def tokq(vecs):
+                m = np.vstack([np.stack(vecs), np.zeros((pad, len(vecs[0])))])
+                return np.stack([fq(m[:, c]) for c in range(m.shape[1])], axis=1)
+            X = tokq([r[0] for r in blk])
+            H = tokq([r[1] for r in blk])
+            DY = tokq([r[2] for r in blk])
+            DG = tokq([r[3][:f] for r in blk])
+            DU = tokq([r[3][f:] for r in blk])
+            for i in range(32):                   # per-token outer products
+                dWg += np.outer(X[i], DG[i])
+                dWu += np.outer(X[i], DU[i])
+                dWd += np.outer(H[i], DY[i])
+        dW[e] = (dWg, dWu, dWd)
+    return dx, dw, dW
+
+
+_BWD_CASES = [dict(T=100, d=64, f=96, E=3, k=2, score=1, bias="normal0.5", seed=31),
+              dict(T=90, d=64, f=64, E=6, k=2, score=0, bias="skew1.5", seed=32)]
+
+
+def _bwd_compare(case, res=None):
+    x, lg, wfn = _inputs(case)
+    dout = synth.make_dout(case)
+    if res is None:
+        res = L.backward(x, lg, dout, case.k, case.score_fn, case.E, wfn)
+    dx, dw, dW = _brute_backward(x, lg, dout, case.k, case.score_fn, case.E, wfn)
+    worst = max(np.max(np.abs(res["dx"] - dx)) / np.max(np.abs(dx)),
+                np.max(np.abs(res["dw"] - dw)) / np.max(np.abs(dw)))
+    for e in range(case.E):
+        for m in range(3):
+            ref = dW[e][m]
+            den = max(np.max(np.abs(ref)), 1e-300)
+            worst = max(worst, np.max(np.abs(res["dW"][e][m] - ref)) / den)
+    return worst
+
+
+@pytest.mark.parametrize("kw", _BWD_CASES)
+def test_quantised_backward_matches_bruteforce(kw):
+    case = _case(**kw)
+    counts = np.bincount(rt.topk_select(synth.make_logits(case), case.k).ravel(),
+                         minlength=case.E)
+    assert (counts > 32).sum() >= 2 and np.any(counts % 32)    # several blocks, ragged ends
+    assert _bwd_compare(case) <= 1e-12
+
+
+def _mutants():
+    """Plausible mistakes in the quantisation sites, each planted in the oracle (CPU)."""
+    orig_tok, orig_fq, orig_bwd = L._tok_fake, L._fq, L.ExpertWeights.bwd
+
+    def tok_misaligned(v, exact=False):          # blocks not restarting at the segment start
+        pad = np.zeros((5, v.shape[1]))
+        return orig_tok(np.vstack([pad, v]), exact)[5:]
+
+    def tok_wrong_axis(v, exact=False):          # weight-gradient operands along features
+        return orig_fq(v, exact)
+
+    def dout_wrong_axis(v, exact=False):         # dOut quantised along the tokens
+        if not exact and getattr(v, "shape", (0,))[-1] == 64 and v.shape[0] in (90, 100):
+            n = v.shape[0]
+            padded = np.vstack([np.asarray(v), np.zeros((128 - n, 64))])
+            return mx.fake_quantize_mx(padded.T).T[:n]
+        return orig_fq(v, exact)
+
+    def forward_wd_copy(self):                   # the forward copy of W_down in the backward
+        wd_k, wgu_k = orig_bwd(self)
+        return _fq_t(self.wd.T, self.exact).T, wgu_k
+
+    def _fq_t(v, exact):
+        return orig_fq(v, exact)
+
+    def no_bf16_save(v, exact):                  # g, u kept in full precision
+        return np.asarray(v, np.float64)
+    return [("_tok_fake", tok_misaligned), ("_tok_fake", tok_wrong_axis),
+            ("_fq", dout_wrong_axis), ("ExpertWeights.bwd", forward_wd_copy),
+            ("_bf", no_bf16_save)]
+
+
+@pytest.mark.parametrize("which", range(5))
+def test_bruteforce_catches_planted_mistakes(monkeypatch, which):
+    name, fn = _mutants()[which]
+    case = _case(**_BWD_CASES[0])
+    if name == "ExpertWeights.bwd":
+        monkeypatch.setattr(L.ExpertWeights, "bwd", fn)
+    else:
+        monkeypatch.setattr(L, name, fn)
+    assert _bwd_compare(case) > 1e-6, name
 
 
 def test_bf16_round_matches_torch_on_fp32_values():

@@ -14,7 +14,7 @@ from typing import Optional
 
 from . import _lib
 from ._lib import (MoeDims, MoeError, MoeSaved, MoeWeights, OP_BACKWARD, OP_FORWARD, OP_ROUTE,
-                   SAVED_FIELDS, WEIGHT_FIELDS, check, load)
+                   SAVED_FIELDS, WEIGHT_FIELDS, WS_BUFFERS, check, load)
 
 SCORE_SOFTMAX_TOPK = 0
 SCORE_SIGMOID_RENORM = 1
@@ -22,7 +22,7 @@ SCORE_SIGMOID_RENORM = 1
 __all__ = ["Dims", "PreparedWeights", "Saved", "load", "MoeError", "workspace",
            "route_layout", "mxfp8_quantize", "prepare_weights", "forward", "backward",
            "grouped_gemm_mx", "device_status", "padded_rows", "umma_scale_bytes",
-           "min_tokens_for_waves", "profile_enable", "profile_collect",
+           "min_tokens_for_waves", "workspace_view", "profile_enable", "profile_collect",
            "SCORE_SOFTMAX_TOPK", "SCORE_SIGMOID_RENORM"]
 
 
@@ -80,6 +80,14 @@ def workspace(dims: Dims, op: int, device="cuda"):
     if n == 0:
         raise MoeError(2, "moe_workspace_bytes")
     return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def workspace_view(ws, dims: Dims, op: int, name: str, nbytes: int):
+    """A uint8 view of ``nbytes`` of an internal workspace buffer (moe_workspace_offset)."""
+    off = load().moe_workspace_offset(ctypes.byref(dims.c()), op, WS_BUFFERS[name])
+    if off < 0:
+        raise MoeError(1, f"moe_workspace_offset({name})")
+    return ws[off:off + nbytes]
 
 
 def route_layout(logits, k: int, score_fn: int = SCORE_SOFTMAX_TOPK, ws=None, stream=None):

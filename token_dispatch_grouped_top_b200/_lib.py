@@ -15,6 +15,11 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned
 
 OP_ROUTE, OP_FORWARD, OP_BACKWARD = 0, 1, 2
 
+# internal workspace buffers that moe_workspace_offset locates (moe_ws_buffer)
+WS_BUFFERS = {"mtile": 0, "y": 1, "dout_q": 2, "dout_s": 3, "g": 4, "dgu_q": 5, "dgu_s": 6,
+              "dxa": 7, "xt_q": 8, "xt_s": 9, "ht_q": 10, "ht_s": 11, "gt_q": 12, "gt_s": 13,
+              "yt_q": 14, "yt_s": 15, "counts": 16}
+
 STAGES = ["route", "permute", "gateup", "down", "combine", "bwd_dout", "bwd_dgrad_down",
           "bwd_dgrad_gateup", "bwd_dx", "bwd_transpose", "bwd_wgrad", "bwd_swiglu"]
 
@@ -45,6 +50,7 @@ SIGNATURES = {
     "moe_saved_bytes": (c_i64, [ctypes.POINTER(MoeDims), c_i32]),
     "moe_workspace_bytes": (c_sz, [ctypes.POINTER(MoeDims), c_i32]),
     "moe_min_tokens_for_waves": (c_i64, [c_i32, c_i32, c_i32, c_i32, c_i64]),
+    "moe_workspace_offset": (c_i64, [ctypes.POINTER(MoeDims), c_i32, c_i32]),
     "moe_status_string": (ctypes.c_char_p, [c_i32]),
     "moe_route_layout": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                  c_vp, c_vp, c_vp, c_sz, c_vp]),

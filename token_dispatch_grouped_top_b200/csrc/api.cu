@@ -388,6 +388,32 @@ size_t moe_workspace_bytes(const moe_dims* dims, int32_t op) {
   return static_cast<size_t>(ws_layout(dims, op).total);
 }
 
+int64_t moe_workspace_offset(const moe_dims* D, int32_t op, int32_t buffer) {
+  if (check_dims(D) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_BACKWARD) return -1;
+  const WsLayout L = ws_layout(D, op);
+  if (buffer == MOE_WS_MTILE) return L.mtile;
+  if (op == MOE_OP_FORWARD && buffer == MOE_WS_Y) return L.y;
+  if (op == MOE_OP_FORWARD && buffer == MOE_WS_COUNTS) return L.counts;
+  if (op != MOE_OP_BACKWARD) return -1;
+  switch (buffer) {
+    case MOE_WS_DOUT_Q: return L.dq;
+    case MOE_WS_DOUT_S: return L.ds;
+    case MOE_WS_G: return L.gbuf;
+    case MOE_WS_DGU_Q: return L.dgu_q;
+    case MOE_WS_DGU_S: return L.dgu_s;
+    case MOE_WS_DXA: return L.dxa;
+    case MOE_WS_XT_Q: return L.xt_q;
+    case MOE_WS_XT_S: return L.xt_s;
+    case MOE_WS_HT_Q: return L.ht_q;
+    case MOE_WS_HT_S: return L.ht_s;
+    case MOE_WS_GT_Q: return L.gt_q;
+    case MOE_WS_GT_S: return L.gt_s;
+    case MOE_WS_YT_Q: return L.yt_q;
+    case MOE_WS_YT_S: return L.yt_s;
+    default: return -1;
+  }
+}
+
 int64_t moe_min_tokens_for_waves(int32_t num_sms, int32_t waves, int32_t tile_m, int32_t tile_n,
                                  int64_t n_cols) {
   if (num_sms <= 0 || waves <= 0 || tile_m <= 0 || tile_n <= 0 || n_cols <= 0) return -1;
