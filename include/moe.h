@@ -60,7 +60,12 @@ typedef enum {
 
 typedef enum { MOE_SCORE_SOFTMAX_TOPK = 0, MOE_SCORE_SIGMOID_RENORM = 1 } moe_score_fn;
 
-typedef enum { MOE_OP_ROUTE = 0, MOE_OP_FORWARD = 1, MOE_OP_BACKWARD = 2 } moe_op;
+typedef enum {
+  MOE_OP_ROUTE = 0,
+  MOE_OP_FORWARD = 1,
+  MOE_OP_BACKWARD = 2,
+  MOE_OP_FORWARD_BF16 = 3  /* moe_forward_bf16 */
+} moe_op;
 
 typedef struct {
   int64_t T;         /* tokens */
@@ -214,6 +219,26 @@ moe_status moe_forward(const moe_dims* dims, const moe_weights* w, const uint16_
                        const float* logits, uint16_t* out, const moe_saved* saved,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* ---- the layer's BF16 variant ----------------------------------------------------------
+ * Article §03 (MoE-layer results are reported with BF16 as well as MXFP8 operands).  The
+ * same layer with bf16 operands throughout and no MX quantisation: g = x Wg, u = x Wu,
+ * h = bf16(silu(g) * u) (round to nearest even), y = h Wd, out_t = sum_j w[t,j] y_{t*k+j}
+ * (fp32 accumulation, bf16 output), on the 5th-generation tensor cores with
+ * tcgen05.mma kind::f16.
+ *
+ * moe_prepare_weights_bf16: W_gate, W_up [E,d,f], W_down [E,f,d] bf16 (x @ W convention) ->
+ * wgu_t [E*2f, d] bf16 (per expert, 128-row blocks alternate W_gate^T block j and W_up^T
+ * block j, as the MX layout) and wd_t [E*d, f] (W_down^T per expert); 2*E*2f*d and
+ * 2*E*d*f bytes.  Setup, not part of the layer's step.
+ * moe_forward_bf16: x [T,d] bf16, logits [T,E] fp32 -> out [T,d] bf16; routing as
+ * moe_route_layout; ws: moe_workspace_bytes(MOE_OP_FORWARD_BF16). */
+moe_status moe_prepare_weights_bf16(const moe_dims* dims, const uint16_t* w_gate,
+                                    const uint16_t* w_up, const uint16_t* w_down,
+                                    uint16_t* wgu_t, uint16_t* wd_t, void* stream);
+moe_status moe_forward_bf16(const moe_dims* dims, const uint16_t* wgu_t, const uint16_t* wd_t,
+                            const uint16_t* x, const float* logits, uint16_t* out, void* ws,
+                            size_t ws_bytes, void* stream);
+
 /* ---- S8: backward ---------------------------------------------------------------------
  * Article §01/§02 (backward = pull reverse-combine + push reverse-dispatch).
  * dout [T,d] bf16 + saved -> dx [T,d] bf16, dw_route [T,k] fp32 (d loss / d topk_w),
@@ -224,6 +249,22 @@ moe_status moe_backward(const moe_dims* dims, const moe_weights* w, const moe_sa
                         const uint16_t* dout, uint16_t* dx, float* dw_route, uint16_t* dWg,
                         uint16_t* dWu, uint16_t* dWd, void* ws, size_t ws_bytes,
                         void* stream);
+
+/* ---- router backward -------------------------------------------------------------------
+ * Article lead and §01 (the router picks each token's experts at every training step, so
+ * training needs the gradient that reaches the router).  d(loss)/d(logits) [T,E] fp32 from
+ * d(loss)/d(combine weights) dw_route [T,k] (the output of moe_backward), the logits [T,E]
+ * and the selected experts topk_idx [T,k] of the forward.  The selection is piecewise
+ * constant, so the E - k unselected logits of a token get exactly 0; the k selected ones
+ * get the chain rule of the score function (softmax over the selected logits:
+ * w_i (dw_i - sum_j w_j dw_j); sigmoid renormalised: s_i (1 - s_i)(dw_i - sum_j w_j dw_j)/S
+ * with S = sum_j s_j), the weights recomputed from the logits as moe_route_layout forms
+ * them.  dims->d and dims->f only have to satisfy the shape rules.  status (nullable,
+ * device int32): an expert id outside [0, E) latches MOE_ERR_DEVICE_BOUNDS there and leaves
+ * that token's row unwritten. */
+moe_status moe_router_backward(const moe_dims* dims, const float* logits,
+                               const int32_t* topk_idx, const float* dw_route, float* dlogits,
+                               int32_t* status, void* stream);
 
 /* ---- grouped block-scaled GEMM (the engine of S4/S5, exposed for direct use) ----------
  * For each group g and each row r in [128*mtile_prefix[g], 128*mtile_prefix[g+1]):
@@ -239,6 +280,25 @@ moe_status moe_grouped_gemm_mx(int32_t G, int64_t rows_a, int32_t N, int32_t K,
                                const uint8_t* a_q, const uint8_t* a_s, const uint8_t* b_q,
                                const uint8_t* b_s, float* d_out, void* ws, size_t ws_bytes,
                                void* stream);
+
+/* ---- failure-detection test hook -------------------------------------------------------
+ * Article §02 (device-local counters signal that a minibatch of dispatched rows is ready;
+ * the grouped GEMM waits on them).  For tests of the bounded wait only: from the next
+ * moe_forward / moe_backward on, the dispatch never publishes minibatch `minibatch` (its
+ * rows are still written); the GEMM's wait for it gives up after its time limit (2 s),
+ * latches MOE_ERR_DEVICE_TIMEOUT in the workspace and the CTAs leave cleanly, so the
+ * results of that call are garbage but the context stays usable.  A negative value turns
+ * the hook off (the default). */
+moe_status moe_debug_withhold_ready(int32_t minibatch);
+
+/* ---- grouped bf16 GEMM (the engine of the BF16 variant, exposed for direct use) --------
+ * As moe_grouped_gemm_mx with bf16 operands A [rows_a, K] and B [G*N, K] (row-major, K
+ * contiguous) and no scales: D[r, n] = sum_k A[r,k] * B[g*N + n, k], fp32 accumulation and
+ * output.  N % 256 == 0, K % 64 == 0, rows_a % 128 == 0; ws >= 256 bytes. */
+moe_status moe_grouped_gemm_bf16(int32_t G, int64_t rows_a, int32_t N, int32_t K,
+                                 const int32_t* mtile_prefix, const int32_t* rows_valid,
+                                 const uint16_t* a, const uint16_t* b, float* d_out, void* ws,
+                                 size_t ws_bytes, void* stream);
 
 /* ---- per-stage timing (measurement support) ------------------------------------------
  * Stage ids of moe_forward / moe_backward launches. */

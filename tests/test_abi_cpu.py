@@ -115,3 +115,41 @@ def test_wave_rule_reproduces_minibatch_figure(lib):
                                         2 * g["intermediate"]) == g["min_tokens"]
     assert lib.moe_min_tokens_for_waves(148, 1, 128, 256, 2 * 2048) == 1184
     assert lib.moe_min_tokens_for_waves(0, 1, 128, 256, 4096) == -1
+
+
+def test_workspace_offsets(lib):
+    # every internal buffer lies inside its operation's workspace, 256-byte aligned; the
+    # ones an operation does not have are -1
+    D = _dims(T=4096, d=2048, f=1536, E=64, k=6, s=0)
+    from token_dispatch_grouped_top_b200._lib import WS_BUFFERS
+    R = lib.moe_padded_rows(ctypes.byref(D))
+    for op, names in ((1, ("mtile", "y", "counts")),
+                      (2, ("mtile", "dout_q", "dout_s", "g", "dgu_q", "dgu_s", "dxa", "xt_q",
+                           "xt_s", "ht_q", "ht_s", "gt_q", "gt_s", "yt_q", "yt_s")),
+                      (3, ("mtile", "y", "counts"))):
+        total = lib.moe_workspace_bytes(ctypes.byref(D), op)
+        for n in names:
+            off = lib.moe_workspace_offset(ctypes.byref(D), op, WS_BUFFERS[n])
+            assert 0 < off < total and off % 256 == 0, (op, n)
+    assert lib.moe_workspace_offset(ctypes.byref(D), 1, WS_BUFFERS["dxa"]) == -1
+    assert lib.moe_workspace_offset(ctypes.byref(D), 2, WS_BUFFERS["y"]) == -1
+    assert lib.moe_workspace_offset(ctypes.byref(D), 4, 0) == -1
+    # the forward's expert outputs hold R fp32 rows of d
+    y = lib.moe_workspace_offset(ctypes.byref(D), 1, WS_BUFFERS["y"])
+    assert y + 4 * R * 2048 <= lib.moe_workspace_bytes(ctypes.byref(D), 1)
+
+
+def test_bf16_variant_and_router_backward_checks(lib):
+    D = _dims(T=16, d=256, f=256, E=8, k=2, s=0)
+    assert lib.moe_forward_bf16(ctypes.byref(D), None, None, None, None, None, None, 0,
+                                None) == 1
+    assert lib.moe_prepare_weights_bf16(ctypes.byref(D), None, None, None, None, None,
+                                        None) == 1
+    # K must be a multiple of 64 bf16 elements (one 128-byte swizzled row)
+    assert lib.moe_grouped_gemm_bf16(2, 128, 256, 96, None, None, None, None, None, None, 0,
+                                     None) == 2
+    assert lib.moe_router_backward(ctypes.byref(D), None, None, None, None, None, None) == 1
+    bad = _dims(T=16, d=256, f=256, E=8, k=9, s=0)
+    assert lib.moe_router_backward(ctypes.byref(bad), None, None, None, None, None, None) == 2
+    assert lib.moe_workspace_bytes(ctypes.byref(D), 3) > 0
+    assert lib.moe_debug_withhold_ready(-1) == 0

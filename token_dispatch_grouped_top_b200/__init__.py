@@ -13,15 +13,17 @@ from dataclasses import dataclass, field
 from typing import Optional
 
 from . import _lib
-from ._lib import (MoeDims, MoeError, MoeSaved, MoeWeights, OP_BACKWARD, OP_FORWARD, OP_ROUTE,
-                   SAVED_FIELDS, WEIGHT_FIELDS, WS_BUFFERS, check, load)
+from ._lib import (MoeDims, MoeError, MoeSaved, MoeWeights, OP_BACKWARD, OP_FORWARD,
+                   OP_FORWARD_BF16, OP_ROUTE, SAVED_FIELDS, WEIGHT_FIELDS, WS_BUFFERS, check,
+                   load)
 
 SCORE_SOFTMAX_TOPK = 0
 SCORE_SIGMOID_RENORM = 1
 
 __all__ = ["Dims", "PreparedWeights", "Saved", "load", "MoeError", "workspace",
            "route_layout", "mxfp8_quantize", "prepare_weights", "forward", "backward",
-           "grouped_gemm_mx", "device_status", "padded_rows", "umma_scale_bytes",
+           "grouped_gemm_mx", "grouped_gemm_bf16", "prepare_weights_bf16", "forward_bf16",
+           "router_backward", "device_status", "padded_rows", "umma_scale_bytes",
            "min_tokens_for_waves", "workspace_view", "profile_enable", "profile_collect",
            "SCORE_SOFTMAX_TOPK", "SCORE_SIGMOID_RENORM"]
 
@@ -219,6 +221,68 @@ def backward(dout, weights: PreparedWeights, saved: Saved, ws=None, stream=None,
                               _ptr(outs["dWg"]), _ptr(outs["dWu"]), _ptr(outs["dWd"]), _ptr(ws),
                               ws.numel(), _stream(stream)), "moe_backward")
     return outs
+
+
+def router_backward(logits, topk_idx, dw_route, score_fn: int = SCORE_SOFTMAX_TOPK,
+                    status=None, stream=None):
+    """d(loss)/d(logits) [T, E] fp32 from d(loss)/d(combine weights) [T, k]."""
+    torch = _torch()
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    dims = Dims(T, 256, 256, E, k, score_fn)
+    dl = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    check(load().moe_router_backward(ctypes.byref(dims.c()), _ptr(logits.contiguous()),
+                                     _ptr(topk_idx.contiguous()), _ptr(dw_route.contiguous()),
+                                     _ptr(dl), _ptr(status), _stream(stream)),
+          "moe_router_backward")
+    return dl
+
+
+@dataclass
+class PreparedWeightsBf16:
+    dims: Dims
+    wgu_t: object = None     # [E*2f, d] bf16, gate/up interleaved in 128-row blocks
+    wd_t: object = None      # [E*d, f] bf16
+
+
+def prepare_weights_bf16(w_gate, w_up, w_down, dims: Dims, stream=None) -> PreparedWeightsBf16:
+    """bf16 W_gate/W_up [E,d,f], W_down [E,f,d] -> the BF16 variant's GEMM layouts."""
+    torch = _torch()
+    dev = w_gate.device
+    pw = PreparedWeightsBf16(dims)
+    pw.wgu_t = torch.empty((dims.E * 2 * dims.f, dims.d), dtype=torch.bfloat16, device=dev)
+    pw.wd_t = torch.empty((dims.E * dims.d, dims.f), dtype=torch.bfloat16, device=dev)
+    check(load().moe_prepare_weights_bf16(ctypes.byref(dims.c()), _ptr(w_gate.contiguous()),
+                                          _ptr(w_up.contiguous()), _ptr(w_down.contiguous()),
+                                          _ptr(pw.wgu_t), _ptr(pw.wd_t), _stream(stream)),
+          "moe_prepare_weights_bf16")
+    return pw
+
+
+def forward_bf16(x, logits, weights: PreparedWeightsBf16, ws=None, out=None, stream=None):
+    """The layer's BF16 variant on the device.  Returns out bf16 [T,d]."""
+    torch = _torch()
+    dims = weights.dims
+    ws = workspace(dims, OP_FORWARD_BF16, x.device) if ws is None else ws
+    out = torch.empty((dims.T, dims.d), dtype=torch.bfloat16, device=x.device) if out is None \
+        else out
+    check(load().moe_forward_bf16(ctypes.byref(dims.c()), _ptr(weights.wgu_t),
+                                  _ptr(weights.wd_t), _ptr(x), _ptr(logits), _ptr(out), _ptr(ws),
+                                  ws.numel(), _stream(stream)), "moe_forward_bf16")
+    return out
+
+
+def grouped_gemm_bf16(mtile_prefix, a, b, N: int, rows_valid=None, ws=None, stream=None):
+    """D[r, n] = sum_k A[r,k] B[g*N+n, k] with bf16 A [rows, K], B [G*N, K]; fp32 [rows, N]."""
+    torch = _torch()
+    G = mtile_prefix.numel() - 1
+    rows, K = a.shape
+    ws = torch.zeros(256, dtype=torch.uint8, device=a.device) if ws is None else ws
+    d = torch.zeros((rows, N), dtype=torch.float32, device=a.device)
+    check(load().moe_grouped_gemm_bf16(G, rows, N, K, _ptr(mtile_prefix), _ptr(rows_valid),
+                                       _ptr(a), _ptr(b), _ptr(d), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "moe_grouped_gemm_bf16")
+    return d
 
 
 def grouped_gemm_mx(mtile_prefix, a_q, a_s, b_q, b_s, N: int, K: int, rows_valid=None,

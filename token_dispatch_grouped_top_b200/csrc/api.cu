@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -173,10 +174,16 @@ struct Carve {
   }
 };
 
+// Tile counters of the grouped GEMM launches, in the workspace header (zeroed per call).
+enum : int64_t { kCtrFwdGateUp = 72, kCtrFwdDown = 76, kCtrBwdDgradDown = 72,
+                 kCtrBwdDgradGateUp = 76, kCtrBwdWgrad0 = 80, kCtrBwdWgrad1 = 84,
+                 kCtrGeneric = 72 };
+
 struct WsLayout {
-  // header: [0] status word; [64] tile counter; [68] done counter; [128 ...) flags
+  // header: [0] status word; [64] routing tile counter; [68] routing done counter;
+  // [72, 96) grouped-GEMM tile counters; [128 ...) flags
   int64_t zero_begin = 64, zero_bytes = 0;
-  int64_t flags = 0, agg = 0, incl = 0, rank = 0, mtile = 0;
+  int64_t flags = 0, agg = 0, incl = 0, rank = 0, mtile = 0, ready = 0, order = 0;
   int64_t idx = 0, w = 0, counts = 0, offsets = 0, perm = 0, inv = 0, pad = 0;
   int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0;
   int64_t tq = 0, ts = 0;  // per-token MX copy of x (forward) or dout (backward)
@@ -191,6 +198,17 @@ int64_t padded_rows(const moe_dims* D) {
   return align_up(A + static_cast<int64_t>(D->E) * 127, 128);
 }
 
+// Readiness minibatch of a token-row GEMM with n_cols output columns: the article's rule
+// that a minibatch should fill at least two full waves of 128 x 256 tiles on the SMs
+// (moe_min_tokens_for_waves), rounded up to whole 128-row tiles.
+int ready_rows(int num_sms, int64_t n_cols) {
+  const int64_t m = moe_min_tokens_for_waves(num_sms, 2, 128, 256, n_cols);
+  return static_cast<int>(align_up(m > 0 ? m : 128, 128));
+}
+
+// Test hook (moe_debug_withhold_ready): a minibatch whose readiness is never published.
+std::atomic<int> g_withhold{-1};
+
 WsLayout ws_layout(const moe_dims* D, int op) {
   WsLayout L;
   const int64_t A = D->T * D->k, E = D->E, R = padded_rows(D);
@@ -203,9 +221,25 @@ WsLayout ws_layout(const moe_dims* D, int op) {
   L.incl = c.take(4 * nt * E);
   L.rank = c.take(4 * A);
   L.mtile = c.take(4 * (E + 1));
+  L.ready = c.take(4 * (R / 128 + 1));
+  L.order = c.take(4 * E);
   if (op >= MOE_OP_FORWARD) {
     L.tq = c.take(D->T * D->d);
     L.ts = c.take(D->T * (D->d / 32));
+  }
+  if (op == MOE_OP_FORWARD_BF16) {
+    L.idx = c.take(4 * A);
+    L.w = c.take(4 * A);
+    L.counts = c.take(4 * E);
+    L.offsets = c.take(4 * (E + 1));
+    L.perm = c.take(4 * A);
+    L.inv = c.take(4 * A);
+    L.pad = c.take(4 * (E + 1));
+    L.xq = c.take(2 * R * D->d);   // bf16 rows of x in padded expert order
+    L.hq = c.take(2 * R * D->f);   // bf16 h
+    L.y = c.take(4 * R * D->d);
+    L.total = c.off;
+    return L;
   }
   if (op == MOE_OP_BACKWARD) {
     const int64_t d = D->d, f = D->f;
@@ -292,7 +326,8 @@ moe_status route_empty(const moe_dims* D, int32_t* counts, int32_t* offsets, int
 moe_status dispatch_pull(const moe_dims* D, const uint16_t* src, const int32_t* offsets,
                          const int32_t* prefix, int prefix_shift, const int32_t* perm,
                          uint8_t* tok_q, uint8_t* tok_s, uint8_t* out_q, uint8_t* out_s,
-                         int32_t* status, int sms, cudaStream_t st) {
+                         int32_t* status, int sms, cudaStream_t st, int32_t* ready = nullptr,
+                         int ready_rows_ = 0) {
   QuantRowsParams Q;
   Q.src = src;
   Q.src_ld = D->d;
@@ -306,6 +341,10 @@ moe_status dispatch_pull(const moe_dims* D, const uint16_t* src, const int32_t* 
   Q.kgroups = D->d / 128;
   MOE_TRY(cuda_ok(launch_quant_rows(Q, sms, st)));
   GatherParams G;
+  G.ready = ready;
+  G.ready_rows = ready_rows_;
+  G.withhold = g_withhold.load();
+  G.row_bytes = D->d;
   G.q_tok = tok_q;
   G.s_tok = tok_s;
   G.T = D->T;
@@ -384,16 +423,17 @@ int64_t moe_saved_bytes(const moe_dims* D, int32_t field) {
 }
 
 size_t moe_workspace_bytes(const moe_dims* dims, int32_t op) {
-  if (check_dims(dims) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_BACKWARD) return 0;
+  if (check_dims(dims) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_FORWARD_BF16) return 0;
   return static_cast<size_t>(ws_layout(dims, op).total);
 }
 
 int64_t moe_workspace_offset(const moe_dims* D, int32_t op, int32_t buffer) {
-  if (check_dims(D) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_BACKWARD) return -1;
+  if (check_dims(D) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_FORWARD_BF16) return -1;
   const WsLayout L = ws_layout(D, op);
   if (buffer == MOE_WS_MTILE) return L.mtile;
-  if (op == MOE_OP_FORWARD && buffer == MOE_WS_Y) return L.y;
-  if (op == MOE_OP_FORWARD && buffer == MOE_WS_COUNTS) return L.counts;
+  if ((op == MOE_OP_FORWARD || op == MOE_OP_FORWARD_BF16) && buffer == MOE_WS_Y) return L.y;
+  if ((op == MOE_OP_FORWARD || op == MOE_OP_FORWARD_BF16) && buffer == MOE_WS_COUNTS)
+    return L.counts;
   if (op != MOE_OP_BACKWARD) return -1;
   switch (buffer) {
     case MOE_WS_DOUT_Q: return L.dq;
@@ -573,10 +613,203 @@ moe_status moe_grouped_gemm_mx(int32_t G, int64_t rows_a, int32_t N, int32_t K,
   P.sfa = a_s;
   P.sfb = b_s;
   P.status = at<int32_t>(ws, 0);
+  P.tile_ctr = at<uint32_t>(ws, kCtrGeneric);
+  MOE_TRY(cuda_ok(cudaMemsetAsync(P.tile_ctr, 0, 4, static_cast<cudaStream_t>(stream))));
   CUtensorMap tc;
   MOE_TRY(make_out_tmap(&tc, d_out, rows_a, N, false));
   return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tc, tc, P, sms,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_grouped_gemm_bf16(int32_t G, int64_t rows_a, int32_t N, int32_t K,
+                                 const int32_t* mtile_prefix, const int32_t* rows_valid,
+                                 const uint16_t* a, const uint16_t* b, float* d_out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  if (G <= 0 || G > 1024 || rows_a < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (N % 256 || K % 64 || rows_a % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!mtile_prefix || !a || !b || !d_out || !ws) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < 256) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  const void* ptrs[] = {a, b, d_out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  if (rows_a == 0) return MOE_OK;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap ta, tb, tc;
+  MOE_TRY(make_tmap(&ta, a, rows_a, 2 * static_cast<int64_t>(K), 128));
+  MOE_TRY(make_tmap(&tb, b, static_cast<int64_t>(G) * N, 2 * static_cast<int64_t>(K), 256));
+  MOE_TRY(make_out_tmap(&tc, d_out, rows_a, N, false));
+  GemmParams P = {};
+  P.G = G;
+  P.N = N;
+  P.K = 2 * K;
+  P.mtile_prefix = mtile_prefix;
+  P.rows_valid = rows_valid;
+  P.status = at<int32_t>(ws, 0);
+  P.tile_ctr = at<uint32_t>(ws, kCtrGeneric);
+  MOE_TRY(cuda_ok(cudaMemsetAsync(P.tile_ctr, 0, 4, st)));
+  return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, tc, tc, P, sms, st));
+}
+
+moe_status moe_prepare_weights_bf16(const moe_dims* D, const uint16_t* wg, const uint16_t* wu,
+                                    const uint16_t* wd, uint16_t* wgu_t, uint16_t* wd_t,
+                                    void* stream) {
+  MOE_TRY(check_dims(D));
+  if (!wg || !wu || !wd || !wgu_t || !wd_t) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {wg, wu, wd, wgu_t, wd_t};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int half = 0; half < 2; ++half) {  // gate / up: column n of W[e] -> interleaved row
+    TransposeBf16Params P;
+    P.src = half == 0 ? wg : wu;
+    P.G = D->E;
+    P.K = D->d;
+    P.ncols = D->f;
+    P.dst = wgu_t;
+    P.map_mode = 1;
+    P.interleave_half = half;
+    MOE_TRY(cuda_ok(launch_transpose_bf16(P, st)));
+  }
+  TransposeBf16Params P;  // down: column n of W_down[e] -> row e*d + n
+  P.src = wd;
+  P.G = D->E;
+  P.K = D->f;
+  P.ncols = D->d;
+  P.dst = wd_t;
+  P.map_mode = 0;
+  P.interleave_half = 0;
+  return cuda_ok(launch_transpose_bf16(P, st));
+}
+
+moe_status moe_forward_bf16(const moe_dims* D, const uint16_t* wgu_t, const uint16_t* wd_t,
+                            const uint16_t* x, const float* logits, uint16_t* out, void* ws,
+                            size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(D));
+  if (!wgu_t || !wd_t || !ws || (D->T > 0 && (!x || !logits || !out)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  {
+    const void* ptrs[] = {wgu_t, wd_t, x, logits, out};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  const WsLayout L = ws_layout(D, MOE_OP_FORWARD_BF16);
+  if (ws_bytes < static_cast<size_t>(L.total)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* w = at<float>(ws, L.w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  int32_t* pad = at<int32_t>(ws, L.pad);
+  int32_t* mtile = at<int32_t>(ws, L.mtile);
+  uint16_t* xp = at<uint16_t>(ws, L.xq);
+  uint16_t* h16 = at<uint16_t>(ws, L.hq);
+  float* y = at<float>(ws, L.y);
+  int32_t* status = at<int32_t>(ws, 0);
+  if (D->T == 0) return route_empty(D, counts, offsets, mtile, pad, st);
+  {
+    StageScope sc(MOE_STAGE_ROUTE, st);
+    MOE_TRY(run_route(D, logits, idx, w, counts, offsets, perm, inv, pad, ws, L, sms, st));
+  }
+  const int64_t R = padded_rows(D);
+  const int mb = ready_rows(sms, 2 * static_cast<int64_t>(D->f));
+  int32_t* ready = at<int32_t>(ws, L.ready);
+  {  // pull dispatch of the bf16 rows, published minibatch by minibatch
+    StageScope sc(MOE_STAGE_PERMUTE, st);
+    SchedInitParams SI;
+    SI.counts = counts;
+    SI.pad_offsets = pad;
+    SI.E = D->E;
+    SI.ready = ready;
+    SI.ready_rows = mb;
+    SI.n_ready = static_cast<int>((R + mb - 1) / mb);
+    SI.order = nullptr;
+    MOE_TRY(cuda_ok(launch_sched_init(SI, st)));
+    GatherParams G;
+    G.ready = ready;
+    G.ready_rows = mb;
+    G.withhold = g_withhold.load();
+    G.row_bytes = 2 * static_cast<int64_t>(D->d);
+    G.q_tok = reinterpret_cast<const uint8_t*>(x);
+    G.s_tok = nullptr;
+    G.T = D->T;
+    G.d = D->d;
+    G.E = D->E;
+    G.k = D->k;
+    G.offsets = offsets;
+    G.mtile_prefix = mtile;
+    G.prefix_shift = 0;
+    G.perm = perm;
+    G.q_out = reinterpret_cast<uint8_t*>(xp);
+    G.s_out = nullptr;
+    G.status = status;
+    MOE_TRY(cuda_ok(launch_gather_rows(G, sms, st)));
+  }
+  {
+    StageScope sc(MOE_STAGE_GATEUP, st);
+    CUtensorMap ta, tb;
+    MOE_TRY(make_tmap(&ta, xp, R, 2 * static_cast<int64_t>(D->d), 128));
+    MOE_TRY(make_tmap(&tb, wgu_t, static_cast<int64_t>(D->E) * 2 * D->f,
+                      2 * static_cast<int64_t>(D->d), 256));
+    GemmParams P = {};
+    P.G = D->E;
+    P.N = 2 * D->f;
+    P.K = 2 * D->d;
+    P.f = D->f;
+    P.mtile_prefix = mtile;
+    P.rows_valid = counts;
+    P.h16 = h16;
+    P.status = status;
+    P.tile_ctr = at<uint32_t>(ws, kCtrFwdGateUp);
+    P.ready = ready;
+    P.ready_rows = mb;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_BF16, ta, tb, ta, tb, P, sms, st, true)));
+  }
+  {
+    StageScope sc(MOE_STAGE_DOWN, st);
+    CUtensorMap ta, tb, ty;
+    MOE_TRY(make_tmap(&ta, h16, R, 2 * static_cast<int64_t>(D->f), 128));
+    MOE_TRY(make_tmap(&tb, wd_t, static_cast<int64_t>(D->E) * D->d,
+                      2 * static_cast<int64_t>(D->f), 256));
+    MOE_TRY(make_out_tmap(&ty, y, R, D->d, false));
+    GemmParams P = {};
+    P.G = D->E;
+    P.N = D->d;
+    P.K = 2 * D->f;
+    P.mtile_prefix = mtile;
+    P.rows_valid = counts;
+    P.status = status;
+    P.tile_ctr = at<uint32_t>(ws, kCtrFwdDown);
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, ty, ty, P, sms, st)));
+  }
+  {
+    StageScope sc(MOE_STAGE_COMBINE, st);
+    CombineParams P;
+    P.y = y;
+    P.topk_w = w;
+    P.topk_idx = idx;
+    P.inv = inv;
+    P.offsets = offsets;
+    P.mtile_prefix = mtile;
+    P.prefix_shift = 0;
+    P.T = D->T;
+    P.d = D->d;
+    P.E = D->E;
+    P.k = D->k;
+    P.out = out;
+    P.status = status;
+    MOE_TRY(cuda_ok(launch_combine(P, sms, st)));
+  }
+  return MOE_OK;
 }
 
 moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* x,
@@ -631,10 +864,21 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
   }
 
   const int64_t R = padded_rows(D);
+  const int mb = ready_rows(sms, 2 * static_cast<int64_t>(D->f));
+  int32_t* ready = at<int32_t>(ws, L.ready);
   {
     StageScope sc(MOE_STAGE_PERMUTE, st);
+    SchedInitParams SI;
+    SI.counts = counts;
+    SI.pad_offsets = pad;
+    SI.E = D->E;
+    SI.ready = ready;
+    SI.ready_rows = mb;
+    SI.n_ready = static_cast<int>((R + mb - 1) / mb);
+    SI.order = nullptr;
+    MOE_TRY(cuda_ok(launch_sched_init(SI, st)));
     MOE_TRY(dispatch_pull(D, x, offsets, mtile, 0, perm, at<uint8_t>(ws, L.tq),
-                          at<uint8_t>(ws, L.ts), xq, xs, status, sms, st));
+                          at<uint8_t>(ws, L.ts), xq, xs, status, sms, st, ready, mb));
   }
   {
     StageScope sc(MOE_STAGE_GATEUP, st);
@@ -654,7 +898,10 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.hs = hs;
     P.gu = gu;
     P.status = status;
-    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_SWIGLU, ta, tb, ta, tb, P, sms, st)));
+    P.tile_ctr = at<uint32_t>(ws, kCtrFwdGateUp);
+    P.ready = ready;
+    P.ready_rows = mb;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_SWIGLU, ta, tb, ta, tb, P, sms, st, true)));
   }
   {
     StageScope sc(MOE_STAGE_DOWN, st);
@@ -670,6 +917,7 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.sfa = hs;
     P.sfb = W->wd_s;
     P.status = status;
+    P.tile_ctr = at<uint32_t>(ws, kCtrFwdDown);
     CUtensorMap ty;
     MOE_TRY(make_out_tmap(&ty, y, R, D->d, false));
     MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, ty, ty, P, sms, st)));
@@ -728,12 +976,26 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
   float* dxa = at<float>(ws, L.dxa);
   float* gbuf = at<float>(ws, L.gbuf);
 
+  // grouped-GEMM tile counters start at zero
+  MOE_TRY(cuda_ok(cudaMemsetAsync(at<uint8_t>(ws, 64), 0, 64, st)));
+  const int mb = ready_rows(sms, f);
+  int32_t* ready = at<int32_t>(ws, L.ready);
+  int32_t* order = at<int32_t>(ws, L.order);
   if (D->T > 0) {
     {  // pull reverse-combine: dOut rows gathered into expert order, MXFP8 along d
       StageScope sc(MOE_STAGE_BWD_DOUT, st);
+      SchedInitParams SI;
+      SI.counts = S->counts;
+      SI.pad_offsets = S->pad_offsets;
+      SI.E = E;
+      SI.ready = ready;
+      SI.ready_rows = mb;
+      SI.n_ready = static_cast<int>((R + mb - 1) / mb);
+      SI.order = order;  // the weight gradients' longest-first expert order
+      MOE_TRY(cuda_ok(launch_sched_init(SI, st)));
       MOE_TRY(dispatch_pull(D, dout, S->offsets, S->pad_offsets, 7, S->perm,
                             at<uint8_t>(ws, L.tq), at<uint8_t>(ws, L.ts), dq, dsc, status, sms,
-                            st));
+                            st, ready, mb));
     }
     {  // G = dout^ . Wd'^T (fp32, padded expert order)
       StageScope sc(MOE_STAGE_BWD_DGRAD_DOWN, st);
@@ -751,7 +1013,10 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.sfa = dsc;
       P.sfb = W->wdT_s;
       P.status = status;
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg, P, sms, st)));
+      P.tile_ctr = at<uint32_t>(ws, kCtrBwdDgradDown);
+      P.ready = ready;
+      P.ready_rows = mb;
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg, P, sms, st, true)));
     }
     {  // d(router weights), SwiGLU backward, [dg|du] -> MXFP8 along f
       StageScope sc(MOE_STAGE_BWD_SWIGLU, st);
@@ -787,6 +1052,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.sfa = dgu_s;
       P.sfb = W->wguT_s;
       P.status = status;
+      P.tile_ctr = at<uint32_t>(ws, kCtrBwdDgradGateUp);
       CUtensorMap tx;
       MOE_TRY(make_out_tmap(&tx, dxa, R, d, false));
       MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tx, tx, P, sms, st)));
@@ -871,6 +1137,8 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     P.out_b = dWu;
     P.split = f;
     P.status = status;
+    P.tile_ctr = at<uint32_t>(ws, kCtrBwdWgrad0);
+    P.order = D->T > 0 ? order : nullptr;
     CUtensorMap tg, tu;
     MOE_TRY(make_out_tmap(&tg, dWg, static_cast<int64_t>(E) * d, f, true));
     MOE_TRY(make_out_tmap(&tu, dWu, static_cast<int64_t>(E) * d, f, true));
@@ -884,10 +1152,40 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     P.out_a = dWd;
     P.out_b = nullptr;
     P.split = d;
+    P.tile_ctr = at<uint32_t>(ws, kCtrBwdWgrad1);
     CUtensorMap tdw;
     MOE_TRY(make_out_tmap(&tdw, dWd, static_cast<int64_t>(E) * f, d, true));
     MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, tdw, tdw, P, sms, st)));
   }
+  return MOE_OK;
+}
+
+moe_status moe_router_backward(const moe_dims* D, const float* logits, const int32_t* topk_idx,
+                               const float* dw_route, float* dlogits, int32_t* status,
+                               void* stream) {
+  MOE_TRY(check_dims(D));
+  if (D->T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !dw_route || !dlogits) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {logits, topk_idx, dw_route, dlogits, status};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  RouterBwdParams P;
+  P.logits = logits;
+  P.topk_idx = topk_idx;
+  P.dw_route = dw_route;
+  P.T = D->T;
+  P.E = D->E;
+  P.k = D->k;
+  P.score_fn = D->score_fn;
+  P.dlogits = dlogits;
+  P.status = status;
+  return cuda_ok(launch_router_bwd(P, sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_debug_withhold_ready(int32_t minibatch) {
+  g_withhold.store(minibatch < 0 ? -1 : minibatch);
   return MOE_OK;
 }
 

@@ -11,8 +11,10 @@
 // Tile 128 x 256 x 128 (rows x cols x K per stage), 4-stage TMA pipeline (3 stages in the
 // TMA-store modes, whose output staging buffers take 64 KB of shared memory).
 //
-// Warp roles (320 threads, one CTA per SM, persistent over a static round-robin tile list
-// that is derived on the device from the per-expert tile prefix -- no host round trip):
+// Warp roles (320 threads, one CTA per SM, persistent; tiles come from a device-side list
+// derived from the per-expert tile prefix -- no host round trip -- handed out one at a
+// time by an atomic counter and passed from the producer to the other roles through a
+// small ring in shared memory):
 //   warp 0      TMA producer: A tile 16 KB + B tile 32 KB via cp.async.bulk.tensor (128-byte
 //               swizzle), scale chunks (512 B for A, 2 x 512 B for B) via cp.async.bulk.
 //   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scales -> TMEM) and tcgen05.mma.
@@ -21,6 +23,12 @@
 //               column half (w-2)/4.
 // Tile order inside an expert is N-major (all M tiles of one weight tile back to back) so
 // that a weight tile is read from HBM once and re-read by the neighbouring CTAs from L2.
+// Experts go in index order, the order in which the dispatch writes their rows: with a
+// readiness table (article §02: device-local counters signal that a minibatch of rows is
+// ready; a minibatch holds two full waves of tiles) the producer loads a tile's rows as
+// soon as their minibatch is complete, so this GEMM runs while the dispatch still writes
+// later experts.  The weight gradients, whose tile cost grows with the expert's token
+// count, hand out the experts longest first.
 //
 // Modes (epilogues):
 //   STORE_F32_TMA  D in fp32 through shared memory and TMA stores (the down projection
@@ -45,11 +53,17 @@ constexpr uint32_t kSfCol = 256;  // + 16 * stage: A scales 4 columns, B scales 
 constexpr uint32_t kABytes = BM * BK, kBBytes = BN * BK;
 constexpr uint32_t kTxBytes = kABytes + kBBytes + 512 + 1024;
 constexpr int kMaxG = 1024;
+constexpr int kRing = 8;  // tiles in flight between the producer and the other roles
 
 // Modes that store their output with TMA need staging space: 3 pipeline stages instead of 4.
 template <int MODE>
 struct ModeCfg {
-  static constexpr bool kTmaStore = MODE == GEMM_STORE_F32_TMA || MODE == GEMM_WGRAD_BF16;
+  // operand kind: MXFP8 with block scales, or bf16 (the layer's BF16 variant, kind::f16)
+  static constexpr bool kBf16 = MODE == GEMM_GATEUP_BF16 || MODE == GEMM_STORE_F32_BF16;
+  static constexpr bool kGateUp = MODE == GEMM_GATEUP_SWIGLU || MODE == GEMM_GATEUP_BF16;
+  static constexpr bool kStoreF32 = MODE == GEMM_STORE_F32_TMA || MODE == GEMM_STORE_F32_BF16;
+  static constexpr uint32_t kTx = kBf16 ? kABytes + kBBytes : kTxBytes;
+  static constexpr bool kTmaStore = kStoreF32 || MODE == GEMM_WGRAD_BF16;
   static constexpr int kStages = kTmaStore ? 3 : 4;
   static constexpr int kStageBufs = kTmaStore ? 2 : 0;  // per epilogue warp, 4 KB each
   // A tile with fewer than 128 valid rows (an expert's last tile) runs with the operands
@@ -58,14 +72,15 @@ struct ModeCfg {
   // (Measured: a gain for the fp32-output GEMMs; with the SwiGLU epilogue, whose
   // transposed form quantises across lanes, the gate/up GEMM became slower, so it keeps
   // full tiles.)
-  static constexpr bool kSwapTail = MODE == GEMM_STORE_F32_TMA;
+  static constexpr bool kSwapTail = kStoreF32;
 };
 
 template <int ST, int NSTG>
 struct GemmSmemT {
   uint8_t a[ST][kABytes];
   uint8_t b[ST][kBBytes];
-  uint8_t stg[NSTG ? kEpiWarps * NSTG : 1][4096];  // 32 rows x 128 bytes, 128-byte swizzle
+  // epilogue staging: 32 rows x 128 bytes, 128-byte swizzle (unused without TMA stores)
+  uint8_t stg[NSTG ? kEpiWarps * NSTG : 1][NSTG ? 4096 : 16];
   uint8_t sfa[ST][512];
   uint8_t sfb[ST][1024];
   uint64_t full[ST];
@@ -73,6 +88,10 @@ struct GemmSmemT {
   uint64_t tmem_full;
   uint64_t tmem_empty;
   uint64_t tmem_empty_hi;  // WGRAD: columns 128..255 drained (tmem_empty: 0..127)
+  uint64_t ring_full[kRing];
+  uint64_t ring_empty[kRing];
+  uint64_t mma_drain;      // the MMA issuer's last commit, awaited before the CTA exits
+  int ring[kRing];         // tile ids (-1: no more tiles)
   uint32_t tmem_base;
   int abort_flag;
   int prefix[kMaxG + 1];
@@ -84,6 +103,7 @@ template <int MODE>
 constexpr size_t smem_bytes() { return sizeof(SmemOf<MODE>) + 1024; }
 static_assert(smem_bytes<GEMM_STORE_F32_TMA>() <= 232448, "shared memory budget (227 KB)");
 static_assert(smem_bytes<GEMM_GATEUP_SWIGLU>() <= 232448, "shared memory budget (227 KB)");
+static_assert(smem_bytes<GEMM_WGRAD_BF16>() <= 232448, "shared memory budget (227 KB)");
 
 struct TileInfo {
   int g, i, j;
@@ -116,12 +136,16 @@ __device__ __forceinline__ TileInfo decode_tile_var_m(int tile, const int* prefi
   return t;
 }
 
-// Variable-K groups (wgrad): group g reduces over K blocks [prefix[g], prefix[g+1]).
-__device__ __forceinline__ TileInfo decode_tile_var_k(int tile, const int* prefix, int MT, int NT) {
+// Variable-K groups (wgrad): group g reduces over K blocks [prefix[g], prefix[g+1]); every
+// group has the same MT x NT tiles, handed out group by group in `order` (if given).
+__device__ __forceinline__ TileInfo decode_tile_var_k(int tile, const int* prefix, int MT, int NT,
+                                                      const int32_t* order) {
   TileInfo t;
   const int per = MT * NT;
   t.g = tile / per;
-  const int local = tile - t.g * per;
+  const int slot = t.g;
+  if (order) t.g = __ldg(order + slot);
+  const int local = tile - slot * per;
   t.i = local / NT;
   t.j = local - t.i * NT;
   t.kb0 = prefix[t.g];
@@ -135,7 +159,8 @@ __device__ __forceinline__ TileInfo decode_tile_var_k(int tile, const int* prefi
 template <int MODE>
 __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const int* valid,
                                                 const GemmParams& P) {
-  if (MODE == GEMM_WGRAD_BF16) return decode_tile_var_k(tile, prefix, P.M / BM, P.N / BN);
+  if (MODE == GEMM_WGRAD_BF16)
+    return decode_tile_var_k(tile, prefix, P.M / BM, P.N / BN, P.order);
   return decode_tile_var_m(tile, prefix, valid, P.G, P.N / BN, P.N, P.K / BK);
 }
 
@@ -172,6 +197,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(smem_u32(&S.tmem_full), 1);
     mbar_init(smem_u32(&S.tmem_empty), kEpiWarps);
     mbar_init(smem_u32(&S.tmem_empty_hi), kEpiWarps);
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(smem_u32(&S.ring_full[r]), 1);
+      mbar_init(smem_u32(&S.ring_empty[r]), 1 + kEpiWarps);
+    }
+    mbar_init(smem_u32(&S.mma_drain), 1);
     S.abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmA);
@@ -191,38 +221,80 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      int stage = 0, rs = 0, ready_b = -1;
+      uint32_t phase = 0, rph = 0;
+      uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and that phase's parity
+      for (;;) {
+        const int tile = static_cast<int>(atomicAdd(P.tile_ctr, 1u));
+        if (!mbar_wait(smem_u32(&S.ring_empty[rs]), rph ^ 1u, abort_flag, P.status)) break;
+        S.ring[rs] = tile < total ? tile : -1;
+        mbar_arrive(smem_u32(&S.ring_full[rs]));
+        if (++rs == kRing) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        if (tile >= total) break;
         const TileInfo ti = decode_tile<MODE>(tile, S.prefix, S.valid, P);
+        if (MODE != GEMM_WGRAD_BF16 && P.ready) {
+          // the tile's rows are loaded once the dispatch has published their minibatch
+          const int b = static_cast<int>(ti.a_row0 / P.ready_rows);
+          if (b > ready_b) {
+            if (!wait_counter_zero(P.ready + b, abort_flag, P.status)) break;
+            fence_proxy_async_global();
+            ready_b = b;
+          }
+        }
         const int64_t rbA = ti.a_row0 >> 7, rbB = ti.b_row0 >> 7;
+        bool ok = true;
         for (int kb = ti.kb0; kb < ti.kb0 + ti.nk; ++kb) {
-          if (!mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, abort_flag, P.status)) break;
+          if (!mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
           const uint32_t fb = smem_u32(&S.full[stage]);
-          mbar_arrive_expect_tx(fb, kTxBytes);
+          mbar_arrive_expect_tx(fb, ModeCfg<MODE>::kTx);
           tma_load_2d(smem_u32(S.a[stage]), &tmA, fb, kb * BK, static_cast<int32_t>(ti.a_row0));
           tma_load_2d(smem_u32(S.b[stage]), &tmB, fb, kb * BK, static_cast<int32_t>(ti.b_row0));
-          bulk_load(smem_u32(S.sfa[stage]), P.sfa + ((rbA * kgroups + kb) << 9), 512, fb);
-          bulk_load(smem_u32(S.sfb[stage]), P.sfb + ((rbB * kgroups + kb) << 9), 512, fb);
-          bulk_load(smem_u32(S.sfb[stage]) + 512, P.sfb + (((rbB + 1) * kgroups + kb) << 9), 512,
-                    fb);
+          if (!ModeCfg<MODE>::kBf16) {
+            bulk_load(smem_u32(S.sfa[stage]), P.sfa + ((rbA * kgroups + kb) << 9), 512, fb);
+            bulk_load(smem_u32(S.sfb[stage]), P.sfb + ((rbB * kgroups + kb) << 9), 512, fb);
+            bulk_load(smem_u32(S.sfb[stage]) + 512, P.sfb + (((rbB + 1) * kgroups + kb) << 9),
+                      512, fb);
+          }
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
+        if (!ok) break;
       }
+      // Leave only once every load this thread issued has landed in shared memory (on the
+      // normal path the MMAs consumed them all; after an abort some may still be in flight).
+      for (int st = 0; st < STAGES; ++st)
+        if ((armed >> st) & 1u) mbar_drain(smem_u32(&S.full[st]), (armed_par >> st) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, rs = 0;
+      uint32_t phase = 0, acc_phase = 0, rph = 0;
+      bool issued = false;
       const uint32_t idesc = idesc_mxf8_e4m3(BM, BN);
-      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      for (;;) {
+        if (!mbar_wait(smem_u32(&S.ring_full[rs]), rph, abort_flag, P.status)) break;
+        const int tile = S.ring[rs];
+        mbar_arrive(smem_u32(&S.ring_empty[rs]));
+        if (++rs == kRing) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        if (tile < 0) break;
         const TileInfo tinfo = decode_tile<MODE>(tile, S.prefix, S.valid, P);
         const int nk = tinfo.nk;
         if (nk == 0) continue;  // empty expert (wgrad): the epilogue writes zeros
+        issued = true;
         const bool swapped = ModeCfg<MODE>::kSwapTail && tinfo.rows < BM;
         const uint32_t idesc_sw = idesc_mxf8_e4m3(BM, (tinfo.rows + 15) & ~15);
         if (!mbar_wait(smem_u32(&S.tmem_empty), acc_phase ^ 1u, abort_flag, P.status)) break;
@@ -278,11 +350,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               break;
             }
             tc_fence_after();
+            const uint32_t a0 = smem_u32(S.a[stage]), b0 = smem_u32(S.b[stage]);
+            if (ModeCfg<MODE>::kBf16) {
+              // bf16 operands: 4 MMAs of K = 16 elements (32 bytes) per 128-byte stage
+              const uint32_t id = swapped ? idesc_f16_bf16(BM, (tinfo.rows + 15) & ~15)
+                                          : idesc_f16_bf16(BM, BN);
+#pragma unroll
+              for (int kk = 0; kk < BK / 32; ++kk) {
+                const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+                if (swapped) {
+                  const uint64_t bt = sdesc_k_sw128(a0 + 32u * kk);
+                  mma_bf16(tbase + kAccCol, sdesc_k_sw128(b0 + 32u * kk), bt, id, acc);
+                  mma_bf16(tbase + kAccCol + 128, sdesc_k_sw128(b0 + 128u * 128u + 32u * kk), bt,
+                           id, acc);
+                } else {
+                  mma_bf16(tbase + kAccCol, sdesc_k_sw128(a0 + 32u * kk),
+                           sdesc_k_sw128(b0 + 32u * kk), id, acc);
+                }
+              }
+              mma_commit(smem_u32(&S.empty[stage]));
+              if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+              }
+              continue;
+            }
             const uint32_t sf = tbase + kSfCol + 16u * stage;
             tmem_cp_scales(sf, sdesc_scale_chunk(smem_u32(S.sfa[stage])));
             tmem_cp_scales(sf + 4, sdesc_scale_chunk(smem_u32(S.sfb[stage])));
             tmem_cp_scales(sf + 8, sdesc_scale_chunk(smem_u32(S.sfb[stage]) + 512));
-            const uint32_t a0 = smem_u32(S.a[stage]), b0 = smem_u32(S.b[stage]);
             if (swapped) {
               // D0[w, t] = sum_k B[w, k] A[t, k] for weight rows w < 128, D1 for rows 128..255
 #pragma unroll
@@ -315,14 +411,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mma_commit(smem_u32(&S.tmem_full));
         acc_phase ^= 1u;
       }
+      // every MMA and scale copy issued here has completed before the CTA moves on
+      if (issued) {
+        mma_commit(smem_u32(&S.mma_drain));
+        mbar_drain(smem_u32(&S.mma_drain), 0);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int h = (warp - 2) >> 2;   // column half
-    uint32_t acc_phase = 0;
-    int stg_buf = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    uint32_t acc_phase = 0, rph = 0;
+    int stg_buf = 0, rs = 0;
+    for (;;) {
+      if (!mbar_wait(smem_u32(&S.ring_full[rs]), rph, abort_flag, P.status)) break;
+      const int tile = S.ring[rs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.ring_empty[rs]));
+      if (++rs == kRing) {
+        rs = 0;
+        rph ^= 1u;
+      }
+      if (tile < 0) break;
       const TileInfo ti = decode_tile<MODE>(tile, S.prefix, S.valid, P);
       if (MODE == GEMM_WGRAD_BF16 && ti.nk == 0) {
         const int64_t m = ti.a_row0 + 32 * q + lane;
@@ -387,7 +497,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&S.tmem_empty));
         acc_phase ^= 1u;
-        if (MODE == GEMM_STORE_F32_TMA) {
+        if (ModeCfg<MODE>::kStoreF32) {
           const int32_t y0 = static_cast<int32_t>(ti.a_row0);
           const int32_t x0 = ti.j * BN + 32 * q;
 #pragma unroll
@@ -414,7 +524,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         continue;
       }
       float v0[32], v1[32], v2[32], v3[32];
-      if (MODE == GEMM_GATEUP_SWIGLU) {
+      if (ModeCfg<MODE>::kGateUp) {
         tmem_ld32(taddr + 64 * h, v0);         // gate features 64h .. 64h+31
         tmem_ld32(taddr + 64 * h + 32, v1);    // gate features 64h+32 .. 64h+63
         tmem_ld32(taddr + 128 + 64 * h, v2);   // up, same features
@@ -432,7 +542,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       acc_phase ^= 1u;
 
       const int m = 32 * q + lane;
-      if (MODE == GEMM_STORE_F32_TMA) {
+      if (ModeCfg<MODE>::kStoreF32) {
         // fp32 rows of 128 columns: four 32-column chunks; whole 32-row boxes are written
         const int32_t x0 = ti.j * BN + 128 * h;
         const int32_t y = static_cast<int32_t>(ti.a_row0 + 32 * q);
@@ -451,7 +561,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (ti.i * BM + m >= S.valid[ti.g]) continue;
       const int64_t row = ti.a_row0 + m;
-      if (MODE == GEMM_GATEUP_SWIGLU) {
+      if (ModeCfg<MODE>::kGateUp) {
         const int f = P.f;
         const int fb = BN / 2 * ti.j + 64 * h;  // first feature of this thread's 64
         if (P.gu) {
@@ -470,6 +580,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int c = 0; c < 32; ++c) {
           v0[c] = v0[c] * sigmoid_fast(v0[c]) * v2[c];
           v1[c] = v1[c] * sigmoid_fast(v1[c]) * v3[c];
+        }
+        if (ModeCfg<MODE>::kBf16) {  // the BF16 variant: h rounded to bf16 (RNE)
+          uint4* hdst = reinterpret_cast<uint4*>(P.h16 + row * f + fb);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            hdst[c] = pack_bf16x8(v0 + 8 * c);
+            hdst[4 + c] = pack_bf16x8(v1 + 8 * c);
+          }
+          continue;
         }
         uint32_t q0[8], q1[8];
         const uint32_t s0 = mx_quant_block32(v0, q0);
@@ -498,35 +617,85 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 template <int MODE>
 static cudaError_t launch_mode(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                const CUtensorMap& tmC0, const CUtensorMap& tmC1,
-                               const GemmParams& P, int num_sms, cudaStream_t stream) {
+                               const GemmParams& P, int num_sms, cudaStream_t stream, bool pdl) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev >= 64 || !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_bytes<MODE>()));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    if (dev < 64) attr_set[dev] = true;
   }
-  grouped_gemm_kernel<MODE><<<num_sms, kGemmThreads, smem_bytes<MODE>(), stream>>>(tmA, tmB, tmC0,
-                                                                                  tmC1, P);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem_bytes<MODE>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE>, tmA, tmB, tmC0, tmC1, P);
 }
 
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmC0, const CUtensorMap& tmC1,
-                                const GemmParams& P, int num_sms, cudaStream_t stream) {
+                                const GemmParams& P, int num_sms, cudaStream_t stream, bool pdl) {
+  if (!P.tile_ctr) return cudaErrorInvalidValue;
   switch (mode) {
     case GEMM_GATEUP_SWIGLU:
-      return launch_mode<GEMM_GATEUP_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
+      return launch_mode<GEMM_GATEUP_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
     case GEMM_WGRAD_BF16:
-      return launch_mode<GEMM_WGRAD_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
+      return launch_mode<GEMM_WGRAD_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
     case GEMM_STORE_F32_TMA:
-      return launch_mode<GEMM_STORE_F32_TMA>(tmA, tmB, tmC0, tmC1, P, num_sms, stream);
+      return launch_mode<GEMM_STORE_F32_TMA>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
+    case GEMM_GATEUP_BF16:
+      return launch_mode<GEMM_GATEUP_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
+    case GEMM_STORE_F32_BF16:
+      return launch_mode<GEMM_STORE_F32_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+// ---------------------------------------------------------------------------------------
+// scheduling tables (one CTA): minibatch readiness counters and the longest-first order
+// ---------------------------------------------------------------------------------------
+constexpr int kSchedThreads = 256;
+
+__global__ void __launch_bounds__(kSchedThreads) sched_init_kernel(SchedInitParams P) {
+  __shared__ int s_cnt[kMaxG];
+  __shared__ int s_pad[kMaxG + 1];
+  const int tid = threadIdx.x, E = P.E;
+  for (int e = tid; e < E; e += kSchedThreads) s_cnt[e] = P.counts[e];
+  for (int e = tid; e <= E; e += kSchedThreads) s_pad[e] = P.pad_offsets[e];
+  for (int b = tid; b < P.n_ready; b += kSchedThreads) P.ready[b] = 0;
+  __syncthreads();
+  // valid rows of every expert segment, added to each minibatch the segment overlaps
+  for (int e = tid; e < E; e += kSchedThreads) {
+    const int lo = s_pad[e], hi = s_pad[e] + s_cnt[e];
+    for (int b = lo / P.ready_rows; b < P.n_ready && b * P.ready_rows < hi; ++b) {
+      const int a0 = max(lo, b * P.ready_rows), a1 = min(hi, (b + 1) * P.ready_rows);
+      if (a1 > a0) atomicAdd(P.ready + b, a1 - a0);
+    }
+  }
+  if (!P.order) return;
+  // order[rank(e)] = e with rank = experts before e in (count descending, index ascending)
+  for (int e = tid; e < E; e += kSchedThreads) {
+    const int c = s_cnt[e];
+    int rank = 0;
+    for (int f = 0; f < E; ++f) rank += (s_cnt[f] > c) || (s_cnt[f] == c && f < e);
+    P.order[rank] = e;
+  }
+}
+
+cudaError_t launch_sched_init(const SchedInitParams& P, cudaStream_t stream) {
+  if (P.E <= 0 || P.E > kMaxG || P.ready_rows <= 0) return cudaErrorInvalidValue;
+  sched_init_kernel<<<1, kSchedThreads, 0, stream>>>(P);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -67,8 +67,16 @@ struct QuantColsParams {
 cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream);
 
 // Pull gather of per-token MX rows: q_out[pad_offsets[e] + r] = q_tok[perm[offsets[e]+r]/k],
-// scales from the canonical per-token layout [T, d/32] into the UMMA layout of [R, d].
+// scales from the canonical per-token layout [T, d/32] into the UMMA layout of [R, d]
+// (s_tok nullable: rows only).
 struct GatherParams {
+  // ready (nullable): after writing a row, its minibatch counter ready[row / ready_rows] is
+  // decremented (release); withhold >= 0 skips that minibatch's decrements (a test hook
+  // that makes a consumer's bounded wait run out).
+  int32_t* ready;
+  int ready_rows;
+  int withhold;
+  int64_t row_bytes;     // bytes per row: d (MX codes) or 2d (bf16 rows, s_tok == nullptr)
   const uint8_t* q_tok;
   const uint8_t* s_tok;
   int64_t T;
@@ -148,6 +156,29 @@ struct SwigluBwdParams {
 };
 cudaError_t launch_swiglu_bwd(const SwigluBwdParams& P, int num_sms, cudaStream_t stream);
 
+// Weight transpose for the BF16 variant: W [G][K][ncols] bf16 -> row rowmap(g, n) of a
+// [*, K] bf16 matrix (map_mode as QuantColsParams: 0 plain, 1 gate/up interleave).
+struct TransposeBf16Params {
+  const uint16_t* src;
+  int G, K, ncols;
+  uint16_t* dst;
+  int map_mode;
+  int interleave_half;
+};
+cudaError_t launch_transpose_bf16(const TransposeBf16Params& P, cudaStream_t stream);
+
+// Router backward: dlogits [T, E] (zero except the k selected experts of each token).
+struct RouterBwdParams {
+  const float* logits;     // [T, E]
+  const int32_t* topk_idx; // [T, k]
+  const float* dw_route;   // [T, k]
+  int64_t T;
+  int E, k, score_fn;
+  float* dlogits;          // [T, E]
+  int32_t* status;         // nullable
+};
+cudaError_t launch_router_bwd(const RouterBwdParams& P, int num_sms, cudaStream_t stream);
+
 // Grouped block-scaled GEMM.
 enum GemmMode : int {
   GEMM_GATEUP_SWIGLU = 1,  // SwiGLU + MX requant of h, optional bf16 g/u save
@@ -155,12 +186,17 @@ enum GemmMode : int {
   GEMM_STORE_F32_TMA = 4,  // D fp32 [rows, N] through shared memory + TMA stores (down
                            // projection, both dgrads, the generic entry point); writes whole
                            // 128-row tiles (rows past a group's count get unused values)
+  // BF16 variant of the layer (kind::f16, bf16 operands, no scale factors; K counted in
+  // bytes, 2 per element):
+  GEMM_GATEUP_BF16 = 5,    // SwiGLU, h rounded to bf16 [rows, f]
+  GEMM_STORE_F32_BF16 = 6, // as STORE_F32_TMA
 };
 
 struct GemmParams {
   int G;
   int N;                 // output columns per group (multiple of 256)
-  int K;                 // reduction length (multiple of 128); WGRAD: total K of A and B
+  int K;                 // reduction length (multiple of 128); WGRAD: total K of A and B;
+                         // the BF16 modes: in bytes (2 x elements)
   int M;                 // WGRAD: output rows per group (multiple of 128)
   int f;                 // GATEUP / DGRAD: expert intermediate size
   const int32_t* mtile_prefix;  // [G+1] (shifted right by prefix_shift when loaded)
@@ -171,16 +207,45 @@ struct GemmParams {
   uint8_t* hq;           // GATEUP: [rows, f]
   uint8_t* hs;           // GATEUP: UMMA scales of [rows, f]
   uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16 save of g | u
+  uint16_t* h16;         // GATEUP_BF16: [rows, f] bf16 h
   // WGRAD: D[g] rows m < M, cols n < N -> (n < split ? out_a : out_b)[g][m][n mod split]
   uint16_t* out_a;
   uint16_t* out_b;
   int split;
   int32_t* status;
+  // Tile scheduling.  Tiles are handed out in order by an atomic counter (zero before the
+  // launch), so a CTA that starts late (its SM still busy with a concurrent kernel) takes
+  // fewer tiles.  ready (nullable): count-down counters of valid rows still to be written
+  // per minibatch of ready_rows padded rows (variable-M modes); a tile's A rows are loaded
+  // once its minibatch's counter is zero.  order (nullable, WGRAD): the order in which the
+  // groups' tiles are handed out (longest first).
+  uint32_t* tile_ctr;
+  const int32_t* ready;
+  int ready_rows;
+  const int32_t* order;
 };
 // tmC0 / tmC1: output tensor maps of the TMA-store modes (STORE_F32_TMA: fp32 [rows, N],
 // box 32 x 32; WGRAD: bf16 out_a / out_b, box 64 cols x 32 rows); ignored otherwise.
+// pdl: launched as a programmatic dependent of the previous kernel in the stream, which
+// must publish the rows this GEMM reads through P.ready.
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmC0, const CUtensorMap& tmC1,
-                                const GemmParams& P, int num_sms, cudaStream_t stream);
+                                const GemmParams& P, int num_sms, cudaStream_t stream,
+                                bool pdl = false);
+
+// Scheduling tables, one CTA: ready[b] = valid rows of expert segments inside padded rows
+// [b*ready_rows, (b+1)*ready_rows) for b < n_ready (count-down counters for a producer
+// kernel to decrement); order (nullable) = experts sorted by descending count (ties: lower
+// index first).
+struct SchedInitParams {
+  const int32_t* counts;
+  const int32_t* pad_offsets;   // [E+1] (multiples of 128)
+  int E;
+  int32_t* ready;
+  int n_ready;
+  int ready_rows;
+  int32_t* order;
+};
+cudaError_t launch_sched_init(const SchedInitParams& P, cudaStream_t stream);
 
 }  // namespace moe

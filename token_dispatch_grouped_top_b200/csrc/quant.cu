@@ -230,9 +230,13 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
 // scales of its token by index from the per-token quantised copy (x quantised once per
 // token, small enough to stay in L2) and writes them to its padded position: codes with
 // 16-byte copies, scales re-laid into the UMMA layout one 4-byte K-group word at a time.
+// The layer's BF16 variant pulls the bf16 rows of x the same way (no scales).
 __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_mt[kMaxE + 1];
+  // the consumer GEMM (launched as a programmatic dependent) may start now: it waits for
+  // each minibatch of rows through the readiness counters, not for this grid to finish
+  launch_dependents();
   for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
     s_off[i] = P.offsets[i];
     s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
@@ -258,14 +262,25 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
       if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
       continue;
     }
-    const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * d);
-    uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * d);
-    const int n16 = d >> 4;
+    const int64_t rb = P.row_bytes;
+    const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * rb);
+    uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * rb);
+    const int n16 = static_cast<int>(rb >> 4);
 #pragma unroll 4
     for (int i = lane; i < n16; i += 32) dst[i] = src[i];
-    const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
-    for (int g = lane; g < kg; g += 32)
-      *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
+    if (P.s_tok) {
+      const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
+      for (int g = lane; g < kg; g += 32)
+        *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
+    }
+    if (P.ready) {
+      // publish the row: every lane's stores are made visible device-wide before the
+      // minibatch counter drops (the consumer reads them after an acquire of the counter)
+      __threadfence();
+      __syncwarp();
+      const int b = static_cast<int>(p / P.ready_rows);
+      if (lane == 0 && b != P.withhold) red_release_add(P.ready + b, -1);
+    }
   }
 }
 
@@ -273,8 +288,61 @@ cudaError_t launch_gather_rows(const GatherParams& P, int num_sms, cudaStream_t 
   const int64_t A = P.T * P.k;
   if (A <= 0) return cudaSuccess;
   const int64_t blocks = (A + 7) / 8;
-  const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
+  // Feeding a concurrent GEMM: one CTA per SM, so that each SM keeps room for one GEMM CTA
+  // (its ~213 KB of shared memory and 320 threads) beside it.
+  const int64_t cap = P.ready ? num_sms : 16LL * num_sms;
+  const int grid = static_cast<int>(blocks < cap ? blocks : cap);
+  static bool carveout_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64 || !carveout_set[dev]) {
+    // configure the SMs this kernel lands on with the largest shared-memory carveout, so
+    // that a GEMM CTA can join it there without waiting for the SM to drain
+    const cudaError_t e = cudaFuncSetAttribute(gather_rows_kernel,
+                                               cudaFuncAttributePreferredSharedMemoryCarveout,
+                                               static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) carveout_set[dev] = true;
+  }
   gather_rows_kernel<<<grid, 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// Weights of the BF16 variant: a 32 x 32 tile of W[g] ([K, ncols], x @ W convention) goes
+// through shared memory so that both the reads (along ncols) and the writes (along K of
+// the output rows) are coalesced.  Setup only, not part of the layer's step.
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(TransposeBf16Params P) {
+  __shared__ uint16_t tile[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  const int64_t tiles_n = P.ncols / 32, tiles_k = P.K / 32;
+  const int64_t total = static_cast<int64_t>(P.G) * tiles_k * tiles_n;
+  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+    const int64_t tn = t % tiles_n, rest = t / tiles_n;
+    const int64_t tk = rest % tiles_k, g = rest / tiles_k;
+    const uint16_t* src = P.src + (g * P.K + tk * 32) * P.ncols + tn * 32;
+    for (int r = ty; r < 32; r += 8) tile[r][tx] = src[static_cast<int64_t>(r) * P.ncols + tx];
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {  // output row = column n of W, its K entries
+      const int64_t n = tn * 32 + r;
+      const int64_t row = P.map_mode == 0
+                              ? g * P.ncols + n
+                              : g * 2 * P.ncols + (n >> 7) * 256 + P.interleave_half * 128 +
+                                    (n & 127);
+      P.dst[row * P.K + tk * 32 + tx] = tile[tx][r];
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_transpose_bf16(const TransposeBf16Params& P, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(P.G) * (P.K / 32) * (P.ncols / 32);
+  if (total <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(total < 65536 ? total : 65536);
+  transpose_bf16_kernel<<<grid, 256, 0, stream>>>(P);
   return cudaGetLastError();
 }
 
