@@ -119,16 +119,18 @@ size_t moe_workspace_bytes(const moe_dims* dims, int32_t op);
 /* Inspection of intermediate results (tests, debugging): the byte offset inside an
  * operation's workspace of one internal buffer, -1 if that operation has no such buffer.
  * The contents are those of the last call that used the workspace, once it has completed
- * on its stream; the layouts are the ones stated per buffer.  R = moe_padded_rows(). */
+ * on its stream; the layouts are the ones stated per buffer.  R = moe_padded_rows().
+ * "Scaled fp16" [rows, C]: fp16 values q and, separately, one byte b per 32 consecutive
+ * values of a row ([rows, C/32]); the value is q * 2^(b - 127). */
 typedef enum {
   MOE_WS_MTILE = 0,   /* every op: [E+1] int32, 128-row tiles per expert, prefix-summed     */
-  MOE_WS_Y = 1,       /* forward: [R,d] fp32 expert outputs y (rows of padded expert order) */
+  MOE_WS_Y = 1,       /* forward: [R,d] expert outputs y, scaled fp16 values (padded order) */
   MOE_WS_DOUT_Q = 2,  /* backward: [R,d] MX codes of dOut gathered to expert order          */
   MOE_WS_DOUT_S = 3,  /*   their UMMA scales                                                */
-  MOE_WS_G = 4,       /* backward: [R,f] fp32 G = dOut^ . W_down'^T                          */
+  MOE_WS_G = 4,       /* backward: [R,f] G = dOut^ . W_down'^T, scaled fp16 values           */
   MOE_WS_DGU_Q = 5,   /* backward: [R,2f] MX codes of [dg | du] (along 2f)                   */
   MOE_WS_DGU_S = 6,
-  MOE_WS_DXA = 7,     /* backward: [R,d] fp32 per-assignment input gradients                 */
+  MOE_WS_DXA = 7,     /* backward: [R,d] per-assignment input gradients, scaled fp16 values  */
   MOE_WS_XT_Q = 8,    /* backward: [d,R] token-direction MX of x^ (UMMA scales of [d,R])     */
   MOE_WS_XT_S = 9,
   MOE_WS_HT_Q = 10,   /* backward: [f,R] token-direction MX of h^                            */
@@ -137,7 +139,10 @@ typedef enum {
   MOE_WS_GT_S = 13,
   MOE_WS_YT_Q = 14,   /* backward: [d,R] token-direction MX of w * dOut^                      */
   MOE_WS_YT_S = 15,
-  MOE_WS_COUNTS = 16  /* forward without a saved struct: [E] int32 tokens per expert        */
+  MOE_WS_COUNTS = 16, /* forward without a saved struct: [E] int32 tokens per expert        */
+  MOE_WS_Y_S = 17,    /* forward: [R,d/32] scale bytes of MOE_WS_Y                           */
+  MOE_WS_G_S = 18,    /* backward: [R,f/32] scale bytes of MOE_WS_G                          */
+  MOE_WS_DXA_S = 19   /* backward: [R,d/32] scale bytes of MOE_WS_DXA                        */
 } moe_ws_buffer;
 int64_t moe_workspace_offset(const moe_dims* dims, int32_t op, int32_t buffer);
 

@@ -47,15 +47,30 @@ def bf16_floor_error(ref: np.ndarray) -> float:
     return rel_fro(bf16_round(ref), ref)
 
 
-def assert_close_out(got: np.ndarray, ref: np.ndarray, rel=2e-3, maxabs_rms=3e-2):
-    """The layer tolerance: relative Frobenius error and max-abs error relative to RMS."""
+# Largest relative error of rounding a value to bf16 (8 significant bits): half a unit in
+# the last place, at most 2^-8 of the value.
+BF16_HALF_ULP_REL = 2.0 ** -8
+
+
+def assert_close_out(got: np.ndarray, ref: np.ndarray, rel=2e-3, maxabs_rms=3e-2,
+                     out_bf16: bool = True):
+    """The layer tolerance: relative Frobenius error <= rel, and element-wise
+    |got - ref| <= maxabs_rms * RMS(ref), on top of (for results stored in bf16) the
+    rounding of that element to bf16 itself, 2^-8 * |ref|: a bf16 result cannot be closer
+    to the fp64 value than its own rounding, which for a heavy-tailed matrix (a weight
+    gradient summed over a few tokens) exceeds 3e-2 * RMS at its largest elements."""
     err = rel_fro(got, ref)
     print(f"  rel_fro {err:.3e} (bf16 rounding of the exact result alone: "
           f"{bf16_floor_error(ref):.3e})")
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    mx = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    dev = np.abs(got - ref)
+    bound = maxabs_rms * rms + (BF16_HALF_ULP_REL * np.abs(ref) if out_bf16 else 0.0)
+    worst = float(np.max(dev / np.maximum(bound, 1e-300))) if got.size else 0.0
+    mx = float(np.max(dev)) if got.size else 0.0
+    print(f"  max abs error {mx:.3e} = {mx / max(rms, 1e-300):.3e} * RMS; worst element "
+          f"uses {worst:.3f} of its bound")
     assert err <= rel, f"relative Frobenius error {err:.3e} > {rel:.1e}"
-    assert mx <= maxabs_rms * rms, f"max abs error {mx:.3e} > {maxabs_rms}*RMS ({rms:.3e})"
+    assert worst <= 1.0, f"max abs error beyond {maxabs_rms}*RMS (+ bf16 rounding): {worst:.3f}"
     return err, mx / max(rms, 1e-300)
 
 
@@ -82,6 +97,13 @@ def mx_values(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """Dequantised float64 values of MX codes [n, K] with canonical scales [n, K/32]."""
     from oracle import mxfp8 as omx
     return omx.e4m3_decode(codes) * np.repeat(omx.e8m0_decode(scales), 32, axis=1)
+
+
+def f16s_values(q_rows, scale_rows) -> np.ndarray:
+    """Scaled fp16 (moe.h): fp16 values [n, C] times 2^(b - 127) per 32-column block."""
+    q = np.asarray(q_rows).view(np.float16).astype(np.float64)
+    s = np.ldexp(1.0, np.asarray(scale_rows, np.int64) - 127)
+    return q * np.repeat(s, 32, axis=1)
 
 
 def expert_rows(pad_offsets: np.ndarray, counts: np.ndarray, e: int) -> np.ndarray:
@@ -118,8 +140,12 @@ def assert_codes_near(got_q, got_s, ref_q, ref_s, ref_vals, what: str, max_frac=
     """MX codes computed from fp32 (device) and fp64 (oracle) values of the same quantity:
     equal except where the value sits on a rounding boundary.  At most ``max_frac`` of the
     elements may differ; a differing code under an equal scale must be the neighbour of the
-    oracle's and the oracle's value must lie next to the midpoint of the two codes' values
-    (within 1e-4 relative: the fp32 evaluation's error is ~1e-6)."""
+    oracle's, and the oracle's value must lie within 5% of one E4M3 step of the midpoint of
+    the two codes' values (a systematic error -- a wrong rounding rule, a wrong scale --
+    would put it anywhere up to half a step away; the device's fp32 GEMM accumulation over
+    thousands of products moves values by up to ~1e-3 relative, a few percent of a step).
+    A pair +0 / -0 is the zero boundary itself: the value rounds to zero either way, its
+    sign decided by a rounding far below the smallest step."""
     from oracle import mxfp8 as omx
     got_q, ref_q = np.asarray(got_q), np.asarray(ref_q)
     scale_eq = np.repeat(np.asarray(got_s) == np.asarray(ref_s), 32, axis=1)
@@ -133,5 +159,12 @@ def assert_codes_near(got_q, got_s, ref_q, ref_s, ref_vals, what: str, max_frac=
         assert np.all(np.abs((g & 0x7F) - (r & 0x7F)) <= 1), what
         sc = np.repeat(omx.e8m0_decode(np.asarray(ref_s)), 32, axis=1)[sel]
         v = np.asarray(ref_vals)[sel] / sc
-        mid = 0.5 * (omx.e4m3_decode(got_q[sel]) + omx.e4m3_decode(ref_q[sel]))
-        assert np.all(np.abs(np.abs(v) - np.abs(mid)) <= 1e-4 * np.abs(v) + 1e-30), what
+        gv, rv = omx.e4m3_decode(got_q[sel]), omx.e4m3_decode(ref_q[sel])
+        zero = (gv == 0) & (rv == 0)            # +0 against -0
+        assert np.all(np.abs(v[zero]) <= 2.0 ** -10), what   # rounds to zero either way
+        step = np.abs(gv - rv)[~zero]
+        if step.size:
+            off = np.abs(np.abs(v[~zero]) - np.abs(0.5 * (gv + rv)[~zero])) / step
+            print(f"  {what}: differing codes sit within {off.max():.2e} of a step of the "
+                  f"midpoint ({int(zero.sum())} signed zeros)")
+            assert np.all(off <= 0.05), what

@@ -51,7 +51,8 @@ def test_sizes(lib):
     assert lib.moe_weights_bytes(ctypes.byref(D), 0) == 256 * 4096 * 7168
     assert lib.moe_weights_bytes(ctypes.byref(D), 3) == 256 * 7168 * 2048 // 32
     assert lib.moe_weights_bytes(ctypes.byref(D), 8) == -1
-    assert lib.moe_workspace_bytes(ctypes.byref(D), 1) > R * 7168 * 5
+    # permuted MX codes (1 byte) + scaled-fp16 expert outputs (2 bytes) per padded row element
+    assert lib.moe_workspace_bytes(ctypes.byref(D), 1) > R * 7168 * 3
     assert lib.moe_workspace_bytes(ctypes.byref(D), 7) == 0
 
 
@@ -134,9 +135,11 @@ def test_workspace_offsets(lib):
     assert lib.moe_workspace_offset(ctypes.byref(D), 1, WS_BUFFERS["dxa"]) == -1
     assert lib.moe_workspace_offset(ctypes.byref(D), 2, WS_BUFFERS["y"]) == -1
     assert lib.moe_workspace_offset(ctypes.byref(D), 4, 0) == -1
-    # the forward's expert outputs hold R fp32 rows of d
+    # the forward's expert outputs: R rows of d scaled-fp16 values, then their scale bytes
     y = lib.moe_workspace_offset(ctypes.byref(D), 1, WS_BUFFERS["y"])
-    assert y + 4 * R * 2048 <= lib.moe_workspace_bytes(ctypes.byref(D), 1)
+    ys = lib.moe_workspace_offset(ctypes.byref(D), 1, WS_BUFFERS["y_s"])
+    assert y + 2 * R * 2048 <= ys
+    assert ys + R * 2048 // 32 <= lib.moe_workspace_bytes(ctypes.byref(D), 1)
 
 
 def test_bf16_variant_and_router_backward_checks(lib):

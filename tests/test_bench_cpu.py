@@ -82,7 +82,8 @@ def test_layer_summary_closed_form():
     assert r["route_permute_combine_hbm_frac"] == pytest.approx(mv / 0.55e-3 / 5e12)
     impl = bench.implementation_bytes(case, True, rows_used=A + 1000, rows_out=A + 500)
     alg = bench.algorithmic_bytes(case, True)
-    assert impl["combine"] - alg["combine"] == 2 * A * case.d     # fp32 instead of bf16 rows
+    # scaled fp16 rows (2 bytes + a scale byte per 32) instead of bf16
+    assert impl["combine"] - alg["combine"] == pytest.approx(A * case.d / 32)
     assert impl["bwd_transpose"] > alg["bwd_transpose"]           # padded rows
     bwd_stages = dict(fwd_stages, bwd_dout=0.2, bwd_dgrad_down=1.3, bwd_swiglu=0.4,
                       bwd_dgrad_gateup=2.7, bwd_dx=0.3, bwd_transpose=1.0, bwd_wgrad=6.2)

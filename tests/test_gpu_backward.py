@@ -70,11 +70,11 @@ def _check(moe, case, tokens=None, experts=None):
     assert_close_out(dx[rows], ref["dx"][rows])
     dw = to_np(grads["dw_route"]).astype(np.float64)
     print(f"{case.name} dw_route:")
-    assert_close_out(dw[rows], ref["dw"][rows])
+    assert_close_out(dw[rows], ref["dw"][rows], out_bf16=False)
     if experts is not None:           # every assignment of the listed experts
         sel = np.isin(ref["idx"].ravel(), experts)
         print(f"{case.name} dw_route of experts {experts} ({int(sel.sum())} assignments):")
-        assert_close_out(dw.ravel()[sel], ref["dw"].ravel()[sel])
+        assert_close_out(dw.ravel()[sel], ref["dw"].ravel()[sel], out_bf16=False)
     names = ("dWg", "dWu", "dWd")
     n_el = n_out = 0
     worst = 0.0

@@ -8,11 +8,13 @@ one place cannot hide in, or spread from, another:
   multiple of 128 rows and of an empty one (where the layout has them): the requantised
   SwiGLU output codes against the oracle (equal except on rounding boundaries, next to the
   midpoint), the expert outputs y against fp64 arithmetic on the device's own h codes
-  (only the kernel's fp32 accumulation differs) and against the oracle end to end;
+  (only the kernel's fp32 accumulation and the scaled-fp16 storage of y differ) and
+  against the oracle end to end;
 * backward: the token-direction MX operands of the weight gradients bit-exact against the
   oracle's quantiser applied to the device's data-path operands; the weight-gradient GEMM
   against fp64 matmul of those identical operands at the layer tolerance (relative
-  Frobenius <= 2e-3, max-abs <= 3e-2*RMS); the dgrad GEMMs, d(combine weight) and the
+  Frobenius <= 2e-3, max-abs <= 3e-2*RMS beyond each element's own rounding to the bf16
+  output); the dgrad GEMMs, d(combine weight) and the
   SwiGLU backward codes likewise on the device's own inputs; dX from the device's
   per-assignment rows.
 """
@@ -24,11 +26,17 @@ from oracle import layer as olayer
 from oracle import mxfp8 as omx
 from tests.gpu_util import (assert_close_out, assert_codes_near, assert_stage_close,
                             bf16_tensor_f64, bits_to_bf16_tensor, canonical_scales,
-                            expert_rows, mx_values, pick_experts, to_np)
+                            expert_rows, f16s_values, mx_values, pick_experts, rel_fro,
+                            to_np)
 
 pytestmark = pytest.mark.gpu
 
-STAGE_REL = 1e-5     # fp32 accumulation against fp64 on identical operands
+# Stage tolerances on identical operands.  The GEMMs accumulate in fp32 (~1e-7 relative
+# here); their results y, G and dXa are then stored as scaled fp16, whose rounding moves
+# each value by at most 2^-11 of itself (fp16 unit roundoff), so the relative Frobenius
+# error of a stored result stays below 2^-11 + the accumulation's share.
+STAGE_REL = 1e-5
+STAGE_REL_F16S = 2.0 ** -11 + 2e-5
 
 
 @pytest.fixture(scope="module")
@@ -69,7 +77,8 @@ def test_forward_full_experts(moe, name):
     counts, offsets = to_np(saved.bufs["counts"]), to_np(saved.bufs["offsets"])
     pad, perm = to_np(saved.bufs["pad_offsets"]), to_np(saved.bufs["perm"])
     hs_all = to_np(saved.bufs["hs"])
-    y = moe.workspace_view(ws, dims, moe.OP_FORWARD, "y", 4 * R * d).view(torch.float32)
+    y = moe.workspace_view(ws, dims, moe.OP_FORWARD, "y", 2 * R * d).view(torch.int16)
+    ys = moe.workspace_view(ws, dims, moe.OP_FORWARD, "y_s", R * (d // 32))
     picks = pick_experts(counts)
     assert "short_last_tile" in picks
     if name == "imbalance":
@@ -87,10 +96,15 @@ def test_forward_full_experts(moe, name):
         hs = canonical_scales(hs_all, R, f, rows)
         what = f"{name} expert {e} ({label}, {counts[e]} rows)"
         assert_codes_near(hq, hs, hq_ref, hs_ref, hpre, what + " h codes")
-        y_gpu = _host_rows(y, R, d, rows).astype(np.float64)
-        assert_stage_close(y_gpu, mx_values(hq, hs) @ W.fwd()[2].T, STAGE_REL, what + " y")
-        print(f"  {what} y end to end:")
-        assert_close_out(y_gpu, y_ref)
+        y_gpu = f16s_values(_host_rows(y, R, d, rows), _host_rows(ys, R, d // 32, rows))
+        assert_stage_close(y_gpu, mx_values(hq, hs) @ W.fwd()[2].T, STAGE_REL_F16S, what + " y")
+        # end to end (through the device's and the oracle's own h codes, which differ at
+        # rounding boundaries): the relative Frobenius bound; an element of y moves by a
+        # few percent of RMS where one of its h codes flipped, so the element-wise bound
+        # is applied to the layer output (sampled tokens, test_gpu_gemm_forward.py)
+        e2e = rel_fro(y_gpu, y_ref)
+        print(f"  {what} y end to end: rel_fro {e2e:.3e}")
+        assert e2e <= 2e-3
     del out
 
 
@@ -140,8 +154,10 @@ def _backward_stage_parity(moe, case, experts=None, dx_tokens=None):
     usb = moe.umma_scale_bytes
     dq_s = to_np(wsv("dout_s", usb(R, d)))
     dgu_s = to_np(wsv("dgu_s", usb(R, 2 * f)))
-    G = wsv("g", 4 * R * f).view(torch.float32)
-    dxa = wsv("dxa", 4 * R * d).view(torch.float32)
+    G = wsv("g", 2 * R * f).view(torch.int16)
+    Gs = wsv("g_s", R * (f // 32))
+    dxa = wsv("dxa", 2 * R * d).view(torch.int16)
+    dxas = wsv("dxa_s", R * (d // 32))
     tr = {nm: (wsv(nm + "_q", C * R),
                canonical_scales(to_np(wsv(nm + "_s", usb(C, R))), C, R, np.arange(C)), C)
           for nm, C in (("xt", d), ("ht", f), ("gt", 2 * f), ("yt", d))}
@@ -185,9 +201,9 @@ def _backward_stage_parity(moe, case, experts=None, dx_tokens=None):
             print(f"  {what} {nm} stage:")
             assert_close_out(bf16_tensor_f64(grads[nm][e]), ref)
         # 3. dgrad of the down projection, d(combine weight), SwiGLU backward codes
-        g_gpu = _host_rows(G, R, f, rows).astype(np.float64)
+        g_gpu = f16s_values(_host_rows(G, R, f, rows), _host_rows(Gs, R, f // 32, rows))
         wdT = _weights_rows(pw, "wdT", wdT_s, E * f, d, e * f + np.arange(f))
-        assert_stage_close(g_gpu, mx_values(dq, dsc) @ wdT.T, STAGE_REL, what + " G")
+        assert_stage_close(g_gpu, mx_values(dq, dsc) @ wdT.T, STAGE_REL_F16S, what + " G")
         assert_stage_close(dw_gpu[asg], np.sum(g_gpu * H, axis=1), STAGE_REL,
                            what + " d(combine weight)")
         gu = bf16_tensor_f64(saved.bufs["gu"].view(R, 2 * f).index_select(0, _rows_t(rows)))
@@ -199,14 +215,15 @@ def _backward_stage_parity(moe, case, experts=None, dx_tokens=None):
         assert_codes_near(dgu_q, dgu_sc, ref_q, ref_s, dgdu, what + " [dg|du] codes")
         # 4. dgrad of gate/up
         wguT = _weights_rows(pw, "wguT", wguT_s, E * d, 2 * f, e * d + np.arange(d))
-        assert_stage_close(_host_rows(dxa, R, d, rows).astype(np.float64), DGU @ wguT.T,
-                           STAGE_REL, what + " dXa")
+        dxa_rows = f16s_values(_host_rows(dxa, R, d, rows), _host_rows(dxas, R, d // 32, rows))
+        assert_stage_close(dxa_rows, DGU @ wguT.T, STAGE_REL_F16S, what + " dXa")
     # 5. dX = sum over the token's k rows of dXa
     toks = np.arange(case.T) if dx_tokens is None else np.asarray(dx_tokens)
     a = (toks[:, None] * k + np.arange(k)[None, :]).ravel()
     e_of = sb["topk_idx"][a]
     prow = pad[e_of] + (sb["inv_perm"][a] - offsets[e_of])
-    rows_dxa = _host_rows(dxa, R, d, prow).astype(np.float64).reshape(toks.size, k, d)
+    rows_dxa = f16s_values(_host_rows(dxa, R, d, prow), _host_rows(dxas, R, d // 32, prow))
+    rows_dxa = rows_dxa.reshape(toks.size, k, d)
     print(f"  {case.name} dX stage:")
     assert_close_out(bf16_tensor_f64(grads["dx"])[toks], rows_dxa.sum(axis=1))
     return counts

@@ -112,6 +112,27 @@ moe_status make_out_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Output maps of a scaled-fp16 result [rows, cols]: box 64 columns x 32 rows with
+// 128-byte swizzle (the regular tiles) and box 32 x 32 unswizzled (swapped last tiles).
+moe_status make_f16s_tmaps(CUtensorMap* m64, CUtensorMap* m32, const void* base, int64_t rows,
+                           int64_t cols) {
+  auto fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+  cuuint32_t estr[2] = {1u, 1u};
+  cuuint32_t box64[2] = {64u, 32u};
+  cuuint32_t box32[2] = {32u, 32u};
+  CUresult r = fn(m64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box64, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
+  r = fn(m32, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box32,
+         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 inline moe_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // ---------------------------------------------------------------------------------------
@@ -185,10 +206,10 @@ struct WsLayout {
   int64_t zero_begin = 64, zero_bytes = 0;
   int64_t flags = 0, agg = 0, incl = 0, rank = 0, mtile = 0, ready = 0, order = 0;
   int64_t idx = 0, w = 0, counts = 0, offsets = 0, perm = 0, inv = 0, pad = 0;
-  int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0;
+  int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0, ys = 0;
   int64_t tq = 0, ts = 0;  // per-token MX copy of x (forward) or dout (backward)
   // backward
-  int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, gbuf = 0;
+  int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, dxas = 0, gbuf = 0, gs = 0;
   int64_t xt_q = 0, xt_s = 0, ht_q = 0, ht_s = 0, gt_q = 0, gt_s = 0, yt_q = 0, yt_s = 0;
   int64_t total = 0;
 };
@@ -237,7 +258,8 @@ WsLayout ws_layout(const moe_dims* D, int op) {
     L.pad = c.take(4 * (E + 1));
     L.xq = c.take(2 * R * D->d);   // bf16 rows of x in padded expert order
     L.hq = c.take(2 * R * D->f);   // bf16 h
-    L.y = c.take(4 * R * D->d);
+    L.y = c.take(2 * R * D->d);    // scaled fp16 expert outputs
+    L.ys = c.take(R * (D->d / 32));
     L.total = c.off;
     return L;
   }
@@ -247,8 +269,10 @@ WsLayout ws_layout(const moe_dims* D, int op) {
     L.ds = c.take(moe_umma_scale_bytes(R, d));
     L.dgu_q = c.take(R * 2 * f);
     L.dgu_s = c.take(moe_umma_scale_bytes(R, 2 * f));
-    L.dxa = c.take(4 * R * d);
-    L.gbuf = c.take(4 * R * f);
+    L.dxa = c.take(2 * R * d);     // scaled fp16
+    L.dxas = c.take(R * (d / 32));
+    L.gbuf = c.take(2 * R * f);    // scaled fp16
+    L.gs = c.take(R * (f / 32));
     L.xt_q = c.take(d * R);
     L.xt_s = c.take(moe_umma_scale_bytes(d, R));
     L.ht_q = c.take(f * R);
@@ -272,7 +296,8 @@ WsLayout ws_layout(const moe_dims* D, int op) {
     L.xs = c.take(moe_umma_scale_bytes(R, D->d));
     L.hq = c.take(R * D->f);
     L.hs = c.take(moe_umma_scale_bytes(R, D->f));
-    L.y = c.take(4 * R * D->d);
+    L.y = c.take(2 * R * D->d);    // scaled fp16 expert outputs
+    L.ys = c.take(R * (D->d / 32));
   }
   L.total = c.off;
   return L;
@@ -432,6 +457,7 @@ int64_t moe_workspace_offset(const moe_dims* D, int32_t op, int32_t buffer) {
   const WsLayout L = ws_layout(D, op);
   if (buffer == MOE_WS_MTILE) return L.mtile;
   if ((op == MOE_OP_FORWARD || op == MOE_OP_FORWARD_BF16) && buffer == MOE_WS_Y) return L.y;
+  if ((op == MOE_OP_FORWARD || op == MOE_OP_FORWARD_BF16) && buffer == MOE_WS_Y_S) return L.ys;
   if ((op == MOE_OP_FORWARD || op == MOE_OP_FORWARD_BF16) && buffer == MOE_WS_COUNTS)
     return L.counts;
   if (op != MOE_OP_BACKWARD) return -1;
@@ -439,6 +465,8 @@ int64_t moe_workspace_offset(const moe_dims* D, int32_t op, int32_t buffer) {
     case MOE_WS_DOUT_Q: return L.dq;
     case MOE_WS_DOUT_S: return L.ds;
     case MOE_WS_G: return L.gbuf;
+    case MOE_WS_G_S: return L.gs;
+    case MOE_WS_DXA_S: return L.dxas;
     case MOE_WS_DGU_Q: return L.dgu_q;
     case MOE_WS_DGU_S: return L.dgu_s;
     case MOE_WS_DXA: return L.dxa;
@@ -713,7 +741,8 @@ moe_status moe_forward_bf16(const moe_dims* D, const uint16_t* wgu_t, const uint
   int32_t* mtile = at<int32_t>(ws, L.mtile);
   uint16_t* xp = at<uint16_t>(ws, L.xq);
   uint16_t* h16 = at<uint16_t>(ws, L.hq);
-  float* y = at<float>(ws, L.y);
+  uint16_t* y = at<uint16_t>(ws, L.y);
+  uint8_t* ys = at<uint8_t>(ws, L.ys);
   int32_t* status = at<int32_t>(ws, 0);
   if (D->T == 0) return route_empty(D, counts, offsets, mtile, pad, st);
   {
@@ -780,7 +809,8 @@ moe_status moe_forward_bf16(const moe_dims* D, const uint16_t* wgu_t, const uint
     MOE_TRY(make_tmap(&ta, h16, R, 2 * static_cast<int64_t>(D->f), 128));
     MOE_TRY(make_tmap(&tb, wd_t, static_cast<int64_t>(D->E) * D->d,
                       2 * static_cast<int64_t>(D->f), 256));
-    MOE_TRY(make_out_tmap(&ty, y, R, D->d, false));
+    CUtensorMap ty32;
+    MOE_TRY(make_f16s_tmaps(&ty, &ty32, y, R, D->d));
     GemmParams P = {};
     P.G = D->E;
     P.N = D->d;
@@ -789,12 +819,14 @@ moe_status moe_forward_bf16(const moe_dims* D, const uint16_t* wgu_t, const uint
     P.rows_valid = counts;
     P.status = status;
     P.tile_ctr = at<uint32_t>(ws, kCtrFwdDown);
-    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, ty, ty, P, sms, st)));
+    P.out_scales = ys;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, ty, ty32, P, sms, st)));
   }
   {
     StageScope sc(MOE_STAGE_COMBINE, st);
     CombineParams P;
     P.y = y;
+    P.ys = ys;
     P.topk_w = w;
     P.topk_idx = idx;
     P.inv = inv;
@@ -854,7 +886,8 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
   uint8_t* hs = saved ? saved->hs : at<uint8_t>(ws, L.hs);
   uint16_t* gu = saved ? saved->gu : nullptr;
   int32_t* mtile = at<int32_t>(ws, L.mtile);
-  float* y = at<float>(ws, L.y);
+  uint16_t* y = at<uint16_t>(ws, L.y);
+  uint8_t* ys = at<uint8_t>(ws, L.ys);
   int32_t* status = at<int32_t>(ws, 0);
 
   if (D->T == 0) return route_empty(D, counts, offsets, mtile, pad, st);
@@ -918,14 +951,16 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
     P.sfb = W->wd_s;
     P.status = status;
     P.tile_ctr = at<uint32_t>(ws, kCtrFwdDown);
-    CUtensorMap ty;
-    MOE_TRY(make_out_tmap(&ty, y, R, D->d, false));
-    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, ty, ty, P, sms, st)));
+    P.out_scales = ys;
+    CUtensorMap ty, ty32;
+    MOE_TRY(make_f16s_tmaps(&ty, &ty32, y, R, D->d));
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, ty, ty32, P, sms, st)));
   }
   {
     StageScope sc(MOE_STAGE_COMBINE, st);
     CombineParams P;
     P.y = y;
+    P.ys = ys;
     P.topk_w = w;
     P.topk_idx = idx;
     P.inv = inv;
@@ -973,8 +1008,10 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
   uint8_t* dsc = at<uint8_t>(ws, L.ds);
   uint8_t* dgu_q = at<uint8_t>(ws, L.dgu_q);
   uint8_t* dgu_s = at<uint8_t>(ws, L.dgu_s);
-  float* dxa = at<float>(ws, L.dxa);
-  float* gbuf = at<float>(ws, L.gbuf);
+  uint16_t* dxa = at<uint16_t>(ws, L.dxa);
+  uint8_t* dxas = at<uint8_t>(ws, L.dxas);
+  uint16_t* gbuf = at<uint16_t>(ws, L.gbuf);
+  uint8_t* gs = at<uint8_t>(ws, L.gs);
 
   // grouped-GEMM tile counters start at zero
   MOE_TRY(cuda_ok(cudaMemsetAsync(at<uint8_t>(ws, 64), 0, 64, st)));
@@ -997,12 +1034,12 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
                             at<uint8_t>(ws, L.tq), at<uint8_t>(ws, L.ts), dq, dsc, status, sms,
                             st, ready, mb));
     }
-    {  // G = dout^ . Wd'^T (fp32, padded expert order)
+    {  // G = dout^ . Wd'^T (scaled fp16, padded expert order)
       StageScope sc(MOE_STAGE_BWD_DGRAD_DOWN, st);
-      CUtensorMap ta, tb, tg;
+      CUtensorMap ta, tb, tg, tg32;
       MOE_TRY(make_tmap(&ta, dq, R, d, 128));
       MOE_TRY(make_tmap(&tb, W->wdT_q, static_cast<int64_t>(E) * f, d, 256));
-      MOE_TRY(make_out_tmap(&tg, gbuf, R, f, false));
+      MOE_TRY(make_f16s_tmaps(&tg, &tg32, gbuf, R, f));
       GemmParams P = {};
       P.G = E;
       P.N = f;
@@ -1016,12 +1053,14 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.tile_ctr = at<uint32_t>(ws, kCtrBwdDgradDown);
       P.ready = ready;
       P.ready_rows = mb;
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg, P, sms, st, true)));
+      P.out_scales = gs;
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg32, P, sms, st, true)));
     }
     {  // d(router weights), SwiGLU backward, [dg|du] -> MXFP8 along f
       StageScope sc(MOE_STAGE_BWD_SWIGLU, st);
       SwigluBwdParams P;
       P.G = gbuf;
+      P.Gs = gs;
       P.gu = S->gu;
       P.h_q = S->hq;
       P.h_s = S->hs;
@@ -1053,14 +1092,16 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.sfb = W->wguT_s;
       P.status = status;
       P.tile_ctr = at<uint32_t>(ws, kCtrBwdDgradGateUp);
-      CUtensorMap tx;
-      MOE_TRY(make_out_tmap(&tx, dxa, R, d, false));
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tx, tx, P, sms, st)));
+      P.out_scales = dxas;
+      CUtensorMap tx, tx32;
+      MOE_TRY(make_f16s_tmaps(&tx, &tx32, dxa, R, d));
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tx, tx32, P, sms, st)));
     }
     {  // push reverse-dispatch: dX[t] = sum_j dXa[row of (t, j)]
       StageScope sc(MOE_STAGE_BWD_DX, st);
       CombineParams P;
       P.y = dxa;
+      P.ys = dxas;
       P.topk_w = nullptr;
       P.topk_idx = S->topk_idx;
       P.inv = S->inv_perm;

@@ -3,6 +3,7 @@
 // the MXFP8 (E4M3 + E8M0) block quantiser.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -358,6 +359,37 @@ __host__ __device__ __forceinline__ int64_t umma_scale_offset(int64_t r, int64_t
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// ----------------------------------------------------------------------------------------
+// Scaled fp16 ("F16S"), the storage of the fp32 intermediates that one kernel writes and
+// the next one reads back (expert outputs y, the dgrad results G and dXa): 32 consecutive
+// values share a power-of-two scale 2^s, stored as the byte s + 127, and each value is the
+// fp16 (round to nearest even) of v * 2^-s.  s = floor(log2 amax) - 14 puts the block's
+// largest magnitude in [2^14, 2^15), below the fp16 maximum; each value keeps 11
+// significant bits (relative error <= 2^-12 of its binade), where fp32 would cost twice
+// the bytes.
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ int f16s_scale_exp(float amax) {
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127;
+  return max(min(e - 14, 113), -127);  // 2^-s stays a normal fp32 number
+}
+
+// Two fp32 -> two fp16 (lo in bits 0-15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 2^s from its stored byte s + 127 (byte 0: 2^-127, a subnormal fp32 number).
+__device__ __forceinline__ float f16s_scale_value(uint32_t b) {
+  return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
+}
+
+// fp16 bits -> fp32 (exact).
+__device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
+}
 
 // Two fp32 -> two bf16 (lo in bits 0-15), round to nearest even, one instruction.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

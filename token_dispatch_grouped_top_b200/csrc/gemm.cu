@@ -508,6 +508,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint8_t* buf = S.stg[2 * (warp - 2) + stg_buf];
             if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
+            const int32_t xc = x0 + 128 * (c >> 1);
+            if (P.out_scales) {
+              // scaled fp16: a token's 32 features are this warp's 32 lanes, so each
+              // block's magnitude is a max over the lanes (non-negative floats order as
+              // their bit patterns); staged unswizzled as 32 tokens x 64 bytes
+              uint32_t my_sb = 0;
+#pragma unroll
+              for (int r = 0; r < 32; ++r) {
+                const uint32_t am = __reduce_max_sync(kFull, __float_as_uint(fabsf(v[r])));
+                const int sx = f16s_scale_exp(__uint_as_float(am));
+                if (lane == r) my_sb = static_cast<uint32_t>(sx + 127);
+                *reinterpret_cast<__half*>(buf + r * 64 + lane * 2) =
+                    __float2half_rn(v[r] * mx_inv_scale(sx));
+              }
+              P.out_scales[static_cast<int64_t>(y0 + tb + lane) * (P.N >> 5) + (xc >> 5)] =
+                  static_cast<uint8_t>(my_sb);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmC1, smem_u32(buf), xc, y0 + tb);
+                bulk_commit();
+              }
+              stg_buf ^= 1;
+              continue;
+            }
 #pragma unroll
             for (int r = 0; r < 32; ++r)  // token r of the chunk, feature = lane
               *reinterpret_cast<float*>(buf + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) +
@@ -515,7 +540,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmC0, smem_u32(buf), x0 + 128 * (c >> 1), y0 + tb);
+              tma_store_2d(&tmC0, smem_u32(buf), xc, y0 + tb);
               bulk_commit();
             }
             stg_buf ^= 1;
@@ -547,6 +572,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int32_t x0 = ti.j * BN + 128 * h;
         const int32_t y = static_cast<int32_t>(ti.a_row0 + 32 * q);
 #pragma unroll
+        if (P.out_scales) {
+          // scaled fp16: each 32-column block of this row gets its own power-of-two scale;
+          // two blocks make one staged 128-byte row (64 fp16 columns)
+          uint32_t sb = 0;
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            uint4 r16[8];
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+              const int c = 2 * c2 + hb;
+              const float* vc = c == 0 ? v0 : c == 1 ? v1 : c == 2 ? v2 : v3;
+              float amax = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(vc[i]));
+              const int sx = f16s_scale_exp(amax);
+              const float inv = mx_inv_scale(sx);
+              sb |= static_cast<uint32_t>(sx + 127) << (8 * c);
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj)
+                r16[4 * hb + jj] = make_uint4(
+                    pack_f16x2(vc[8 * jj] * inv, vc[8 * jj + 1] * inv),
+                    pack_f16x2(vc[8 * jj + 2] * inv, vc[8 * jj + 3] * inv),
+                    pack_f16x2(vc[8 * jj + 4] * inv, vc[8 * jj + 5] * inv),
+                    pack_f16x2(vc[8 * jj + 6] * inv, vc[8 * jj + 7] * inv));
+            }
+            stage_and_store(S.stg[2 * (warp - 2) + stg_buf], r16, &tmC0, x0 + 64 * c2, y, lane);
+            stg_buf ^= 1;
+          }
+          *reinterpret_cast<uint32_t*>(P.out_scales + (ti.a_row0 + m) * (P.N >> 5) + (x0 >> 5)) =
+              sb;
+          continue;
+        }
         for (int c = 0; c < 4; ++c) {
           const float* vc = c == 0 ? v0 : c == 1 ? v1 : c == 2 ? v2 : v3;
           uint4 r16[8];

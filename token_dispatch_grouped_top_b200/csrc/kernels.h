@@ -94,7 +94,8 @@ cudaError_t launch_gather_rows(const GatherParams& P, int num_sms, cudaStream_t 
 // Push combine: out[t] = sum_j w[t,j] * Y[pad_offsets[e] + inv[a] - offsets[e]], bf16.
 // topk_w == nullptr: unit weights (the backward's reverse dispatch, dX = sum_j dXa).
 struct CombineParams {
-  const float* y;        // [R, d] fp32
+  const uint16_t* y;     // [R, d] scaled fp16 values (common.cuh)
+  const uint8_t* ys;     // [R, d/32] their scale bytes
   const float* topk_w;
   const int32_t* topk_idx;
   const int32_t* inv;
@@ -140,7 +141,8 @@ cudaError_t launch_transpose_quant(const CUtensorMap& tm_src, const CUtensorMap&
 
 // SwiGLU backward + d(router weights) per assignment row, from G = dout^ . Wd'^T.
 struct SwigluBwdParams {
-  const float* G;           // [R, f] fp32, padded expert order
+  const uint16_t* G;        // [R, f] scaled fp16 values, padded expert order
+  const uint8_t* Gs;        // [R, f/32] their scale bytes
   const uint16_t* gu;       // [R, 2f] saved bf16 g | u
   const uint8_t* h_q;       // [R, f] forward h codes + UMMA scales
   const uint8_t* h_s;
@@ -208,6 +210,10 @@ struct GemmParams {
   uint8_t* hs;           // GATEUP: UMMA scales of [rows, f]
   uint16_t* gu;          // GATEUP: nullable [rows, 2f] bf16 save of g | u
   uint16_t* h16;         // GATEUP_BF16: [rows, f] bf16 h
+  // STORE_F32 modes: nullable.  When given, D is stored as scaled fp16 (common.cuh) --
+  // fp16 values through tmC0 (box 64 x 32, 128-byte swizzle; swapped tails through tmC1,
+  // box 32 x 32, no swizzle) and one scale byte per 32 columns here, [rows, N/32].
+  uint8_t* out_scales;
   // WGRAD: D[g] rows m < M, cols n < N -> (n < split ? out_a : out_b)[g][m][n mod split]
   uint16_t* out_a;
   uint16_t* out_b;

@@ -154,7 +154,8 @@ cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream) {
 }
 
 // S6: one warp per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
-// ascending, fp32), rounded to bf16.  With unit weights this is the backward's push
+// ascending, fp32; Y read as scaled fp16, each value times its block scale), rounded to
+// bf16.  With unit weights this is the backward's push
 // reverse-dispatch, dX[t] = sum_j dXa[row of (t, j)].
 __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
   __shared__ int s_off[kMaxE + 1];
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
       if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
       continue;
     }
+    const int64_t nsb = P.d >> 5;  // scale bytes per row
     for (int64_t c0 = 0; c0 < P.d; c0 += 256) {
       const int64_t col0 = c0 + lane * 4, col1 = col0 + 128;  // d % 256 == 0
       float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
@@ -195,17 +197,19 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
       for (int j = 0; j < k; ++j) {
         const int64_t row = __shfl_sync(kFull, my_row, j);
         const float w = __shfl_sync(kFull, my_w, j);
-        const float* yr = P.y + row * P.d;
-        const float4 y0 = __ldg(reinterpret_cast<const float4*>(yr + col0));
-        const float4 y1 = __ldg(reinterpret_cast<const float4*>(yr + col1));
-        acc0.x += w * y0.x;
-        acc0.y += w * y0.y;
-        acc0.z += w * y0.z;
-        acc0.w += w * y0.w;
-        acc1.x += w * y1.x;
-        acc1.y += w * y1.y;
-        acc1.z += w * y1.z;
-        acc1.w += w * y1.w;
+        const uint16_t* yr = P.y + row * P.d;
+        const uint2 q0 = __ldg(reinterpret_cast<const uint2*>(yr + col0));
+        const uint2 q1 = __ldg(reinterpret_cast<const uint2*>(yr + col1));
+        const float w0 = w * f16s_scale_value(__ldg(P.ys + row * nsb + (col0 >> 5)));
+        const float w1 = w * f16s_scale_value(__ldg(P.ys + row * nsb + (col1 >> 5)));
+        acc0.x += w0 * f16_bits_to_f32(q0.x);
+        acc0.y += w0 * f16_bits_to_f32(q0.x >> 16);
+        acc0.z += w0 * f16_bits_to_f32(q0.y);
+        acc0.w += w0 * f16_bits_to_f32(q0.y >> 16);
+        acc1.x += w1 * f16_bits_to_f32(q1.x);
+        acc1.y += w1 * f16_bits_to_f32(q1.x >> 16);
+        acc1.z += w1 * f16_bits_to_f32(q1.y);
+        acc1.w += w1 * f16_bits_to_f32(q1.y >> 16);
       }
       uint2 o0, o1;
       o0.x = pack_bf16x2(acc0.x, acc0.y);
@@ -231,9 +235,12 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
 // token, small enough to stay in L2) and writes them to its padded position: codes with
 // 16-byte copies, scales re-laid into the UMMA layout one 4-byte K-group word at a time.
 // The layer's BF16 variant pulls the bf16 rows of x the same way (no scales).
+constexpr int kGatherChunk = 64;  // rows per CTA step; readiness is published per chunk
+
 __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_mt[kMaxE + 1];
+  __shared__ int s_b[kGatherChunk];  // minibatch of each row of the chunk (-1: none)
   // the consumer GEMM (launched as a programmatic dependent) may start now: it waits for
   // each minibatch of rows through the readiness counters, not for this grid to finish
   launch_dependents();
@@ -242,44 +249,65 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
     s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t A = P.T * P.k;
   const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
   const int d = P.d;
   const int64_t kg = d >> 7;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); q < A;
-       q += warps) {
-    int lo = 0, hi = P.E;  // s_off[lo] <= q < s_off[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (s_off[mid] <= q) lo = mid; else hi = mid;
-    }
-    const int a = P.perm[q];
-    const int64_t t = a / P.k;
-    const int64_t p = static_cast<int64_t>(s_mt[lo]) * 128 + (q - s_off[lo]);
-    if (a < 0 || t >= P.T || p >= R) {
-      if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
-      continue;
-    }
-    const int64_t rb = P.row_bytes;
-    const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * rb);
-    uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * rb);
-    const int n16 = static_cast<int>(rb >> 4);
+  const int64_t nchunks = (A + kGatherChunk - 1) / kGatherChunk;
+  // Chunks of consecutive positions in expert order, one per CTA step, so the rows of the
+  // first experts (the ones the GEMM starts with) are published first.
+  for (int64_t chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
+    for (int r = warp; r < kGatherChunk; r += 8) {
+      const int64_t q = chunk * kGatherChunk + r;
+      int b = -1;
+      if (q < A) {
+        int lo = 0, hi = P.E;  // s_off[lo] <= q < s_off[hi]
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (s_off[mid] <= q) lo = mid; else hi = mid;
+        }
+        const int a = P.perm[q];
+        const int64_t t = a / P.k;
+        const int64_t p = static_cast<int64_t>(s_mt[lo]) * 128 + (q - s_off[lo]);
+        if (a < 0 || t >= P.T || p >= R) {
+          if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+        } else {
+          const int64_t rb = P.row_bytes;
+          const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * rb);
+          uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * rb);
+          const int n16 = static_cast<int>(rb >> 4);
 #pragma unroll 4
-    for (int i = lane; i < n16; i += 32) dst[i] = src[i];
-    if (P.s_tok) {
-      const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
-      for (int g = lane; g < kg; g += 32)
-        *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
+          for (int i = lane; i < n16; i += 32) dst[i] = src[i];
+          if (P.s_tok) {
+            const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
+            for (int g = lane; g < kg; g += 32)
+              *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
+          }
+          if (P.ready) b = static_cast<int>(p / P.ready_rows);
+        }
+      }
+      if (P.ready && lane == 0) s_b[r] = b;
     }
     if (P.ready) {
-      // publish the row: every lane's stores are made visible device-wide before the
-      // minibatch counter drops (the consumer reads them after an acquire of the counter)
+      // Publish the chunk: every thread's stores are made visible device-wide, then one
+      // thread lowers the minibatch counters by the chunk's rows (release; the consumer
+      // acquires the counter before its TMA loads read the rows).
       __threadfence();
-      __syncwarp();
-      const int b = static_cast<int>(p / P.ready_rows);
-      if (lane == 0 && b != P.withhold) red_release_add(P.ready + b, -1);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int cur = -1, n = 0;
+        for (int r = 0; r <= kGatherChunk; ++r) {
+          const int b = r < kGatherChunk ? s_b[r] : -1;
+          if (b != cur) {
+            if (cur >= 0 && cur != P.withhold) red_release_add(P.ready + cur, -n);
+            cur = b;
+            n = 0;
+          }
+          ++n;
+        }
+      }
+      __syncthreads();  // s_b is rewritten by the next chunk
     }
   }
 }
@@ -287,11 +315,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
 cudaError_t launch_gather_rows(const GatherParams& P, int num_sms, cudaStream_t stream) {
   const int64_t A = P.T * P.k;
   if (A <= 0) return cudaSuccess;
-  const int64_t blocks = (A + 7) / 8;
-  // Feeding a concurrent GEMM: one CTA per SM, so that each SM keeps room for one GEMM CTA
-  // (its ~213 KB of shared memory and 320 threads) beside it.
-  const int64_t cap = P.ready ? num_sms : 16LL * num_sms;
-  const int grid = static_cast<int>(blocks < cap ? blocks : cap);
+  const int64_t blocks = (A + kGatherChunk - 1) / kGatherChunk;
+  const int grid = static_cast<int>(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
   static bool carveout_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);

@@ -239,14 +239,24 @@ __global__ void __launch_bounds__(kRouteThreads) route_rank_kernel(RouteParams P
       }
       const bool found = code > 0;
       const int n = found ? code : -(code + 2);  // predecessors hi, hi-1, ..., hi-n+1
-#pragma unroll 4
-      for (int i = 0; i < n; ++i) {
-        const int pr = hi - i;
-        const int* src = (found && i == n - 1 ? P.incl : P.agg) + pr * rowE;
+      // The window's count vectors are read with all loads in flight at once (16 per
+      // batch): summing them one L2 round trip at a time made this loop the routing
+      // kernel's critical path.
+      for (int i0 = 0; i0 < n; i0 += 16) {
 #pragma unroll
         for (int r = 0; r < kPer; ++r) {
           const int e = tid + kRouteThreads * r;
-          if (e < E) excl[r] += __ldcg(src + e);
+          if (e < E) {
+            int v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const int i = i0 + u;
+              const int* src = (found && i == n - 1 ? P.incl : P.agg) + (hi - i) * rowE;
+              v[u] = i < n ? __ldcg(src + e) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) excl[r] += v[u];
+          }
         }
       }
       __syncthreads();  // s_flag is rewritten in the next window
