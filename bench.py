@@ -58,7 +58,7 @@ def _workload(case, pass_):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -75,7 +75,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -159,14 +159,14 @@ def algorithmic_bytes(case, bwd: bool) -> dict:
     return by
 
 
-# Bytes per element of the intermediates y, G and dXa: scaled fp16 (2-byte values plus one
-# scale byte per 32).
+# Bytes per element of the intermediates y and dXa: scaled fp16 (2-byte values plus one
+# scale byte per 32); G stays fp32.
 F16S = 2 + 1 / 32
 
 
 def implementation_bytes(case, bwd: bool, rows_used: int, rows_out: int) -> dict:
     """Bytes the kernels actually move where they differ from the algorithmic count:
-    scaled-fp16 expert outputs / dgrad results, and the tile-padded rows (``rows_used``:
+    scaled-fp16 expert outputs and input gradients, fp32 G, and the tile-padded rows (``rows_used``:
     rows inside some expert segment; ``rows_out``: rows a GEMM with such an output
     writes)."""
     T, d, f, k = case.T, case.d, case.f, case.k
@@ -177,8 +177,8 @@ def implementation_bytes(case, bwd: bool, rows_used: int, rows_out: int) -> dict
     impl["down"] = alg["down"] - 2 * A * d + F16S * rows_out * d
     impl["combine"] = F16S * A * d + 2 * T * d
     if bwd:
-        impl["bwd_dgrad_down"] = alg["bwd_dgrad_down"] - 2 * A * f + F16S * rows_out * f
-        impl["bwd_swiglu"] = A * f * (F16S + 4 + 3 * mx)
+        impl["bwd_dgrad_down"] = alg["bwd_dgrad_down"] - 2 * A * f + 4 * rows_out * f
+        impl["bwd_swiglu"] = A * f * (4 + 4 + 3 * mx)
         impl["bwd_dgrad_gateup"] = alg["bwd_dgrad_gateup"] - 2 * A * d + F16S * rows_out * d
         impl["bwd_dx"] = F16S * A * d + 2 * T * d
         impl["bwd_transpose"] = 2 * rows_used * (2 * d + 3 * f) * mx

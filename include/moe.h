@@ -127,7 +127,7 @@ typedef enum {
   MOE_WS_Y = 1,       /* forward: [R,d] expert outputs y, scaled fp16 values (padded order) */
   MOE_WS_DOUT_Q = 2,  /* backward: [R,d] MX codes of dOut gathered to expert order          */
   MOE_WS_DOUT_S = 3,  /*   their UMMA scales                                                */
-  MOE_WS_G = 4,       /* backward: [R,f] G = dOut^ . W_down'^T, scaled fp16 values           */
+  MOE_WS_G = 4,       /* backward: [R,f] fp32 G = dOut^ . W_down'^T                          */
   MOE_WS_DGU_Q = 5,   /* backward: [R,2f] MX codes of [dg | du] (along 2f)                   */
   MOE_WS_DGU_S = 6,
   MOE_WS_DXA = 7,     /* backward: [R,d] per-assignment input gradients, scaled fp16 values  */
@@ -141,7 +141,6 @@ typedef enum {
   MOE_WS_YT_S = 15,
   MOE_WS_COUNTS = 16, /* forward without a saved struct: [E] int32 tokens per expert        */
   MOE_WS_Y_S = 17,    /* forward: [R,d/32] scale bytes of MOE_WS_Y                           */
-  MOE_WS_G_S = 18,    /* backward: [R,f/32] scale bytes of MOE_WS_G                          */
   MOE_WS_DXA_S = 19   /* backward: [R,d/32] scale bytes of MOE_WS_DXA                        */
 } moe_ws_buffer;
 int64_t moe_workspace_offset(const moe_dims* dims, int32_t op, int32_t buffer);

@@ -18,8 +18,7 @@ OP_ROUTE, OP_FORWARD, OP_BACKWARD, OP_FORWARD_BF16 = 0, 1, 2, 3
 # internal workspace buffers that moe_workspace_offset locates (moe_ws_buffer)
 WS_BUFFERS = {"mtile": 0, "y": 1, "dout_q": 2, "dout_s": 3, "g": 4, "dgu_q": 5, "dgu_s": 6,
               "dxa": 7, "xt_q": 8, "xt_s": 9, "ht_q": 10, "ht_s": 11, "gt_q": 12, "gt_s": 13,
-              "yt_q": 14, "yt_s": 15, "counts": 16, "y_s": 17, "g_s": 18,
-              "dxa_s": 19}
+              "yt_q": 14, "yt_s": 15, "counts": 16, "y_s": 17, "dxa_s": 19}
 
 STAGES = ["route", "permute", "gateup", "down", "combine", "bwd_dout", "bwd_dgrad_down",
           "bwd_dgrad_gateup", "bwd_dx", "bwd_transpose", "bwd_wgrad", "bwd_swiglu"]

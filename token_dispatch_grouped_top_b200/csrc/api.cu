@@ -209,7 +209,7 @@ struct WsLayout {
   int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0, ys = 0;
   int64_t tq = 0, ts = 0;  // per-token MX copy of x (forward) or dout (backward)
   // backward
-  int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, dxas = 0, gbuf = 0, gs = 0;
+  int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, dxas = 0, gbuf = 0;
   int64_t xt_q = 0, xt_s = 0, ht_q = 0, ht_s = 0, gt_q = 0, gt_s = 0, yt_q = 0, yt_s = 0;
   int64_t total = 0;
 };
@@ -271,8 +271,7 @@ WsLayout ws_layout(const moe_dims* D, int op) {
     L.dgu_s = c.take(moe_umma_scale_bytes(R, 2 * f));
     L.dxa = c.take(2 * R * d);     // scaled fp16
     L.dxas = c.take(R * (d / 32));
-    L.gbuf = c.take(2 * R * f);    // scaled fp16
-    L.gs = c.take(R * (f / 32));
+    L.gbuf = c.take(4 * R * f);    // fp32: it feeds the MX requantisation of [dg|du]
     L.xt_q = c.take(d * R);
     L.xt_s = c.take(moe_umma_scale_bytes(d, R));
     L.ht_q = c.take(f * R);
@@ -465,7 +464,6 @@ int64_t moe_workspace_offset(const moe_dims* D, int32_t op, int32_t buffer) {
     case MOE_WS_DOUT_Q: return L.dq;
     case MOE_WS_DOUT_S: return L.ds;
     case MOE_WS_G: return L.gbuf;
-    case MOE_WS_G_S: return L.gs;
     case MOE_WS_DXA_S: return L.dxas;
     case MOE_WS_DGU_Q: return L.dgu_q;
     case MOE_WS_DGU_S: return L.dgu_s;
@@ -1010,8 +1008,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
   uint8_t* dgu_s = at<uint8_t>(ws, L.dgu_s);
   uint16_t* dxa = at<uint16_t>(ws, L.dxa);
   uint8_t* dxas = at<uint8_t>(ws, L.dxas);
-  uint16_t* gbuf = at<uint16_t>(ws, L.gbuf);
-  uint8_t* gs = at<uint8_t>(ws, L.gs);
+  float* gbuf = at<float>(ws, L.gbuf);
 
   // grouped-GEMM tile counters start at zero
   MOE_TRY(cuda_ok(cudaMemsetAsync(at<uint8_t>(ws, 64), 0, 64, st)));
@@ -1034,12 +1031,12 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
                             at<uint8_t>(ws, L.tq), at<uint8_t>(ws, L.ts), dq, dsc, status, sms,
                             st, ready, mb));
     }
-    {  // G = dout^ . Wd'^T (scaled fp16, padded expert order)
+    {  // G = dout^ . Wd'^T (fp32, padded expert order)
       StageScope sc(MOE_STAGE_BWD_DGRAD_DOWN, st);
-      CUtensorMap ta, tb, tg, tg32;
+      CUtensorMap ta, tb, tg;
       MOE_TRY(make_tmap(&ta, dq, R, d, 128));
       MOE_TRY(make_tmap(&tb, W->wdT_q, static_cast<int64_t>(E) * f, d, 256));
-      MOE_TRY(make_f16s_tmaps(&tg, &tg32, gbuf, R, f));
+      MOE_TRY(make_out_tmap(&tg, gbuf, R, f, false));
       GemmParams P = {};
       P.G = E;
       P.N = f;
@@ -1053,14 +1050,12 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.tile_ctr = at<uint32_t>(ws, kCtrBwdDgradDown);
       P.ready = ready;
       P.ready_rows = mb;
-      P.out_scales = gs;
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg32, P, sms, st, true)));
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg, P, sms, st, true)));
     }
     {  // d(router weights), SwiGLU backward, [dg|du] -> MXFP8 along f
       StageScope sc(MOE_STAGE_BWD_SWIGLU, st);
       SwigluBwdParams P;
       P.G = gbuf;
-      P.Gs = gs;
       P.gu = S->gu;
       P.h_q = S->hq;
       P.h_s = S->hs;

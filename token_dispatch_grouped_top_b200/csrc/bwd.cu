@@ -204,7 +204,9 @@ cudaError_t launch_transpose_quant(const CUtensorMap& tm_src, const CUtensorMap&
 
 // ---------------------------------------------------------------------------------------
 // SwiGLU backward and d(router weights), one warp per assignment row, after the dgrad GEMM
-// of the down projection has written G = dout^ . Wd'^T (scaled fp16, padded expert order):
+// of the down projection has written G = dout^ . Wd'^T (fp32, padded expert order; it is
+// kept in fp32 because dg, du are requantised from it, where a coarser G would move values
+// across E4M3 rounding boundaries):
 //   dw_route[a] = <G, h^>,  dh = w * G,  dg = dh * u * s * (1 + g (1 - s)),
 //   du = dh * g * s,  s = sigmoid(g)  (g, u: the saved bf16 pre-activations),
 // then [dg | du] quantised to MXFP8 along f (the operand of the dX GEMM).  Lane l covers 8
@@ -259,24 +261,20 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams P) {
     const int64_t row = s_pad[lo] + (q - s_off[lo]);
     const int a = P.perm[q];
     const float w = P.topk_w[a];
-    const uint16_t* Grow = P.G + row * f;
-    const uint8_t* Gsrow = P.Gs + row * (f >> 5);
+    const float* Grow = P.G + row * f;
     const uint16_t* grow = P.gu + row * 2 * f;
     const uint8_t* hrow = P.h_q + row * f;
     float dwp = 0.f;
     for (int c0 = 0; c0 < f; c0 += 256) {
       const int fi = c0 + lane * 8;
-      const uint4 Gq = *reinterpret_cast<const uint4*>(Grow + fi);
-      const float gsc = f16s_scale_value(Gsrow[fi >> 5]);
+      const float4 G0 = *reinterpret_cast<const float4*>(Grow + fi);
+      const float4 G1 = *reinterpret_cast<const float4*>(Grow + fi + 4);
       const uint4 gq = *reinterpret_cast<const uint4*>(grow + fi);
       const uint4 uq = *reinterpret_cast<const uint4*>(grow + f + fi);
       const uint2 hq = *reinterpret_cast<const uint2*>(hrow + fi);
       const uint32_t hsb = P.h_s[umma_scale_offset(row, fi >> 5, f >> 7)];
       const float hsc = hsb ? __uint_as_float(hsb << 23) : __uint_as_float(0x00400000u);
-      const float Gv[8] = {gsc * f16_bits_to_f32(Gq.x), gsc * f16_bits_to_f32(Gq.x >> 16),
-                           gsc * f16_bits_to_f32(Gq.y), gsc * f16_bits_to_f32(Gq.y >> 16),
-                           gsc * f16_bits_to_f32(Gq.z), gsc * f16_bits_to_f32(Gq.z >> 16),
-                           gsc * f16_bits_to_f32(Gq.w), gsc * f16_bits_to_f32(Gq.w >> 16)};
+      const float Gv[8] = {G0.x, G0.y, G0.z, G0.w, G1.x, G1.y, G1.z, G1.w};
       const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
       const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
       const uint32_t hw[2] = {hq.x, hq.y};

@@ -141,8 +141,7 @@ cudaError_t launch_transpose_quant(const CUtensorMap& tm_src, const CUtensorMap&
 
 // SwiGLU backward + d(router weights) per assignment row, from G = dout^ . Wd'^T.
 struct SwigluBwdParams {
-  const uint16_t* G;        // [R, f] scaled fp16 values, padded expert order
-  const uint8_t* Gs;        // [R, f/32] their scale bytes
+  const float* G;           // [R, f] fp32, padded expert order
   const uint16_t* gu;       // [R, 2f] saved bf16 g | u
   const uint8_t* h_q;       // [R, f] forward h codes + UMMA scales
   const uint8_t* h_s;
