@@ -324,7 +324,8 @@ typedef enum {
 
 /* When enabled, every stage launched by moe_forward / moe_backward is bracketed by CUDA
  * events on the launch stream (host-side bookkeeping only; not for use during graph
- * capture).  moe_profile_collect synchronises on the recorded events, writes the summed
+ * capture).  The events serialise the stages (the gate/up GEMM then starts after the dispatch
+ * has finished instead of as its CTAs retire).  moe_profile_collect synchronises on the recorded events, writes the summed
  * milliseconds and the number of bracketed launches per stage id, and clears the record. */
 moe_status moe_profile_enable(int32_t on);
 moe_status moe_profile_collect(double* ms_per_stage, int32_t* launches_per_stage,

@@ -765,7 +765,7 @@ moe_status moe_forward_bf16(const moe_dims* D, const uint16_t* wgu_t, const uint
     G.ready = ready;
     G.ready_rows = mb;
     G.withhold = g_withhold.load();
-    G.row_bytes = 2 * static_cast<int64_t>(D->d);
+      G.row_bytes = 2 * static_cast<int64_t>(D->d);
     G.q_tok = reinterpret_cast<const uint8_t*>(x);
     G.s_tok = nullptr;
     G.T = D->T;

@@ -190,62 +190,34 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
       continue;
     }
     const int64_t nsb = P.d >> 5;  // scale bytes per row
-    // lane covers 8 consecutive columns of each 256-column half of a 512-column step; the
-    // k rows' loads (16 bytes each) are issued before any is used
-    for (int64_t c0 = 0; c0 < P.d; c0 += 512) {
-      float acc[2][8];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[hh][i] = 0.f;
-      const bool second = c0 + 256 < P.d;  // warp-uniform (d % 256 == 0)
-      for (int j0 = 0; j0 < k; j0 += 8) {
-        uint4 q[8][2];
-        float wsc[8][2];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (j0 + u < k) {  // warp-uniform
-            const int64_t row = __shfl_sync(kFull, my_row, j0 + u);
-            const float w = __shfl_sync(kFull, my_w, j0 + u);
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int64_t col = c0 + 256 * hh + 8 * lane;
-              if (hh == 0 || second) {
-                q[u][hh] = __ldg(reinterpret_cast<const uint4*>(P.y + row * P.d + col));
-                wsc[u][hh] = w * f16s_scale_value(__ldg(P.ys + row * nsb + (col >> 5)));
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {  // j ascending: the sum order is fixed
-          if (j0 + u < k) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              if (hh == 0 || second) {
-                const uint32_t wv[4] = {q[u][hh].x, q[u][hh].y, q[u][hh].z, q[u][hh].w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  acc[hh][2 * i] += wsc[u][hh] * f16_bits_to_f32(wv[i]);
-                  acc[hh][2 * i + 1] += wsc[u][hh] * f16_bits_to_f32(wv[i] >> 16);
-                }
-              }
-            }
-          }
-        }
+    for (int64_t c0 = 0; c0 < P.d; c0 += 256) {
+      const int64_t col0 = c0 + lane * 4, col1 = col0 + 128;  // d % 256 == 0
+      float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+#pragma unroll 4
+      for (int j = 0; j < k; ++j) {
+        const int64_t row = __shfl_sync(kFull, my_row, j);
+        const float w = __shfl_sync(kFull, my_w, j);
+        const uint16_t* yr = P.y + row * P.d;
+        const uint2 q0 = __ldg(reinterpret_cast<const uint2*>(yr + col0));
+        const uint2 q1 = __ldg(reinterpret_cast<const uint2*>(yr + col1));
+        const float w0 = w * f16s_scale_value(__ldg(P.ys + row * nsb + (col0 >> 5)));
+        const float w1 = w * f16s_scale_value(__ldg(P.ys + row * nsb + (col1 >> 5)));
+        acc0.x += w0 * f16_bits_to_f32(q0.x);
+        acc0.y += w0 * f16_bits_to_f32(q0.x >> 16);
+        acc0.z += w0 * f16_bits_to_f32(q0.y);
+        acc0.w += w0 * f16_bits_to_f32(q0.y >> 16);
+        acc1.x += w1 * f16_bits_to_f32(q1.x);
+        acc1.y += w1 * f16_bits_to_f32(q1.x >> 16);
+        acc1.z += w1 * f16_bits_to_f32(q1.y);
+        acc1.w += w1 * f16_bits_to_f32(q1.y >> 16);
       }
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (hh == 0 || second) {
-          const int64_t col = c0 + 256 * hh + 8 * lane;
-          uint4 o;
-          o.x = pack_bf16x2(acc[hh][0], acc[hh][1]);
-          o.y = pack_bf16x2(acc[hh][2], acc[hh][3]);
-          o.z = pack_bf16x2(acc[hh][4], acc[hh][5]);
-          o.w = pack_bf16x2(acc[hh][6], acc[hh][7]);
-          *reinterpret_cast<uint4*>(P.out + t * P.d + col) = o;
-        }
-      }
+      uint2 o0, o1;
+      o0.x = pack_bf16x2(acc0.x, acc0.y);
+      o0.y = pack_bf16x2(acc0.z, acc0.w);
+      o1.x = pack_bf16x2(acc1.x, acc1.y);
+      o1.y = pack_bf16x2(acc1.z, acc1.w);
+      *reinterpret_cast<uint2*>(P.out + t * P.d + col0) = o0;
+      *reinterpret_cast<uint2*>(P.out + t * P.d + col1) = o1;
     }
   }
 }
@@ -305,8 +277,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
           const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * rb);
           uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * rb);
           const int n16 = static_cast<int>(rb >> 4);
-          // 8 loads per lane in flight (4 KB per warp) before the stores: the dispatch runs
-          // on few SMs beside the GEMM and needs the memory-level parallelism
+          // 8 loads per lane in flight (4 KB per warp) before the stores
           for (int i0 = lane; i0 < n16; i0 += 32 * 8) {
             uint4 v[8];
 #pragma unroll
@@ -353,11 +324,11 @@ cudaError_t launch_gather_rows(const GatherParams& P, int num_sms, cudaStream_t 
   const int64_t A = P.T * P.k;
   if (A <= 0) return cudaSuccess;
   const int64_t blocks = (A + kGatherChunk - 1) / kGatherChunk;
-  // Feeding a concurrent GEMM (article §02: part of the SMs dispatch while the rest
-  // compute): one CTA on each of a quarter of the SMs, so every SM keeps room for a GEMM
-  // CTA (~208 KB of shared memory, 320 threads) from the start.  Alone: 8 CTAs per SM.
-  const int64_t cap = P.ready ? (num_sms + 3) / 4 : 8LL * num_sms;
-  const int grid = static_cast<int>(blocks < cap ? blocks : cap);
+  // All SMs: the whole grid is resident at once (so the consumer GEMM, a programmatic
+  // dependent, launches at once and takes each SM as its dispatch CTAs finish).  Running
+  // the dispatch on a quarter of the SMs beside the GEMM from the start was measured
+  // slower (the GEMM's registers leave room for only ~8 dispatch warps per SM).
+  const int grid = static_cast<int>(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
   static bool carveout_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
