@@ -69,10 +69,9 @@ struct ModeCfg {
   // A tile with fewer than 128 valid rows (an expert's last tile) runs with the operands
   // swapped: the two 128-row halves of the B tile are the M side of two MMAs and the
   // valid A rows, rounded up to 16, the N side -- the tensor work shrinks with the rows.
-  // (Measured: a gain for the fp32-output GEMMs; with the SwiGLU epilogue, whose
-  // transposed form quantises across lanes, the gate/up GEMM became slower, so it keeps
-  // full tiles.)
-  static constexpr bool kSwapTail = kStoreF32;
+  // In the gate/up modes the halves are the gate and the up rows of the same 128
+  // features, so SwiGLU stays lane-local and a 32-feature MX block is one warp's lanes.
+  static constexpr bool kSwapTail = kStoreF32 || kGateUp;
 };
 
 template <int ST, int NSTG>
@@ -162,6 +161,82 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
   if (MODE == GEMM_WGRAD_BF16)
     return decode_tile_var_k(tile, prefix, P.M / BM, P.N / BN, P.order);
   return decode_tile_var_m(tile, prefix, valid, P.G, P.N / BN, P.N, P.K / BK);
+}
+
+// Swapped last tile of an fp32-output GEMM: the accumulator chunk v holds, for this lane's
+// output column (feature xc + lane), 32 consecutive tokens tb..tb+31.  Stored as 32 rows of
+// the output through shared memory and a TMA store: fp32 (box 32 x 32, 128-byte swizzle,
+// tm32f) or scaled fp16 (box 32 x 32 unswizzled, tm16; a token's 32 features are this
+// warp's lanes, so each block's maximum is taken across the lanes -- the bit patterns of
+// non-negative floats order as the values).  stg: this warp's two staging buffers.
+__device__ __forceinline__ void store_swapped_chunk(const float (&v)[32], int tb, int32_t xc,
+                                                    int32_t y0, int rows, uint8_t (*stg)[4096],
+                                                    int& stg_buf, const GemmParams& P,
+                                                    const CUtensorMap* tm32f,
+                                                    const CUtensorMap* tm16, int lane) {
+  if (tb >= rows) return;  // warp-uniform
+  uint8_t* buf = stg[stg_buf];
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+  if (P.out_scales) {
+    uint32_t my_sb = 0;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const uint32_t am = __reduce_max_sync(kFull, __float_as_uint(fabsf(v[r])));
+      const int sx = f16s_scale_exp(__uint_as_float(am));
+      if (lane == r) my_sb = static_cast<uint32_t>(sx + 127);
+      *reinterpret_cast<__half*>(buf + r * 64 + lane * 2) = __float2half_rn(v[r] * mx_inv_scale(sx));
+    }
+    P.out_scales[static_cast<int64_t>(y0 + tb + lane) * (P.N >> 5) + (xc >> 5)] =
+        static_cast<uint8_t>(my_sb);
+  } else {
+#pragma unroll
+    for (int r = 0; r < 32; ++r)  // token r of the chunk, feature = lane
+      *reinterpret_cast<float*>(buf + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) +
+                                ((lane & 3) << 2)) = v[r];
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(P.out_scales ? tm16 : tm32f, smem_u32(buf), xc, y0 + tb);
+    bulk_commit();
+  }
+  stg_buf ^= 1;
+}
+
+__device__ __forceinline__ float sigmoid_fast(float x);
+
+// Swapped last tile of a gate/up GEMM: g and u hold, for this lane's feature fblk + lane, 32
+// consecutive tokens tb..tb+31 of the tile.  h = silu(g) * u per token, then either bf16
+// (the BF16 variant) or MXFP8 along the features: the 32-feature block is this warp's
+// lanes, its maximum taken across them; each warp store writes one token's 32 contiguous
+// codes (or bf16 values), and lane 0 the block's scale byte.
+template <bool kBf16>
+__device__ __forceinline__ void gateup_swapped_chunk(const float (&g)[32], const float (&u)[32],
+                                                     int tb, int fblk, const TileInfo& ti,
+                                                     const GemmParams& P, int lane) {
+  const int f = P.f;
+  const int feat = fblk + lane;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    if (tb + r < ti.rows) {  // warp-uniform
+      const int64_t row = ti.a_row0 + tb + r;
+      if (P.gu) {
+        P.gu[row * 2 * f + feat] = static_cast<uint16_t>(pack_bf16x2(g[r], 0.f));
+        P.gu[row * 2 * f + f + feat] = static_cast<uint16_t>(pack_bf16x2(u[r], 0.f));
+      }
+      const float hv = g[r] * sigmoid_fast(g[r]) * u[r];
+      if (kBf16) {
+        P.h16[row * f + feat] = static_cast<uint16_t>(pack_bf16x2(hv, 0.f));
+      } else {
+        const uint32_t am = __reduce_max_sync(kFull, __float_as_uint(fabsf(hv)));
+        const int sx = mx_scale_exp(__uint_as_float(am));
+        P.hq[row * f + feat] = static_cast<uint8_t>(cvt_e4m3x2(hv * mx_inv_scale(sx), 0.f) & 0xFFu);
+        if (lane == 0)
+          P.hs[umma_scale_offset(row, fblk >> 5, f >> 7)] = static_cast<uint8_t>(sx + 127);
+      }
+    }
+  }
 }
 
 // sigmoid(x) = 1 / (1 + e^-x) with the fast exponential and a rounded reciprocal: the
@@ -497,54 +572,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&S.tmem_empty));
         acc_phase ^= 1u;
-        if (ModeCfg<MODE>::kStoreF32) {
+        if constexpr (ModeCfg<MODE>::kGateUp) {
+          // d0*: gate, d1*: up, of feature `feat` (this lane) for tokens tok0 + 0..63.  Per
+          // token: h = silu(g) * u, its 32-feature block maximum across the warp (bit
+          // patterns of non-negative floats order as the values), then 32 contiguous code
+          // bytes (or bf16 values) per warp store.
+          const int fblk = (BN / 2) * ti.j + 32 * q;  // first feature of this warp's block
+          gateup_swapped_chunk<ModeCfg<MODE>::kBf16>(d0a, d1a, tok0, fblk, ti, P, lane);
+          gateup_swapped_chunk<ModeCfg<MODE>::kBf16>(d0b, d1b, tok0 + 32, fblk, ti, P, lane);
+        } else if constexpr (ModeCfg<MODE>::kStoreF32) {
           const int32_t y0 = static_cast<int32_t>(ti.a_row0);
           const int32_t x0 = ti.j * BN + 32 * q;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int tb = tok0 + 32 * (c & 1);
-            if (tb >= ti.rows) continue;  // warp-uniform
-            const float* v = c == 0 ? d0a : c == 1 ? d0b : c == 2 ? d1a : d1b;
-            uint8_t* buf = S.stg[2 * (warp - 2) + stg_buf];
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
-            const int32_t xc = x0 + 128 * (c >> 1);
-            if (P.out_scales) {
-              // scaled fp16: a token's 32 features are this warp's 32 lanes, so each
-              // block's magnitude is a max over the lanes (non-negative floats order as
-              // their bit patterns); staged unswizzled as 32 tokens x 64 bytes
-              uint32_t my_sb = 0;
-#pragma unroll
-              for (int r = 0; r < 32; ++r) {
-                const uint32_t am = __reduce_max_sync(kFull, __float_as_uint(fabsf(v[r])));
-                const int sx = f16s_scale_exp(__uint_as_float(am));
-                if (lane == r) my_sb = static_cast<uint32_t>(sx + 127);
-                *reinterpret_cast<__half*>(buf + r * 64 + lane * 2) =
-                    __float2half_rn(v[r] * mx_inv_scale(sx));
-              }
-              P.out_scales[static_cast<int64_t>(y0 + tb + lane) * (P.N >> 5) + (xc >> 5)] =
-                  static_cast<uint8_t>(my_sb);
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&tmC1, smem_u32(buf), xc, y0 + tb);
-                bulk_commit();
-              }
-              stg_buf ^= 1;
-              continue;
-            }
-#pragma unroll
-            for (int r = 0; r < 32; ++r)  // token r of the chunk, feature = lane
-              *reinterpret_cast<float*>(buf + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) +
-                                        ((lane & 3) << 2)) = v[r];
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&tmC0, smem_u32(buf), xc, y0 + tb);
-              bulk_commit();
-            }
-            stg_buf ^= 1;
-          }
+          // one call per 32-token chunk, each with its own register array (indexed with
+          // compile-time offsets only, so the arrays stay in registers)
+          uint8_t(*stg)[4096] = &S.stg[2 * (warp - 2)];
+          store_swapped_chunk(d0a, tok0, x0, y0, ti.rows, stg, stg_buf, P, &tmC0, &tmC1, lane);
+          store_swapped_chunk(d0b, tok0 + 32, x0, y0, ti.rows, stg, stg_buf, P, &tmC0, &tmC1,
+                              lane);
+          store_swapped_chunk(d1a, tok0, x0 + 128, y0, ti.rows, stg, stg_buf, P, &tmC0, &tmC1,
+                              lane);
+          store_swapped_chunk(d1b, tok0 + 32, x0 + 128, y0, ti.rows, stg, stg_buf, P, &tmC0,
+                              &tmC1, lane);
         }
         continue;
       }
@@ -571,7 +619,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // fp32 rows of 128 columns: four 32-column chunks; whole 32-row boxes are written
         const int32_t x0 = ti.j * BN + 128 * h;
         const int32_t y = static_cast<int32_t>(ti.a_row0 + 32 * q);
-#pragma unroll
         if (P.out_scales) {
           // scaled fp16: each 32-column block of this row gets its own power-of-two scale;
           // two blocks make one staged 128-byte row (64 fp16 columns)
@@ -604,6 +651,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               sb;
           continue;
         }
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float* vc = c == 0 ? v0 : c == 1 ? v1 : c == 2 ? v2 : v3;
           uint4 r16[8];
