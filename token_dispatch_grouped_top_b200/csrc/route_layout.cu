@@ -155,8 +155,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_rank_kernel(RouteParams P
   if (warp < kRouteTile / 32) {
     const int g = warp, tl = 32 * g + lane;
     const bool valid = t0 + tl < P.T;
-    if (valid)
-      for (int j = 0; j < k; ++j) atomicOr(&s_mask[g][s_idx[tl][j]], 1u << lane);
+    // lanes choosing the same expert in slot j are grouped first, so each expert's word
+    // takes one atomic per slot instead of one per lane (hot experts are chosen by most
+    // lanes of a group: per-lane atomics on one word serialise)
+    for (int j = 0; j < k; ++j) {
+      const int e = valid ? s_idx[tl][j] : -1 - lane;  // invalid lanes match nobody
+      const uint32_t same = __match_any_sync(kFull, e);
+      if (valid && (same & ((1u << lane) - 1u)) == 0u) atomicOr(&s_mask[g][e], same);
+    }
     __syncwarp();
     if (valid) {
       const uint32_t below = (1u << lane) - 1u;
