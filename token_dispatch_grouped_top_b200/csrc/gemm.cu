@@ -69,9 +69,11 @@ struct ModeCfg {
   // A tile with fewer than 128 valid rows (an expert's last tile) runs with the operands
   // swapped: the two 128-row halves of the B tile are the M side of two MMAs and the
   // valid A rows, rounded up to 16, the N side -- the tensor work shrinks with the rows.
-  // In the gate/up modes the halves are the gate and the up rows of the same 128
-  // features, so SwiGLU stays lane-local and a 32-feature MX block is one warp's lanes.
-  static constexpr bool kSwapTail = kStoreF32 || kGateUp;
+  // Measured: a gain for the fp32 / scaled-fp16 output GEMMs.  The gate/up GEMM keeps
+  // full tiles: its swapped form (SwiGLU lane-local, the MX block maximum across the
+  // warp, one token's codes per warp store) made the epilogue of the tail tiles the
+  // bottleneck (2.26 -> 2.57 ms at the DeepSeek-V3 shape).
+  static constexpr bool kSwapTail = kStoreF32;
 };
 
 template <int ST, int NSTG>
@@ -202,41 +204,6 @@ __device__ __forceinline__ void store_swapped_chunk(const float (&v)[32], int tb
     bulk_commit();
   }
   stg_buf ^= 1;
-}
-
-__device__ __forceinline__ float sigmoid_fast(float x);
-
-// Swapped last tile of a gate/up GEMM: g and u hold, for this lane's feature fblk + lane, 32
-// consecutive tokens tb..tb+31 of the tile.  h = silu(g) * u per token, then either bf16
-// (the BF16 variant) or MXFP8 along the features: the 32-feature block is this warp's
-// lanes, its maximum taken across them; each warp store writes one token's 32 contiguous
-// codes (or bf16 values), and lane 0 the block's scale byte.
-template <bool kBf16>
-__device__ __forceinline__ void gateup_swapped_chunk(const float (&g)[32], const float (&u)[32],
-                                                     int tb, int fblk, const TileInfo& ti,
-                                                     const GemmParams& P, int lane) {
-  const int f = P.f;
-  const int feat = fblk + lane;
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    if (tb + r < ti.rows) {  // warp-uniform
-      const int64_t row = ti.a_row0 + tb + r;
-      if (P.gu) {
-        P.gu[row * 2 * f + feat] = static_cast<uint16_t>(pack_bf16x2(g[r], 0.f));
-        P.gu[row * 2 * f + f + feat] = static_cast<uint16_t>(pack_bf16x2(u[r], 0.f));
-      }
-      const float hv = g[r] * sigmoid_fast(g[r]) * u[r];
-      if (kBf16) {
-        P.h16[row * f + feat] = static_cast<uint16_t>(pack_bf16x2(hv, 0.f));
-      } else {
-        const uint32_t am = __reduce_max_sync(kFull, __float_as_uint(fabsf(hv)));
-        const int sx = mx_scale_exp(__uint_as_float(am));
-        P.hq[row * f + feat] = static_cast<uint8_t>(cvt_e4m3x2(hv * mx_inv_scale(sx), 0.f) & 0xFFu);
-        if (lane == 0)
-          P.hs[umma_scale_offset(row, fblk >> 5, f >> 7)] = static_cast<uint8_t>(sx + 127);
-      }
-    }
-  }
 }
 
 // sigmoid(x) = 1 / (1 + e^-x) with the fast exponential and a rounded reciprocal: the
@@ -572,15 +539,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&S.tmem_empty));
         acc_phase ^= 1u;
-        if constexpr (ModeCfg<MODE>::kGateUp) {
-          // d0*: gate, d1*: up, of feature `feat` (this lane) for tokens tok0 + 0..63.  Per
-          // token: h = silu(g) * u, its 32-feature block maximum across the warp (bit
-          // patterns of non-negative floats order as the values), then 32 contiguous code
-          // bytes (or bf16 values) per warp store.
-          const int fblk = (BN / 2) * ti.j + 32 * q;  // first feature of this warp's block
-          gateup_swapped_chunk<ModeCfg<MODE>::kBf16>(d0a, d1a, tok0, fblk, ti, P, lane);
-          gateup_swapped_chunk<ModeCfg<MODE>::kBf16>(d0b, d1b, tok0 + 32, fblk, ti, P, lane);
-        } else if constexpr (ModeCfg<MODE>::kStoreF32) {
+        if constexpr (ModeCfg<MODE>::kStoreF32) {
           const int32_t y0 = static_cast<int32_t>(ti.a_row0);
           const int32_t x0 = ti.j * BN + 32 * q;
           // one call per 32-token chunk, each with its own register array (indexed with
