@@ -153,80 +153,106 @@ cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// S6: one warp per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
+// S6: one CTA per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
 // ascending, fp32; Y read as scaled fp16, each value times its block scale), rounded to
-// bf16.  With unit weights this is the backward's push
-// reverse-dispatch, dX[t] = sum_j dXa[row of (t, j)].
-__global__ void __launch_bounds__(256) combine_kernel(CombineParams P) {
+// bf16.  With unit weights this is the backward's push reverse-dispatch, dX[t] = sum_j
+// dXa[row of (t, j)].  The CTA reads each of the token's k rows as one contiguous stretch
+// (thread i takes 16-byte chunks i, i + 256, ...), so every DRAM access is a long run of a
+// single row rather than k short pieces of different rows.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineChunks = 4;  // 16-byte chunks per thread per column block
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineParams P) {
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_mt[kMaxE + 1];
+  __shared__ int64_t s_row[32];
+  __shared__ float s_w[32];
+  __shared__ int s_bad;
   for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
     s_off[i] = P.offsets[i];
     s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
   const int k = P.k;
   const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
-       t < P.T; t += warps) {
-    int64_t my_row = 0;
-    float my_w = 0.f;
-    bool bad = false;
-    if (lane < k) {
-      const int64_t a = t * k + lane;
+  const int64_t nsb = P.d >> 5;  // scale bytes per row
+  for (int64_t t = blockIdx.x; t < P.T; t += gridDim.x) {
+    if (tid == 0) s_bad = 0;
+    __syncthreads();
+    if (tid < k) {
+      const int64_t a = t * k + tid;
       const int e = P.topk_idx[a];
-      if (e < 0 || e >= P.E) {
-        bad = true;
-      } else {
-        my_row = static_cast<int64_t>(s_mt[e]) * 128 + (P.inv[a] - s_off[e]);
-        my_w = P.topk_w ? P.topk_w[a] : 1.f;
-        if (my_row < 0 || my_row >= R) bad = true;
+      int64_t row = -1;
+      if (e >= 0 && e < P.E) row = static_cast<int64_t>(s_mt[e]) * 128 + (P.inv[a] - s_off[e]);
+      if (row < 0 || row >= R) {
+        s_bad = 1;
+        row = 0;
       }
+      s_row[tid] = row;
+      s_w[tid] = P.topk_w ? P.topk_w[a] : 1.f;
     }
-    if (__any_sync(kFull, bad)) {
-      if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+    __syncthreads();
+    if (s_bad) {
+      if (tid == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+      __syncthreads();  // s_row / s_bad are rewritten for the next token
       continue;
     }
-    const int64_t nsb = P.d >> 5;  // scale bytes per row
-    for (int64_t c0 = 0; c0 < P.d; c0 += 256) {
-      const int64_t col0 = c0 + lane * 4, col1 = col0 + 128;  // d % 256 == 0
-      float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-#pragma unroll 4
-      for (int j = 0; j < k; ++j) {
-        const int64_t row = __shfl_sync(kFull, my_row, j);
-        const float w = __shfl_sync(kFull, my_w, j);
+    for (int64_t cb = 0; cb < P.d; cb += 8 * kCombineThreads * kCombineChunks) {
+      float acc[kCombineChunks][8];
+#pragma unroll
+      for (int c = 0; c < kCombineChunks; ++c)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[c][i] = 0.f;
+      for (int j = 0; j < k; ++j) {  // j ascending: the sum order is fixed
+        const int64_t row = s_row[j];
+        const float w = s_w[j];
         const uint16_t* yr = P.y + row * P.d;
-        const uint2 q0 = __ldg(reinterpret_cast<const uint2*>(yr + col0));
-        const uint2 q1 = __ldg(reinterpret_cast<const uint2*>(yr + col1));
-        const float w0 = w * f16s_scale_value(__ldg(P.ys + row * nsb + (col0 >> 5)));
-        const float w1 = w * f16s_scale_value(__ldg(P.ys + row * nsb + (col1 >> 5)));
-        acc0.x += w0 * f16_bits_to_f32(q0.x);
-        acc0.y += w0 * f16_bits_to_f32(q0.x >> 16);
-        acc0.z += w0 * f16_bits_to_f32(q0.y);
-        acc0.w += w0 * f16_bits_to_f32(q0.y >> 16);
-        acc1.x += w1 * f16_bits_to_f32(q1.x);
-        acc1.y += w1 * f16_bits_to_f32(q1.x >> 16);
-        acc1.z += w1 * f16_bits_to_f32(q1.y);
-        acc1.w += w1 * f16_bits_to_f32(q1.y >> 16);
+        const uint8_t* sr = P.ys + row * nsb;
+        uint4 q[kCombineChunks];
+        float ws[kCombineChunks];
+#pragma unroll
+        for (int c = 0; c < kCombineChunks; ++c) {
+          const int64_t col = cb + 8 * (tid + kCombineThreads * c);
+          if (col < P.d) {
+            q[c] = __ldg(reinterpret_cast<const uint4*>(yr + col));
+            ws[c] = w * f16s_scale_value(__ldg(sr + (col >> 5)));
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < kCombineChunks; ++c) {
+          const int64_t col = cb + 8 * (tid + kCombineThreads * c);
+          if (col < P.d) {
+            const uint32_t wv[4] = {q[c].x, q[c].y, q[c].z, q[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[c][2 * i] += ws[c] * f16_bits_to_f32(wv[i]);
+              acc[c][2 * i + 1] += ws[c] * f16_bits_to_f32(wv[i] >> 16);
+            }
+          }
+        }
       }
-      uint2 o0, o1;
-      o0.x = pack_bf16x2(acc0.x, acc0.y);
-      o0.y = pack_bf16x2(acc0.z, acc0.w);
-      o1.x = pack_bf16x2(acc1.x, acc1.y);
-      o1.y = pack_bf16x2(acc1.z, acc1.w);
-      *reinterpret_cast<uint2*>(P.out + t * P.d + col0) = o0;
-      *reinterpret_cast<uint2*>(P.out + t * P.d + col1) = o1;
+#pragma unroll
+      for (int c = 0; c < kCombineChunks; ++c) {
+        const int64_t col = cb + 8 * (tid + kCombineThreads * c);
+        if (col < P.d) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[c][0], acc[c][1]);
+          o.y = pack_bf16x2(acc[c][2], acc[c][3]);
+          o.z = pack_bf16x2(acc[c][4], acc[c][5]);
+          o.w = pack_bf16x2(acc[c][6], acc[c][7]);
+          *reinterpret_cast<uint4*>(P.out + t * P.d + col) = o;
+        }
+      }
     }
+    __syncthreads();  // s_row / s_w are rewritten for the next token
   }
 }
 
 cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t stream) {
   if (P.T <= 0) return cudaSuccess;
-  const int64_t blocks = (P.T + 7) / 8;
-  const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
-  combine_kernel<<<grid, 256, 0, stream>>>(P);
+  const int grid = static_cast<int>(P.T < 8LL * num_sms ? P.T : 8LL * num_sms);
+  combine_kernel<<<grid, kCombineThreads, 0, stream>>>(P);
   return cudaGetLastError();
 }
 
@@ -285,7 +311,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
               v[u] = i0 + 32 * u < n16 ? ld_nc_v4(src + i0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-              if (i0 + 32 * u < n16) dst[i0 + 32 * u] = v[u];
+              if (i0 + 32 * u < n16) __stcs(dst + i0 + 32 * u, v[u]);
           }
           if (P.s_tok) {
             const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
