@@ -31,6 +31,7 @@ SCORE_SIGMOID_RENORM = 1
 
 # stream ids for SeedSequence spawning (fixed so that every input has its own stream)
 _STREAM_X, _STREAM_LOGITS, _STREAM_BIAS, _STREAM_DOUT, _STREAM_EXPERT_PICK = 1, 2, 3, 4, 5
+_STREAM_ROUTER, _STREAM_DLOGITS = 6, 7
 _WG, _WU, _WD = 0, 1, 2
 
 
@@ -119,6 +120,18 @@ def make_logits(case: MoeCase) -> np.ndarray:
     """Router logits [T, E] fp32: N(0,1) noise plus the per-expert bias, added in fp32."""
     noise = _rng(case.seed, _STREAM_LOGITS).standard_normal((case.T, case.E), dtype=np.float32)
     return (noise + expert_bias(case)[None, :]).astype(np.float32)
+
+
+def make_router_weight(case: MoeCase) -> np.ndarray:
+    """Router weight W_r [E, d] (one row per expert): bf16 bits of N(0, 1/sqrt(d)) draws, so
+    that x . W_r^T has the unit scale of the configurations' logits."""
+    z = _rng(case.seed, _STREAM_ROUTER).standard_normal((case.E, case.d), dtype=np.float32)
+    return f32_to_bf16_bits(z * np.float32(1.0 / np.sqrt(float(case.d))))
+
+
+def make_dlogits(case: MoeCase) -> np.ndarray:
+    """A gradient of the logits [T, E] fp32: N(0, 1) draws."""
+    return _rng(case.seed, _STREAM_DLOGITS).standard_normal((case.T, case.E), dtype=np.float32)
 
 
 # ---------------------------------------------------------------------------------------
