@@ -64,7 +64,8 @@ typedef enum {
   MOE_OP_ROUTE = 0,
   MOE_OP_FORWARD = 1,
   MOE_OP_BACKWARD = 2,
-  MOE_OP_FORWARD_BF16 = 3  /* moe_forward_bf16 */
+  MOE_OP_FORWARD_BF16 = 3, /* moe_forward_bf16 */
+  MOE_OP_ROUTER = 4        /* moe_router_logits, moe_router_grads */
 } moe_op;
 
 typedef struct {
@@ -269,6 +270,34 @@ moe_status moe_backward(const moe_dims* dims, const moe_weights* w, const moe_sa
 moe_status moe_router_backward(const moe_dims* dims, const float* logits,
                                const int32_t* topk_idx, const float* dw_route, float* dlogits,
                                int32_t* status, void* stream);
+
+/* ---- router GEMM in front of the routing step ------------------------------------------
+ * Article lead and §01 (at every step a router decides which experts each token goes to;
+ * the pages give no formula: read as a bias-free linear layer whose outputs are the
+ * logits moe_route_layout ranks).
+ *   logits[t, e] = sum_i x[t, i] * wr[e, i]
+ * x [T,d] bf16 and wr [E,d] bf16 (one row per expert: a linear layer's weight layout),
+ * row-major; logits [T,E] fp32.  Runs on the tensor cores (tcgen05.mma kind::f16, fp32
+ * accumulation) as a one-group grouped GEMM; W_r is first copied into the workspace padded
+ * to whole 256-expert tiles.  Needs E % 8 == 0 (besides the moe_dims rules); workspace of
+ * moe_workspace_bytes(dims, MOE_OP_ROUTER) bytes, 256-byte aligned, caller-owned, no
+ * zeroing needed; device status latched at its offset 0.  All pointers device memory,
+ * 16-byte aligned; nothing is allocated, nothing synchronised. */
+moe_status moe_router_logits(const moe_dims* dims, const uint16_t* x, const uint16_t* wr,
+                             float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- router GEMM backward ----------------------------------------------------------------
+ * Article lead and §01 (training differentiates through the router).  From the logits'
+ * gradient G [T,E] fp32 (e.g. moe_router_backward's output):
+ *   dx_r[t, i] = sum_e bf16(G[t, e]) * wr[e, i]     [T,d] fp32: the router's share of dx
+ *   dwr[e, i]  = sum_t bf16(G[t, e]) * x[t, i]      [E,d] fp32
+ * bf16(.) rounds to nearest, ties to even: both products run on the tensor cores with bf16
+ * operands and fp32 accumulation, like the forward.  The operand copies it needs (bf16(G)
+ * and its transpose, W_r^T, x^T, zero-padded to whole tiles) live in the workspace
+ * (MOE_OP_ROUTER size).  T == 0 writes dwr = 0.  Same rules as moe_router_logits. */
+moe_status moe_router_grads(const moe_dims* dims, const float* dlogits, const uint16_t* x,
+                            const uint16_t* wr, float* dx_r, float* dwr, void* ws,
+                            size_t ws_bytes, void* stream);
 
 /* ---- grouped block-scaled GEMM (the engine of S4/S5, exposed for direct use) ----------
  * For each group g and each row r in [128*mtile_prefix[g], 128*mtile_prefix[g+1]):

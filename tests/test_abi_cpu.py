@@ -156,3 +156,25 @@ def test_bf16_variant_and_router_backward_checks(lib):
     assert lib.moe_router_backward(ctypes.byref(bad), None, None, None, None, None, None) == 2
     assert lib.moe_workspace_bytes(ctypes.byref(D), 3) > 0
     assert lib.moe_debug_withhold_ready(-1) == 0
+
+
+def test_router_gemm_checks(lib):
+    # host-side checks only: every failing call returns before any device work
+    vp = ctypes.c_void_p
+    D = _dims(T=100, d=512, f=256, E=16, k=2, s=0)
+    n = lib.moe_workspace_bytes(ctypes.byref(D), 4)
+    # header + W_r padded to 256 rows + bf16(G) [128, 64] + its transpose [128, 128]
+    # + W_r^T [512, 64] + x^T [512, 128]
+    assert n >= 256 + 256 * 512 * 2 + 128 * 64 * 2 + 128 * 128 * 2 + 512 * 64 * 2 + 512 * 128 * 2
+    a, ws = vp(1 << 20), vp(1 << 24)
+    E12 = _dims(T=100, d=512, f=256, E=12, k=2, s=0)
+    assert lib.moe_router_logits(ctypes.byref(E12), a, a, a, ws, 1 << 30, None) == 2
+    assert lib.moe_router_logits(ctypes.byref(D), None, a, a, ws, n, None) == 1
+    assert lib.moe_router_logits(ctypes.byref(D), vp((1 << 20) + 8), a, a, ws, n, None) == 3
+    assert lib.moe_router_logits(ctypes.byref(D), a, a, a, vp((1 << 24) + 16), n, None) == 3
+    assert lib.moe_router_logits(ctypes.byref(D), a, a, a, ws, n - 1, None) == 4
+    assert lib.moe_router_grads(ctypes.byref(D), a, a, a, a, None, ws, n, None) == 1
+    assert lib.moe_router_grads(ctypes.byref(E12), a, a, a, a, a, ws, 1 << 30, None) == 2
+    assert lib.moe_router_grads(ctypes.byref(D), a, a, a, a, a, ws, n - 1, None) == 4
+    big = _dims()
+    assert lib.moe_workspace_bytes(ctypes.byref(big), 4) >= 7168 * 8192 * 2

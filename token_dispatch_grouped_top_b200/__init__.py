@@ -14,7 +14,7 @@ from typing import Optional
 
 from . import _lib
 from ._lib import (MoeDims, MoeError, MoeSaved, MoeWeights, OP_BACKWARD, OP_FORWARD,
-                   OP_FORWARD_BF16, OP_ROUTE, SAVED_FIELDS, WEIGHT_FIELDS, WS_BUFFERS, check,
+                   OP_FORWARD_BF16, OP_ROUTE, OP_ROUTER, SAVED_FIELDS, WEIGHT_FIELDS, WS_BUFFERS, check,
                    load)
 
 SCORE_SOFTMAX_TOPK = 0
@@ -23,7 +23,7 @@ SCORE_SIGMOID_RENORM = 1
 __all__ = ["Dims", "PreparedWeights", "Saved", "load", "MoeError", "workspace",
            "route_layout", "mxfp8_quantize", "prepare_weights", "forward", "backward",
            "grouped_gemm_mx", "grouped_gemm_bf16", "prepare_weights_bf16", "forward_bf16",
-           "router_backward", "device_status", "padded_rows", "umma_scale_bytes",
+           "router_backward", "router_logits", "router_grads", "device_status", "padded_rows", "umma_scale_bytes",
            "min_tokens_for_waves", "workspace_view", "profile_enable", "profile_collect",
            "SCORE_SOFTMAX_TOPK", "SCORE_SIGMOID_RENORM"]
 
@@ -236,6 +236,42 @@ def router_backward(logits, topk_idx, dw_route, score_fn: int = SCORE_SOFTMAX_TO
                                      _ptr(dl), _ptr(status), _stream(stream)),
           "moe_router_backward")
     return dl
+
+
+def _router_dims(T: int, d: int, E: int) -> Dims:
+    # the router calls read T, d and E; f, k and the score function only satisfy the rules
+    return Dims(T, d, 256, E, 1, SCORE_SOFTMAX_TOPK)
+
+
+def router_logits(x, wr, ws=None, out=None, stream=None):
+    """logits [T, E] fp32 = x [T, d] bf16 . wr^T, wr [E, d] bf16 (one row per expert)."""
+    torch = _torch()
+    T, d = x.shape
+    E = wr.shape[0]
+    dims = _router_dims(T, d, E)
+    ws = workspace(dims, OP_ROUTER, x.device) if ws is None else ws
+    out = torch.empty((T, E), dtype=torch.float32, device=x.device) if out is None else out
+    check(load().moe_router_logits(ctypes.byref(dims.c()), _ptr(x.contiguous()),
+                                   _ptr(wr.contiguous()), _ptr(out), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "moe_router_logits")
+    return out
+
+
+def router_grads(dlogits, x, wr, ws=None, stream=None):
+    """(dx_r [T, d] fp32, dwr [E, d] fp32) of logits = x . wr^T from d(loss)/d(logits),
+    the gradient rounded to bf16 as the operand of both tensor-core products."""
+    torch = _torch()
+    T, d = x.shape
+    E = wr.shape[0]
+    dims = _router_dims(T, d, E)
+    ws = workspace(dims, OP_ROUTER, x.device) if ws is None else ws
+    dx = torch.empty((T, d), dtype=torch.float32, device=x.device)
+    dw = torch.empty((E, d), dtype=torch.float32, device=x.device)
+    check(load().moe_router_grads(ctypes.byref(dims.c()), _ptr(dlogits.contiguous()),
+                                  _ptr(x.contiguous()), _ptr(wr.contiguous()), _ptr(dx),
+                                  _ptr(dw), _ptr(ws), ws.numel(), _stream(stream)),
+          "moe_router_grads")
+    return dx, dw
 
 
 @dataclass

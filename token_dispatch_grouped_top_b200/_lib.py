@@ -13,7 +13,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned
           4: "workspace too small", 5: "CUDA runtime error", 6: "device-side wait timed out",
           7: "device-side index out of bounds", 8: "no sm_100 device"}
 
-OP_ROUTE, OP_FORWARD, OP_BACKWARD, OP_FORWARD_BF16 = 0, 1, 2, 3
+OP_ROUTE, OP_FORWARD, OP_BACKWARD, OP_FORWARD_BF16, OP_ROUTER = 0, 1, 2, 3, 4
 
 # internal workspace buffers that moe_workspace_offset locates (moe_ws_buffer)
 WS_BUFFERS = {"mtile": 0, "y": 1, "dout_q": 2, "dout_s": 3, "g": 4, "dgu_q": 5, "dgu_s": 6,
@@ -74,6 +74,9 @@ SIGNATURES = {
     "moe_forward_bf16": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                  c_sz, c_vp]),
     "moe_router_backward": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "moe_router_logits": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "moe_router_grads": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                 c_sz, c_vp]),
     "moe_profile_enable": (c_i32, [c_i32]),
     "moe_debug_withhold_ready": (c_i32, [c_i32]),
     "moe_profile_collect": (c_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_i32),

@@ -307,6 +307,59 @@ inline T* at(void* ws, int64_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// Workspace of the router GEMM calls (MOE_OP_ROUTER): a 256-byte header (status word at 0,
+// three tile counters at 64, the one-group tile prefixes at 128 and valid rows at 160),
+// then the zero-padded bf16 operand copies:
+//   wr_pad [NE, d]     W_r with its rows padded to whole 256-row N tiles (forward B)
+//   dlog   [Tp128, Ep] bf16(G), rows to whole 128-row tiles, K (experts) to 64   (dx A)
+//   dlogT  [Ep128, Tp] bf16(G)^T, rows (experts) to 128, K (tokens) to 64        (dW A)
+//   wrT    [d, Ep]     W_r^T, K (experts) padded to 64                           (dx B)
+//   xT     [d, Tp]     x^T, K (tokens) padded to 64                              (dW B)
+struct RouterWsLayout {
+  int64_t NE, Ep, Tp, Tp128, Ep128;
+  int64_t wr_pad, dlog, dlogT, wrT, xT, total;
+};
+constexpr int64_t kRouterCtr = 64, kRouterPrefix = 128, kRouterValid = 160;
+
+RouterWsLayout router_ws_layout(const moe_dims* D) {
+  auto up = [](int64_t v, int64_t m) { return (v + m - 1) / m * m; };
+  RouterWsLayout L;
+  const int64_t T = std::max<int64_t>(D->T, 1), E = D->E, d = D->d;
+  L.NE = up(E, 256);
+  L.Ep = up(E, 64);
+  L.Tp = up(T, 64);
+  L.Tp128 = up(T, 128);
+  L.Ep128 = up(E, 128);
+  int64_t off = 256;
+  auto take = [&](int64_t bytes) {
+    const int64_t o = off;
+    off += up(bytes, 256);
+    return o;
+  };
+  L.wr_pad = take(L.NE * d * 2);
+  L.dlog = take(L.Tp128 * L.Ep * 2);
+  L.dlogT = take(L.Ep128 * L.Tp * 2);
+  L.wrT = take(d * L.Ep * 2);
+  L.xT = take(d * L.Tp * 2);
+  L.total = off;
+  return L;
+}
+
+moe_status router_checks(const moe_dims* D, const void* const* ptrs, int n, void* ws,
+                         size_t ws_bytes) {
+  MOE_TRY(check_dims(D));
+  if (D->E % 8) return MOE_ERR_UNSUPPORTED_SHAPE;  // row pitches of [*, E] in 16-byte units
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (!ptrs[i]) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(ptrs[i])) return MOE_ERR_MISALIGNED;
+  }
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  if (ws_bytes < static_cast<size_t>(router_ws_layout(D).total))
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return MOE_OK;
+}
+
 moe_status run_route(const moe_dims* D, const float* logits, int32_t* idx, float* w,
                      int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* pad,
                      void* ws, const WsLayout& L, int num_sms, cudaStream_t st) {
@@ -447,7 +500,8 @@ int64_t moe_saved_bytes(const moe_dims* D, int32_t field) {
 }
 
 size_t moe_workspace_bytes(const moe_dims* dims, int32_t op) {
-  if (check_dims(dims) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_FORWARD_BF16) return 0;
+  if (check_dims(dims) != MOE_OK || op < MOE_OP_ROUTE || op > MOE_OP_ROUTER) return 0;
+  if (op == MOE_OP_ROUTER) return static_cast<size_t>(router_ws_layout(dims).total);
   return static_cast<size_t>(ws_layout(dims, op).total);
 }
 
@@ -1218,6 +1272,99 @@ moe_status moe_router_backward(const moe_dims* D, const float* logits, const int
   P.dlogits = dlogits;
   P.status = status;
   return cuda_ok(launch_router_bwd(P, sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_router_logits(const moe_dims* D, const uint16_t* x, const uint16_t* wr,
+                             float* logits, void* ws, size_t ws_bytes, void* stream) {
+  const void* ptrs[] = {wr, x, logits};
+  MOE_TRY(router_checks(D, ptrs, D && D->T > 0 ? 3 : 1, ws, ws_bytes));
+  if (D->T == 0) return MOE_OK;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const RouterWsLayout L = router_ws_layout(D);
+  const int64_t T = D->T, d = D->d, E = D->E;
+  RouterSetupParams S = {};
+  S.n = 1;
+  S.rows[0] = T;
+  S.prefix = at<int32_t>(ws, kRouterPrefix);
+  S.valid = at<int32_t>(ws, kRouterValid);
+  S.ctr = at<uint32_t>(ws, kRouterCtr);
+  MOE_TRY(cuda_ok(launch_router_setup(S, st)));
+  uint16_t* wr_pad = at<uint16_t>(ws, L.wr_pad);
+  MOE_TRY(cuda_ok(launch_pad_copy_bf16(wr, E, d, d, wr_pad, L.NE, d, st)));
+  CUtensorMap ta, tb, tc;
+  MOE_TRY(make_tmap(&ta, x, T, 2 * d, 128));
+  MOE_TRY(make_tmap(&tb, wr_pad, L.NE, 2 * d, 256));
+  MOE_TRY(make_out_tmap(&tc, logits, T, E, false));
+  GemmParams P = {};
+  P.G = 1;
+  P.N = static_cast<int>(L.NE);
+  P.K = static_cast<int>(2 * d);
+  P.mtile_prefix = S.prefix;
+  P.rows_valid = S.valid;
+  P.status = at<int32_t>(ws, 0);
+  P.tile_ctr = S.ctr;
+  P.n_valid = static_cast<int>(E);
+  return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, tc, tc, P, sms, st));
+}
+
+moe_status moe_router_grads(const moe_dims* D, const float* dlogits, const uint16_t* x,
+                            const uint16_t* wr, float* dx_r, float* dwr, void* ws,
+                            size_t ws_bytes, void* stream) {
+  const void* ptrs[] = {wr, dwr, dlogits, x, dx_r};
+  MOE_TRY(router_checks(D, ptrs, D && D->T > 0 ? 5 : 2, ws, ws_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t T = D->T, d = D->d, E = D->E;
+  if (T == 0)  // no tokens: the weight gradient is zero
+    return cuda_ok(cudaMemsetAsync(dwr, 0, static_cast<size_t>(E * d * 4), st));
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  const RouterWsLayout L = router_ws_layout(D);
+  RouterSetupParams S = {};
+  S.n = 2;
+  S.rows[0] = T;  // dx_r = bf16(G) . W_r: token rows
+  S.rows[1] = E;  // dW_r = bf16(G)^T . x: expert rows
+  S.prefix = at<int32_t>(ws, kRouterPrefix);
+  S.valid = at<int32_t>(ws, kRouterValid);
+  S.ctr = at<uint32_t>(ws, kRouterCtr);
+  MOE_TRY(cuda_ok(launch_router_setup(S, st)));
+  uint16_t* dlog = at<uint16_t>(ws, L.dlog);
+  uint16_t* dlogT = at<uint16_t>(ws, L.dlogT);
+  uint16_t* wrT = at<uint16_t>(ws, L.wrT);
+  uint16_t* xT = at<uint16_t>(ws, L.xT);
+  MOE_TRY(cuda_ok(launch_pad_copy_f32_bf16(dlogits, T, E, E, dlog, L.Tp128, L.Ep, st)));
+  MOE_TRY(cuda_ok(launch_transpose_pad_f32_bf16(dlogits, T, E, E, dlogT, L.Ep128, L.Tp, st)));
+  MOE_TRY(cuda_ok(launch_transpose_pad_bf16(wr, E, d, d, wrT, d, L.Ep, st)));
+  MOE_TRY(cuda_ok(launch_transpose_pad_bf16(x, T, d, d, xT, d, L.Tp, st)));
+  {
+    CUtensorMap ta, tb, tc;
+    MOE_TRY(make_tmap(&ta, dlog, L.Tp128, 2 * L.Ep, 128));
+    MOE_TRY(make_tmap(&tb, wrT, d, 2 * L.Ep, 256));
+    MOE_TRY(make_out_tmap(&tc, dx_r, T, d, false));
+    GemmParams P = {};
+    P.G = 1;
+    P.N = static_cast<int>(d);
+    P.K = static_cast<int>(2 * L.Ep);
+    P.mtile_prefix = S.prefix;
+    P.rows_valid = S.valid;
+    P.status = at<int32_t>(ws, 0);
+    P.tile_ctr = S.ctr;
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, tc, tc, P, sms, st)));
+  }
+  CUtensorMap ta, tb, tc;
+  MOE_TRY(make_tmap(&ta, dlogT, L.Ep128, 2 * L.Tp, 128));
+  MOE_TRY(make_tmap(&tb, xT, d, 2 * L.Tp, 256));
+  MOE_TRY(make_out_tmap(&tc, dwr, E, d, false));
+  GemmParams P = {};
+  P.G = 1;
+  P.N = static_cast<int>(d);
+  P.K = static_cast<int>(2 * L.Tp);
+  P.mtile_prefix = S.prefix + 2;
+  P.rows_valid = S.valid + 1;
+  P.status = at<int32_t>(ws, 0);
+  P.tile_ctr = S.ctr + 1;
+  return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, tc, tc, P, sms, st));
 }
 
 moe_status moe_debug_withhold_ready(int32_t minibatch) {

@@ -177,6 +177,7 @@ __device__ __forceinline__ void store_swapped_chunk(const float (&v)[32], int tb
                                                     const CUtensorMap* tm32f,
                                                     const CUtensorMap* tm16, int lane) {
   if (tb >= rows) return;  // warp-uniform
+  if (P.n_valid && xc >= P.n_valid) return;  // columns past the group's width
   uint8_t* buf = stg[stg_buf];
   if (lane == 0) bulk_wait_read<1>();
   __syncwarp();
@@ -612,6 +613,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          if (P.n_valid && x0 + 32 * c >= P.n_valid) break;  // columns past the group's width
           const float* vc = c == 0 ? v0 : c == 1 ? v1 : c == 2 ? v2 : v3;
           uint4 r16[8];
 #pragma unroll

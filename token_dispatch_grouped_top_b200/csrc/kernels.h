@@ -228,6 +228,10 @@ struct GemmParams {
   const int32_t* ready;
   int ready_rows;
   const int32_t* order;
+  // STORE_F32 modes: output columns n >= n_valid are not stored (0: all N).  Lets a group
+  // width that is not a multiple of 256 (the router's E experts) run on whole N tiles of
+  // a zero-padded B.
+  int n_valid;
 };
 // tmC0 / tmC1: output tensor maps of the TMA-store modes (STORE_F32_TMA: fp32 [rows, N],
 // box 32 x 32; WGRAD: bf16 out_a / out_b, box 64 cols x 32 rows); ignored otherwise.
@@ -252,5 +256,32 @@ struct SchedInitParams {
   int32_t* order;
 };
 cudaError_t launch_sched_init(const SchedInitParams& P, cudaStream_t stream);
+
+// Router GEMM (logits = x . W_r^T) and its backward on the grouped GEMM engine (one group):
+// the one-group tile lists and the zero-padded bf16 operand copies.
+struct RouterSetupParams {
+  int n;               // GEMMs (<= 3)
+  int64_t rows[3];     // A rows of each GEMM
+  int32_t* prefix;     // [2n]: {0, ceil(rows/128)} per GEMM
+  int32_t* valid;      // [n]: rows per GEMM
+  uint32_t* ctr;       // [n]: tile counters, zeroed
+};
+cudaError_t launch_router_setup(const RouterSetupParams& P, cudaStream_t stream);
+// dst [dst_rows, dst_cols] bf16 = src[r][c] (r < R, c < C; src row pitch ld elements),
+// zero elsewhere; fp32 sources are rounded to bf16 (nearest, ties to even).
+cudaError_t launch_pad_copy_bf16(const uint16_t* src, int64_t R, int64_t C, int64_t ld,
+                                 uint16_t* dst, int64_t dst_rows, int64_t dst_cols,
+                                 cudaStream_t stream);
+cudaError_t launch_pad_copy_f32_bf16(const float* src, int64_t R, int64_t C, int64_t ld,
+                                     uint16_t* dst, int64_t dst_rows, int64_t dst_cols,
+                                     cudaStream_t stream);
+// dst [dst_rows >= C, dst_cols >= R] bf16 = transpose of src [R, C] (row pitch ld), zero
+// outside; fp32 sources rounded to bf16 as above.
+cudaError_t launch_transpose_pad_bf16(const uint16_t* src, int64_t R, int64_t C, int64_t ld,
+                                      uint16_t* dst, int64_t dst_rows, int64_t dst_cols,
+                                      cudaStream_t stream);
+cudaError_t launch_transpose_pad_f32_bf16(const float* src, int64_t R, int64_t C, int64_t ld,
+                                          uint16_t* dst, int64_t dst_rows, int64_t dst_cols,
+                                          cudaStream_t stream);
 
 }  // namespace moe
