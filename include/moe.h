@@ -299,6 +299,59 @@ moe_status moe_router_grads(const moe_dims* dims, const float* dlogits, const ui
                             const uint16_t* wr, float* dx_r, float* dwr, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* ---- expert parallelism over NVLink (NEXT-2) ---------------------------------------------
+ * Article §01 and §02: G GPUs ("ranks") each own E/G experts (rank r: experts
+ * [r*E/G, (r+1)*E/G)) and route their own tokens; the owner of an expert pulls the rows it
+ * needs from the tokens' GPUs by source and offset into its own memory (pull dispatch),
+ * runs its grouped GEMMs, and pushes each output row back to its token's GPU (push
+ * combine), where the weighted merge runs.  Peers are reached through a device array of
+ * moe_ep_peer entries, one per rank, read and written by these kernels with plain loads
+ * and stores: on a multi-GPU node the entries hold peer mappings of the other GPUs'
+ * buffers (CUDA IPC or symmetric memory, NVLink traffic); with one GPU, buffers of several
+ * ranks on that GPU.  A step has three phases; every rank starts a phase only once every
+ * rank has finished the previous one (a barrier between phases, e.g. a stream-ordered
+ * NCCL all-reduce of one word; with one GPU, stream order):
+ *   1. moe_ep_prepare  (each rank)  route + layout of its tokens, MX quantisation of x
+ *   2. moe_ep_experts  (each rank)  pull its experts' rows from every rank, gate/up +
+ *                                   SwiGLU + MX requant, down, push the rows back
+ *   3. moe_ep_combine  (each rank)  out[t] = sum_j w[t,j] * y[t*k + j]
+ * The result equals moe_forward on each rank's tokens: the same operands and per-row
+ * arithmetic, only the rows' placement in the GEMM tiles differs. */
+typedef struct {
+  int64_t T;               /* tokens of this rank */
+  const int32_t* counts;   /* [E] rows per expert (moe_ep_prepare) */
+  const int32_t* offsets;  /* [E+1] exclusive prefix of counts */
+  const int32_t* perm;     /* [T*k] position -> assignment id a = t*k + j */
+  const uint8_t* xq;       /* [T, d] E4M3 codes of the rank's tokens, along d */
+  const uint8_t* xs;       /* [T, d/32] their E8M0 scale bytes, row-major */
+  uint16_t* y;             /* [T*k, d] expert outputs pushed back (scaled fp16 values) */
+  uint8_t* ys;             /* [T*k, d/32] their scale bytes (common to 32 columns) */
+} moe_ep_peer;
+
+/* Phase 1: dims->T = this rank's tokens, dims->E = all experts.  moe_route_layout's outputs
+ * plus xq [T,d], xs [T,d/32] (row-major scales).  ws: moe_workspace_bytes(ROUTE). */
+moe_status moe_ep_prepare(const moe_dims* dims, const uint16_t* x, const float* logits,
+                          int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                          int32_t* perm, int32_t* inv_perm, uint8_t* xq, uint8_t* xs,
+                          void* ws, size_t ws_bytes, void* stream);
+/* Workspace of moe_ep_experts: dims->T = the tokens of ALL ranks together (the receive
+ * buffer holds the worst case, sum_s T_s * min(k, E/G) rows plus tile padding, so no
+ * count ever goes to the host); 0 on bad arguments (E % world != 0, world outside 1..64). */
+size_t moe_ep_workspace_bytes(const moe_dims* dims, int32_t world);
+/* Phase 2 on rank `rank`: dims as for moe_ep_workspace_bytes; peers [world] device array;
+ * w: this rank's E/G experts, prepared by moe_prepare_weights with dims.E = E/G (expert
+ * r*E/G + i of the layer is its expert i).  Received rows are laid out expert by expert,
+ * source rank by source rank, in each source's segment order.  A count or index found out
+ * of range latches MOE_ERR_DEVICE_BOUNDS (status at the workspace's offset 0) and the rank
+ * then receives nothing. */
+moe_status moe_ep_experts(const moe_dims* dims, int32_t rank, int32_t world,
+                          const moe_ep_peer* peers, const moe_weights* w, void* ws,
+                          size_t ws_bytes, void* stream);
+/* Phase 3: dims->T = this rank's tokens; y, ys: this rank's moe_ep_peer.y / .ys, filled by
+ * every owner's push; out [T,d] bf16.  status: nullable device int32 (bounds latch). */
+moe_status moe_ep_combine(const moe_dims* dims, const float* topk_w, const uint16_t* y,
+                          const uint8_t* ys, uint16_t* out, int32_t* status, void* stream);
+
 /* ---- grouped block-scaled GEMM (the engine of S4/S5, exposed for direct use) ----------
  * For each group g and each row r in [128*mtile_prefix[g], 128*mtile_prefix[g+1]):
  *   D[r, n] = sum_k A[r,k] * B[g*N + n, k],  n < N,  fp32 accumulation, fp32 output

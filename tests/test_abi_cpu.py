@@ -178,3 +178,29 @@ def test_router_gemm_checks(lib):
     assert lib.moe_router_grads(ctypes.byref(D), a, a, a, a, a, ws, n - 1, None) == 4
     big = _dims()
     assert lib.moe_workspace_bytes(ctypes.byref(big), 4) >= 7168 * 8192 * 2
+
+
+def test_expert_parallel_checks(lib):
+    vp = ctypes.c_void_p
+    D = _dims(T=4096, d=512, f=256, E=16, k=4, s=0)
+    n4 = lib.moe_ep_workspace_bytes(ctypes.byref(D), 4)
+    # receive rows: T * min(k, E/G) + E/G * 127, rounded to 128 -> codes, h, y (2 bytes)
+    rows = -(-(4096 * 4 + 4 * 127) // 128) * 128
+    assert n4 >= rows * (512 + 256 + 2 * 512)
+    assert lib.moe_ep_workspace_bytes(ctypes.byref(D), 3) == 0      # E % world != 0
+    assert lib.moe_ep_workspace_bytes(ctypes.byref(D), 0) == 0
+    assert lib.moe_ep_workspace_bytes(ctypes.byref(D), 65) == 0
+    D16 = _dims(T=4096, d=512, f=256, E=16, k=4, s=0)
+    assert lib.moe_ep_workspace_bytes(ctypes.byref(D16), 16) < n4  # min(k, E/G) = 1 row
+    a, ws = vp(1 << 20), vp(1 << 24)
+    from token_dispatch_grouped_top_b200._lib import MoeWeights
+    W = MoeWeights(*([1 << 20] * 8))
+    assert lib.moe_ep_experts(ctypes.byref(D), 0, 3, a, ctypes.byref(W), ws, n4, None) == 2
+    assert lib.moe_ep_experts(ctypes.byref(D), 4, 4, a, ctypes.byref(W), ws, n4, None) == 1
+    assert lib.moe_ep_experts(ctypes.byref(D), 0, 4, None, ctypes.byref(W), ws, n4, None) == 1
+    assert lib.moe_ep_experts(ctypes.byref(D), 0, 4, vp((1 << 20) + 8), ctypes.byref(W), ws,
+                              n4, None) == 3
+    assert lib.moe_ep_experts(ctypes.byref(D), 0, 4, a, ctypes.byref(W), ws, n4 - 1, None) == 4
+    assert lib.moe_ep_combine(ctypes.byref(D), None, a, a, a, None, None) == 1
+    assert lib.moe_ep_prepare(ctypes.byref(D), None, a, a, a, a, a, a, a, a, a, ws, 1 << 30,
+                              None) == 1

@@ -67,3 +67,52 @@ def test_reference_arm_other_ranks_exit_quietly():
                        capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
     assert r.returncode == 0, r.stderr[-1000:]
     assert r.stdout.strip() == ""
+
+
+def _ep_rank_main(rank, world, port, results):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from token_dispatch_grouped_top_b200 import ep
+    from token_dispatch_grouped_top_b200._lib import EP_PEER_FIELDS, MoeEpPeer
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        # this rank's entry: its token count and (stand-in) buffer addresses
+        mine = {"T": 100 + rank}
+        mine.update({n: (rank + 1) * 0x10000 + 0x100 * i for i, n in enumerate(EP_PEER_FIELDS)})
+        # a remote rank's addresses are mapped (here: offset by 1 << 40, as a peer mapping)
+        entries = ep.gather_entries(mine, map_fn=lambda r, e: {
+            n: (v + (1 << 40) if n != "T" else v) for n, v in e.items()})
+        table = ep.peer_table(entries, "cpu")
+        arr = (MoeEpPeer * world).from_buffer_copy(bytes(table.numpy()))
+        rows = [(arr[i].T,) + tuple(getattr(arr[i], n) for n in EP_PEER_FIELDS)
+                for i in range(world)]
+        results.put((rank, rows))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_peer_table_gloo():
+    # the host side of the expert-parallel step: every rank gathers every rank's entry in
+    # rank order, maps the remote ones, and packs the same moe_ep_peer layout
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    results = ctx.Queue()
+    port = _free_port()
+    world = 2
+    procs = [ctx.Process(target=_ep_rank_main, args=(r, world, port, results))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = dict(results.get(timeout=10) for _ in range(world))
+    from token_dispatch_grouped_top_b200._lib import EP_PEER_FIELDS
+    for me, rows in got.items():
+        assert len(rows) == world
+        for r, row in enumerate(rows):
+            assert row[0] == 100 + r
+            shift = 0 if r == me else 1 << 40
+            assert list(row[1:]) == [(r + 1) * 0x10000 + 0x100 * i + shift
+                                     for i in range(len(EP_PEER_FIELDS))]

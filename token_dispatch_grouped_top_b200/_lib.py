@@ -42,6 +42,14 @@ class MoeSaved(ctypes.Structure):
     _fields_ = [(n, c_vp) for n in SAVED_FIELDS]
 
 
+EP_PEER_FIELDS = ["counts", "offsets", "perm", "xq", "xs", "y", "ys"]
+
+
+class MoeEpPeer(ctypes.Structure):
+    """One rank's entry of the expert-parallel peer table (moe_ep_peer)."""
+    _fields_ = [("T", c_i64)] + [(n, c_vp) for n in EP_PEER_FIELDS]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "moe_padded_rows": (c_i64, [ctypes.POINTER(MoeDims)]),
@@ -77,6 +85,11 @@ SIGNATURES = {
     "moe_router_logits": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "moe_router_grads": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                  c_sz, c_vp]),
+    "moe_ep_prepare": (c_i32, [ctypes.POINTER(MoeDims)] + [c_vp] * 11 + [c_sz, c_vp]),
+    "moe_ep_workspace_bytes": (c_sz, [ctypes.POINTER(MoeDims), c_i32]),
+    "moe_ep_experts": (c_i32, [ctypes.POINTER(MoeDims), c_i32, c_i32, c_vp,
+                               ctypes.POINTER(MoeWeights), c_vp, c_sz, c_vp]),
+    "moe_ep_combine": (c_i32, [ctypes.POINTER(MoeDims), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moe_profile_enable": (c_i32, [c_i32]),
     "moe_debug_withhold_ready": (c_i32, [c_i32]),
     "moe_profile_collect": (c_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_i32),

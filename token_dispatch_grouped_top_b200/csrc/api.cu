@@ -345,6 +345,48 @@ RouterWsLayout router_ws_layout(const moe_dims* D) {
   return L;
 }
 
+// Workspace of moe_ep_experts on one rank: a 256-byte header (status at 0, tile counters at
+// 72 and 76), the receive layout, then the receive buffers for the worst case of
+// R_cap = sum_s T_s * min(k, E_loc) rows plus each segment's tile padding:
+//   recv_counts [E_loc], recv_off [E_loc+1], mtile [E_loc+1], src_base [world*E_loc] int32
+//   origin [R_cap] int64, xq [R_cap,d] + UMMA scales, hq [R_cap,f] + UMMA scales,
+//   y [R_cap,d] scaled fp16 + [R_cap,d/32] scale bytes
+struct EpWsLayout {
+  int64_t E_loc, R_cap;
+  int64_t recv_counts, recv_off, mtile, src_base, origin, xq, xs, hq, hs, y, ys, total;
+};
+
+bool ep_ws_layout(const moe_dims* D, int32_t world, EpWsLayout* out) {
+  if (check_dims(D) != MOE_OK || world < 1 || world > 64 || D->E % world) return false;
+  auto up = [](int64_t v, int64_t m) { return (v + m - 1) / m * m; };
+  EpWsLayout L;
+  L.E_loc = D->E / world;
+  const int64_t per_tok = std::min<int64_t>(D->k, L.E_loc);
+  L.R_cap = std::max<int64_t>(up(D->T * per_tok + L.E_loc * 127, 128), 128);
+  if (L.R_cap >= (int64_t(1) << 31)) return false;  // row indices are int32
+  const int64_t d = D->d, f = D->f;
+  int64_t off = 256;
+  auto take = [&](int64_t bytes) {
+    const int64_t o = off;
+    off += up(bytes, 256);
+    return o;
+  };
+  L.recv_counts = take(4 * L.E_loc);
+  L.recv_off = take(4 * (L.E_loc + 1));
+  L.mtile = take(4 * (L.E_loc + 1));
+  L.src_base = take(4 * static_cast<int64_t>(world) * L.E_loc);
+  L.origin = take(8 * L.R_cap);
+  L.xq = take(L.R_cap * d);
+  L.xs = take(L.R_cap * d / 32);
+  L.hq = take(L.R_cap * f);
+  L.hs = take(L.R_cap * f / 32);
+  L.y = take(2 * L.R_cap * d);
+  L.ys = take(L.R_cap * d / 32);
+  L.total = off;
+  *out = L;
+  return true;
+}
+
 moe_status router_checks(const moe_dims* D, const void* const* ptrs, int n, void* ws,
                          size_t ws_bytes) {
   MOE_TRY(check_dims(D));
@@ -876,7 +918,7 @@ moe_status moe_forward_bf16(const moe_dims* D, const uint16_t* wgu_t, const uint
   }
   {
     StageScope sc(MOE_STAGE_COMBINE, st);
-    CombineParams P;
+    CombineParams P = {};
     P.y = y;
     P.ys = ys;
     P.topk_w = w;
@@ -1010,7 +1052,7 @@ moe_status moe_forward(const moe_dims* D, const moe_weights* W, const uint16_t* 
   }
   {
     StageScope sc(MOE_STAGE_COMBINE, st);
-    CombineParams P;
+    CombineParams P = {};
     P.y = y;
     P.ys = ys;
     P.topk_w = w;
@@ -1148,7 +1190,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     }
     {  // push reverse-dispatch: dX[t] = sum_j dXa[row of (t, j)]
       StageScope sc(MOE_STAGE_BWD_DX, st);
-      CombineParams P;
+      CombineParams P = {};
       P.y = dxa;
       P.ys = dxas;
       P.topk_w = nullptr;
@@ -1195,7 +1237,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.dst_q = dq_out;
       P.dst_s = ds_out;
       CUtensorMap tsrc, tdst;
-      MOE_TRY(make_tmap(&tsrc, q, R, C, 128, false));
+      MOE_TRY(make_tmap(&tsrc, q, R, C, 32, false));  // 32-row boxes
       MOE_TRY(make_tmap(&tdst, dq_out, C, R, 128, true));
       return cuda_ok(launch_transpose_quant(tsrc, tdst, P, sms, st));
     };
@@ -1365,6 +1407,132 @@ moe_status moe_router_grads(const moe_dims* D, const float* dlogits, const uint1
   P.status = at<int32_t>(ws, 0);
   P.tile_ctr = S.ctr + 1;
   return cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_BF16, ta, tb, tc, tc, P, sms, st));
+}
+
+moe_status moe_ep_prepare(const moe_dims* D, const uint16_t* x, const float* logits,
+                          int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                          int32_t* perm, int32_t* inv_perm, uint8_t* xq, uint8_t* xs, void* ws,
+                          size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(D));
+  if (D->T > 0 && (!x || !xq || !xs)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(moe_route_layout(D, logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, nullptr,
+                           ws, ws_bytes, stream));
+  if (D->T == 0) return MOE_OK;
+  return mxfp8_quantize(x, D->T, D->d, D->d, xq, xs, 0, stream);
+}
+
+size_t moe_ep_workspace_bytes(const moe_dims* D, int32_t world) {
+  EpWsLayout L;
+  return ep_ws_layout(D, world, &L) ? static_cast<size_t>(L.total) : 0;
+}
+
+moe_status moe_ep_experts(const moe_dims* D, int32_t rank, int32_t world,
+                          const moe_ep_peer* peers, const moe_weights* W, void* ws,
+                          size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(D));
+  if (world < 1 || world > 64 || D->E % world) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rank < 0 || rank >= world || !peers || !W || !ws) return MOE_ERR_INVALID_ARG;
+  if (!W->wgu_q || !W->wgu_s || !W->wd_q || !W->wd_s) return MOE_ERR_INVALID_ARG;
+  {
+    const void* ptrs[] = {peers, W->wgu_q, W->wgu_s, W->wd_q, W->wd_s};
+    for (const void* p : ptrs)
+      if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  if (!aligned256(ws)) return MOE_ERR_MISALIGNED;
+  EpWsLayout L;
+  if (!ep_ws_layout(D, world, &L)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < static_cast<size_t>(L.total)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t d = D->d, f = D->f;
+  const int E_loc = static_cast<int>(L.E_loc);
+  int32_t* status = at<int32_t>(ws, 0);
+  MOE_TRY(cuda_ok(cudaMemsetAsync(at<uint8_t>(ws, 64), 0, 64, st)));  // tile counters
+  EpParams P = {};
+  P.peers = peers;
+  P.world = world;
+  P.rank = rank;
+  P.E_loc = E_loc;
+  P.k = D->k;
+  P.d = static_cast<int>(d);
+  P.R_cap = L.R_cap;
+  P.recv_counts = at<int32_t>(ws, L.recv_counts);
+  P.recv_off = at<int32_t>(ws, L.recv_off);
+  P.mtile = at<int32_t>(ws, L.mtile);
+  P.src_base = at<int32_t>(ws, L.src_base);
+  P.origin = at<int64_t>(ws, L.origin);
+  P.xq = at<uint8_t>(ws, L.xq);
+  P.xs = at<uint8_t>(ws, L.xs);
+  P.y = at<uint16_t>(ws, L.y);
+  P.ys = at<uint8_t>(ws, L.ys);
+  P.status = status;
+  MOE_TRY(cuda_ok(launch_ep_layout(P, st)));
+  MOE_TRY(cuda_ok(launch_ep_pull(P, sms, st)));
+  uint8_t* hq = at<uint8_t>(ws, L.hq);
+  uint8_t* hs = at<uint8_t>(ws, L.hs);
+  {  // gate/up + SwiGLU + MX requantisation of h, over the received rows of E_loc experts
+    CUtensorMap ta, tb;
+    MOE_TRY(make_tmap(&ta, P.xq, L.R_cap, d, 128));
+    MOE_TRY(make_tmap(&tb, W->wgu_q, L.E_loc * 2 * f, d, 256));
+    GemmParams G = {};
+    G.G = E_loc;
+    G.N = static_cast<int>(2 * f);
+    G.K = static_cast<int>(d);
+    G.f = static_cast<int>(f);
+    G.mtile_prefix = P.mtile;
+    G.rows_valid = P.recv_counts;
+    G.sfa = P.xs;
+    G.sfb = W->wgu_s;
+    G.hq = hq;
+    G.hs = hs;
+    G.status = status;
+    G.tile_ctr = at<uint32_t>(ws, kCtrFwdGateUp);
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_SWIGLU, ta, tb, ta, tb, G, sms, st)));
+  }
+  {  // down: y as scaled fp16
+    CUtensorMap ta, tb, ty, ty32;
+    MOE_TRY(make_tmap(&ta, hq, L.R_cap, f, 128));
+    MOE_TRY(make_tmap(&tb, W->wd_q, L.E_loc * d, f, 256));
+    MOE_TRY(make_f16s_tmaps(&ty, &ty32, at<uint16_t>(ws, L.y), L.R_cap, d));
+    GemmParams G = {};
+    G.G = E_loc;
+    G.N = static_cast<int>(d);
+    G.K = static_cast<int>(f);
+    G.mtile_prefix = P.mtile;
+    G.rows_valid = P.recv_counts;
+    G.sfa = hs;
+    G.sfb = W->wd_s;
+    G.status = status;
+    G.tile_ctr = at<uint32_t>(ws, kCtrFwdDown);
+    G.out_scales = at<uint8_t>(ws, L.ys);
+    MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, ty, ty32, G, sms, st)));
+  }
+  return cuda_ok(launch_ep_push(P, sms, st));
+}
+
+moe_status moe_ep_combine(const moe_dims* D, const float* topk_w, const uint16_t* y,
+                          const uint8_t* ys, uint16_t* out, int32_t* status, void* stream) {
+  MOE_TRY(check_dims(D));
+  if (D->T == 0) return MOE_OK;
+  if (!topk_w || !y || !ys || !out) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {topk_w, y, ys, out, status};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  int sms = 0;
+  MOE_TRY(device_sms(&sms));
+  CombineParams P = {};
+  P.y = y;
+  P.ys = ys;
+  P.topk_w = topk_w;
+  P.T = D->T;
+  P.d = D->d;
+  P.E = D->E;
+  P.k = D->k;
+  P.out = out;
+  P.status = status;
+  P.direct_rows = 1;
+  return cuda_ok(launch_combine(P, sms, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_debug_withhold_ready(int32_t minibatch) {

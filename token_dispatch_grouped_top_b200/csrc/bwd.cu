@@ -56,41 +56,75 @@ __device__ __forceinline__ void bulk_store(void* dst, uint32_t smem_src, uint32_
                : "memory");
 }
 
+// Two fp32 products in one packed instruction (each lane rounded to nearest even, as the
+// scalar multiply): (a0, a1) *= (b0, b1).
+__device__ __forceinline__ void mul2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "mul.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
 // One thread: column c of the tile, 32-row block b: decode 32 codes down the column,
 // scale them (rows at or past `lim` are zero), requantise along the rows, write the
 // 32 output bytes into row c of the swizzled output tile and the scale byte into the
-// output chunk.
+// output chunk.  The row multipliers come four at a time (one 16-byte shared load) and
+// both multiplications run on packed pairs.
 template <bool kRagged>
 __device__ __forceinline__ void tq_column_block(const uint8_t* col, const float* mul, int b,
                                                 int lim, uint8_t* orow, int c, uint8_t* sout) {
   float v[32];
 #pragma unroll
-  for (int r = 0; r < 32; r += 2) {  // rows r, r+1: one hardware E4M3x2 -> f16x2 decode
-    const int rr = 32 * b + r;
-    const uint32_t pair = static_cast<uint32_t>(col[rr * 128]) |
-                          (static_cast<uint32_t>(col[(rr + 1) * 128]) << 8);
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
-    v[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu))) * mul[rr];
-    v[r + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16))) * mul[rr + 1];
-    if (kRagged) {
-      if (r >= lim) v[r] = 0.f;
-      if (r + 1 >= lim) v[r + 1] = 0.f;
+  for (int r4 = 0; r4 < 32; r4 += 4) {
+    const float4 m = *reinterpret_cast<const float4*>(mul + 32 * b + r4);
+#pragma unroll
+    for (int h = 0; h < 4; h += 2) {  // rows r, r+1: one hardware E4M3x2 -> f16x2 decode
+      const int r = r4 + h, rr = 32 * b + r;
+      const uint32_t pair = static_cast<uint32_t>(col[rr * 128]) |
+                            (static_cast<uint32_t>(col[(rr + 1) * 128]) << 8);
+      uint32_t h2;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
+      v[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+      v[r + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+      mul2(v[r], v[r + 1], h ? m.z : m.x, h ? m.w : m.y);
+      if (kRagged) {
+        if (r >= lim) v[r] = 0.f;
+        if (r + 1 >= lim) v[r + 1] = 0.f;
+      }
     }
   }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int s = mx_scale_exp(amax);
+  const float inv = mx_inv_scale(s);
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) mul2(v[i], v[i + 1], inv, inv);
   uint32_t qw[8];
-  const uint32_t sb = mx_quant_block32(v, qw);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    qw[i] = cvt_e4m3x2(v[4 * i], v[4 * i + 1]) | (cvt_e4m3x2(v[4 * i + 2], v[4 * i + 3]) << 16);
   *reinterpret_cast<uint4*>(orow + (((2 * b) ^ (c & 7)) << 4)) =
       make_uint4(qw[0], qw[1], qw[2], qw[3]);
   *reinterpret_cast<uint4*>(orow + (((2 * b + 1) ^ (c & 7)) << 4)) =
       make_uint4(qw[4], qw[5], qw[6], qw[7]);
-  sout[(c & 31) * 16 + (c >> 5) * 4 + b] = static_cast<uint8_t>(sb);
+  sout[(c & 31) * 16 + (c >> 5) * 4 + b] = static_cast<uint8_t>(s + 127);
+}
+
+// A 32-row block entirely past the segment's valid rows: zero codes, scale byte 0 (the
+// all-zero block's scale 2^-127), as the requantisation of zeros gives.
+__device__ __forceinline__ void tq_zero_block(int b, uint8_t* orow, int c, uint8_t* sout) {
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  *reinterpret_cast<uint4*>(orow + (((2 * b) ^ (c & 7)) << 4)) = z;
+  *reinterpret_cast<uint4*>(orow + (((2 * b + 1) ^ (c & 7)) << 4)) = z;
+  sout[(c & 31) * 16 + (c >> 5) * 4 + b] = 0;
 }
 
 // Persistent: each CTA walks 128 x 128 tiles (column block fastest) of the rows that
 // belong to some expert segment (rows [0, pad_offsets[E]); the rest of the R-row buffer is
-// never read by the weight-gradient GEMM).  Thread 0 keeps the next tile's codes (TMA,
-// 16 KB) and scale chunk (512 B) in flight while all threads work on the current one;
+// never read by the weight-gradient GEMM).  Thread 0 keeps the next tile's codes (TMA, the
+// 32-row boxes that hold valid rows) and scale chunk (512 B) in flight while all threads
+// work on the current one;
 // the transposed tile and its scale chunk leave through TMA / bulk stores, so global
 // memory sees whole 128-byte lines both ways.  Thread (c, h) handles column c for the
 // 32-row blocks h and h + 2.
@@ -114,11 +148,28 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(
   const int ncb = P.C >> 7;
   const int ntiles = (S.pad[P.E] >> 7) * ncb;
   const int64_t kg_src = P.C >> 7, kg_dst = P.R >> 7;
+  // valid rows of the 128-row block starting at padded row p0: its expert's segment starts
+  // on a 128-row boundary, so the block lies in one segment and holds 1..128 valid rows
+  auto valid_rows = [&](int64_t p0) {
+    int lo = 0, hi = P.E;  // pad[lo] <= p0 < pad[hi]: the expert owning these rows
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (S.pad[mid] <= p0) lo = mid; else hi = mid;
+    }
+    const int64_t rel = p0 - S.pad[lo];
+    int nv = static_cast<int>(P.counts[lo] - rel);
+    nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
+    return make_int2(lo, nv);
+  };
+  // only the 32-row boxes holding valid rows are loaded (the rest of the buffer is padding)
   auto issue = [&](int tile, int buf) {
     const int rb = tile / ncb, cb = tile - rb * ncb;
+    const int nv = valid_rows(static_cast<int64_t>(rb) * 128).y;
+    const int nbox = nv > 0 ? (nv + 31) >> 5 : 1;
     const uint32_t fb = smem_u32(&S.full[buf]);
-    mbar_arrive_expect_tx(fb, kTqTile + 512);
-    tma_load_2d(smem_u32(S.in[buf]), &tm_src, fb, cb * 128, rb * 128);
+    mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nbox) * 4096u + 512u);
+    for (int i = 0; i < nbox; ++i)
+      tma_load_2d(smem_u32(S.in[buf]) + 4096u * i, &tm_src, fb, cb * 128, rb * 128 + 32 * i);
     bulk_load(smem_u32(S.sin[buf]), P.s + ((static_cast<int64_t>(rb) * kg_src + cb) << 9), 512,
               fb);
   };
@@ -134,14 +185,9 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(
     }
     const int rb = tile / ncb, cb = tile - rb * ncb;
     const int64_t p0 = static_cast<int64_t>(rb) * 128;
-    int lo = 0, hi = P.E;  // pad[lo] <= p0 < pad[hi]: the expert owning these rows
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (S.pad[mid] <= p0) lo = mid; else hi = mid;
-    }
+    const int2 ev = valid_rows(p0);
+    const int lo = ev.x, nv = ev.y;
     const int64_t rel = p0 - S.pad[lo];
-    int nv = static_cast<int>(P.counts[lo] - rel);
-    nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
     float w = 0.f;
     if (tid < 128 && tid < nv)
       w = P.src == TSRC_MX_W ? P.topk_w[P.perm[P.offsets[lo] + rel + tid]] : 1.f;
@@ -165,8 +211,10 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(
       const int lim = nv - 32 * b;
       if (lim >= 32)
         tq_column_block<false>(col, mul, b, lim, orow, c, S.sout[buf]);
-      else
+      else if (lim > 0)
         tq_column_block<true>(col, mul, b, lim, orow, c, S.sout[buf]);
+      else
+        tq_zero_block(b, orow, c, S.sout[buf]);  // a block of padding rows only (never loaded)
     }
     fence_proxy_async_smem();
     __syncthreads();

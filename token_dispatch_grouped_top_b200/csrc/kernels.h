@@ -106,6 +106,10 @@ struct CombineParams {
   int d, E, k;
   uint16_t* out;
   int32_t* status;
+  // direct_rows != 0: the row of assignment a = t*k + j is a itself (Y in assignment order,
+  // as the expert-parallel push combine delivers it); topk_idx, inv, offsets and
+  // mtile_prefix are then unused.
+  int direct_rows;
 };
 cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t stream);
 
@@ -256,6 +260,27 @@ struct SchedInitParams {
   int32_t* order;
 };
 cudaError_t launch_sched_init(const SchedInitParams& P, cudaStream_t stream);
+
+// Expert parallelism (NEXT-2): the owner rank's receive layout, pull dispatch and push of
+// the expert outputs, over the peers' buffers (moe_ep_peer table in device memory).
+struct EpParams {
+  const moe_ep_peer* peers;  // [world]
+  int world, rank, E_loc, k, d;
+  int64_t R_cap;             // rows of the receive buffers (multiple of 128)
+  int32_t* recv_counts;      // [E_loc]
+  int32_t* recv_off;         // [E_loc+1] exclusive prefix (unpadded)
+  int32_t* mtile;            // [E_loc+1] 128-row tile prefix of the padded segments
+  int32_t* src_base;         // [world * E_loc]: first row of source s inside expert el
+  int64_t* origin;           // [R_cap]: (source rank << 32) | assignment id, per padded row
+  uint8_t* xq;               // [R_cap, d] received codes
+  uint8_t* xs;               // UMMA scales of [R_cap, d]
+  const uint16_t* y;         // [R_cap, d] expert outputs (scaled fp16) to push
+  const uint8_t* ys;         // [R_cap, d/32]
+  int32_t* status;
+};
+cudaError_t launch_ep_layout(const EpParams& P, cudaStream_t stream);
+cudaError_t launch_ep_pull(const EpParams& P, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_push(const EpParams& P, int num_sms, cudaStream_t stream);
 
 // Router GEMM (logits = x . W_r^T) and its backward on the grouped GEMM engine (one group):
 // the one-group tile lists and the zero-padded bf16 operand copies.

@@ -168,23 +168,29 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineParams 
   __shared__ int64_t s_row[32];
   __shared__ float s_w[32];
   __shared__ int s_bad;
-  for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
-    s_off[i] = P.offsets[i];
-    s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
+  if (!P.direct_rows) {
+    for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
+      s_off[i] = P.offsets[i];
+      s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
+    }
   }
   __syncthreads();
   const int tid = threadIdx.x;
   const int k = P.k;
-  const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
+  const int64_t R = P.direct_rows ? P.T * k : static_cast<int64_t>(s_mt[P.E]) * 128;
   const int64_t nsb = P.d >> 5;  // scale bytes per row
   for (int64_t t = blockIdx.x; t < P.T; t += gridDim.x) {
     if (tid == 0) s_bad = 0;
     __syncthreads();
     if (tid < k) {
       const int64_t a = t * k + tid;
-      const int e = P.topk_idx[a];
       int64_t row = -1;
-      if (e >= 0 && e < P.E) row = static_cast<int64_t>(s_mt[e]) * 128 + (P.inv[a] - s_off[e]);
+      if (P.direct_rows) {
+        row = a;
+      } else {
+        const int e = P.topk_idx[a];
+        if (e >= 0 && e < P.E) row = static_cast<int64_t>(s_mt[e]) * 128 + (P.inv[a] - s_off[e]);
+      }
       if (row < 0 || row >= R) {
         s_bad = 1;
         row = 0;
@@ -263,7 +269,7 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
 // The layer's BF16 variant pulls the bf16 rows of x the same way (no scales).
 constexpr int kGatherChunk = 64;  // rows per CTA step; readiness is published per chunk
 
-__global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
+__global__ void __launch_bounds__(256, 5) gather_rows_kernel(GatherParams P) {
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_mt[kMaxE + 1];
   __shared__ int s_b[kGatherChunk];  // minibatch of each row of the chunk (-1: none)
@@ -284,9 +290,12 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
   // Chunks of consecutive positions in expert order, one per CTA step, so the rows of the
   // first experts (the ones the GEMM starts with) are published first.
   for (int64_t chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
-    for (int r = warp; r < kGatherChunk; r += 8) {
-      const int64_t q = chunk * kGatherChunk + r;
-      int b = -1;
+    // The warp's rows warp, warp + 8, ... of the chunk: lane j < 8 resolves row j's
+    // expert (binary search), token and padded position at once, so the rows' copies
+    // below do not each wait for their own index load first.
+    int64_t my_t = -1, my_p = 0;  // -1: no row (past A, or a failed bounds check)
+    if (lane < kGatherChunk / 8) {
+      const int64_t q = chunk * kGatherChunk + warp + 8 * lane;
       if (q < A) {
         int lo = 0, hi = P.E;  // s_off[lo] <= q < s_off[hi]
         while (hi - lo > 1) {
@@ -297,29 +306,48 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherParams P) {
         const int64_t t = a / P.k;
         const int64_t p = static_cast<int64_t>(s_mt[lo]) * 128 + (q - s_off[lo]);
         if (a < 0 || t >= P.T || p >= R) {
-          if (lane == 0) latch(P.status, MOE_ERR_DEVICE_BOUNDS);
+          latch(P.status, MOE_ERR_DEVICE_BOUNDS);
         } else {
-          const int64_t rb = P.row_bytes;
-          const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * rb);
-          uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * rb);
-          const int n16 = static_cast<int>(rb >> 4);
-          // 8 loads per lane in flight (4 KB per warp) before the stores
-          for (int i0 = lane; i0 < n16; i0 += 32 * 8) {
-            uint4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              v[u] = i0 + 32 * u < n16 ? ld_nc_v4(src + i0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              if (i0 + 32 * u < n16) __stcs(dst + i0 + 32 * u, v[u]);
-          }
-          if (P.s_tok) {
-            const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
-            for (int g = lane; g < kg; g += 32)
-              *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
-          }
-          if (P.ready) b = static_cast<int>(p / P.ready_rows);
+          my_t = t;
+          my_p = p;
         }
+      }
+    }
+#pragma unroll 1
+    for (int j = 0; j < kGatherChunk / 8; ++j) {
+      const int r = warp + 8 * j;
+      const int64_t t = __shfl_sync(kFull, my_t, j), p = __shfl_sync(kFull, my_p, j);
+      int b = -1;
+      if (t >= 0) {
+        const int64_t rb = P.row_bytes;
+        const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * rb);
+        uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * rb);
+        const int n16 = static_cast<int>(rb >> 4);
+        // the row's scale words are loaded with its first batch of codes
+        const uint32_t* ssrc =
+            P.s_tok ? reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5)) : nullptr;
+        const uint32_t sw0 = ssrc && lane < kg ? ssrc[lane] : 0u;
+        const uint32_t sw1 = ssrc && lane + 32 < kg ? ssrc[lane + 32] : 0u;
+        // 8 loads per lane in flight (4 KB per warp) before the stores
+        for (int i0 = lane; i0 < n16; i0 += 32 * 8) {
+          uint4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            v[u] = i0 + 32 * u < n16 ? ld_nc_v4(src + i0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (i0 + 32 * u < n16) __stcs(dst + i0 + 32 * u, v[u]);
+        }
+        if (ssrc) {
+          if (lane < kg)
+            *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * lane, kg)) = sw0;
+          if (lane + 32 < kg)
+            *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * (lane + 32), kg)) =
+                sw1;
+          for (int g = lane + 64; g < kg; g += 32)  // rows wider than 8192 columns
+            *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
+        }
+        if (P.ready) b = static_cast<int>(p / P.ready_rows);
       }
       if (P.ready && lane == 0) s_b[r] = b;
     }
