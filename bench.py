@@ -657,6 +657,102 @@ def run_ours(args, case):
         print(json.dumps(line), flush=True)
 
 
+def run_ep(args, case):
+    """Expert-parallel forward (moe_ep_prepare / moe_ep_experts / moe_ep_combine) with G
+    ranks run on this one GPU in phase order, each rank's buffers separate and reached
+    through the peer table: one JSON line (not the default line) with the step time, the
+    per-stage times of the pull dispatch and the push combine and their bytes, and the
+    single-GPU forward over the same tokens on the same GPU.  One GPU does every rank's
+    work, so the line measures the expert-parallel kernels and the per-rank overhead, not
+    multi-GPU scaling."""
+    import numpy as np
+    import torch
+
+    import synth
+    import token_dispatch_grouped_top_b200 as moe
+    from token_dispatch_grouped_top_b200 import ep
+
+    G = args.ep_ranks
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    E_loc, k = case.E // G, case.k
+    wg, wu, wd = synth.expert_weights_torch(case, dev)
+    dl = moe.Dims(case.T, case.d, case.f, E_loc, min(k, E_loc), case.score_fn)
+    wl = [moe.prepare_weights(wg[r * E_loc:(r + 1) * E_loc].contiguous(),
+                              wu[r * E_loc:(r + 1) * E_loc].contiguous(),
+                              wd[r * E_loc:(r + 1) * E_loc].contiguous(), dl) for r in range(G)]
+    dims = moe.Dims(case.T, case.d, case.f, case.E, k, case.score_fn)
+    full = moe.prepare_weights(wg, wu, wd, dims)
+    del wg, wu, wd
+    torch.cuda.empty_cache()
+    x = torch.from_numpy(synth.make_x(case).view(np.int16)).view(torch.bfloat16).to(dev)
+    lg = torch.from_numpy(synth.make_logits(case)).to(dev)
+    cuts = np.linspace(0, case.T, G + 1).astype(int)
+    xs = [x[cuts[r]:cuts[r + 1]].contiguous() for r in range(G)]
+    lgs = [lg[cuts[r]:cuts[r + 1]].contiguous() for r in range(G)]
+    dims_r = [moe.Dims(int(cuts[r + 1] - cuts[r]), case.d, case.f, case.E, k, case.score_fn)
+              for r in range(G)]
+    dims_all = moe.Dims(case.T, case.d, case.f, case.E, k, case.score_fn)
+    rws = [moe.workspace(dims_r[r], moe.OP_ROUTE, dev) for r in range(G)]
+    states = [ep.prepare(dims_r[r], xs[r], lgs[r], ws=rws[r]) for r in range(G)]
+    table = ep.peer_table([s.entry() for s in states], dev)
+    wss = [ep.experts(dims_all, r, G, table, wl[r]) for r in range(G)]
+    outs = [ep.combine(dims_r[r], states[r]) for r in range(G)]
+
+    def step():
+        for r in range(G):
+            ep.prepare(dims_r[r], xs[r], lgs[r], ws=rws[r], state=states[r])
+        for r in range(G):
+            ep.experts(dims_all, r, G, table, wl[r], ws=wss[r])
+        for r in range(G):
+            ep.combine(dims_r[r], states[r], out=outs[r])
+
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    for _ in range(args.warmup):
+        step()
+    ms = timed(step, args.steps)
+    ws1 = moe.workspace(dims, moe.OP_FORWARD, dev)
+    out1 = torch.empty((case.T, case.d), dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        moe.forward(x, lg, full, ws=ws1, out=out1)
+    ms1 = timed(lambda: moe.forward(x, lg, full, ws=ws1, out=out1), args.steps)
+    moe.profile_enable(True)
+    moe.profile_collect()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    stages = moe.profile_collect()
+    moe.profile_enable(False)
+    status = max(moe.device_status(w) for w in wss)
+    A = case.T * k
+    pull_b = A * (case.d + case.d // 32) * 2          # token rows read from the sources, written
+    push_b = A * (2 * case.d + case.d // 32) * 2      # output rows read, written to the sources
+    st = {}
+    for name, (tot, n) in stages.items():
+        per = tot / max(n, 1)
+        st[name] = {"ms_per_launch": per, "launches": n}
+        if name in ("ep_pull", "ep_push"):
+            bts = (pull_b if name == "ep_pull" else push_b) / G   # per rank launch
+            st[name]["alg_bytes"] = bts
+            st[name]["gbs"] = bts / (per * 1e-3) / 1e9
+    line = {"metric": "expert-parallel forward, ranks emulated on one GPU", "ranks": G,
+            "value": case.T * args.steps / (ms * args.steps * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "single_gpu_forward_ms": ms1, "steps": args.steps,
+            "warmup": args.warmup, "stages": st, "device_status": status,
+            "config": {"workload": case.name, "T": case.T, "d": case.d, "f": case.f,
+                       "E": case.E, "k": k, "E_per_rank": E_loc}}
+    print(json.dumps(line), flush=True)
+
+
 def sweep(args):
     """One JSON line per synthetic configuration and pass (forward, forward+backward).
     Not the default line: a table for the design notes."""
@@ -683,12 +779,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true", help="every synthetic config, one line each")
+    ap.add_argument("--ep-ranks", type=int, default=0,
+                    help="expert-parallel forward with this many ranks emulated on one GPU")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     import synth
     case = synth.CONFIGS[args.config]
     if args.sweep:
         sweep(args)
+        return
+    if args.ep_ranks:
+        run_ep(args, case)
         return
     if args.impl == "reference":
         run_reference(args, case)

@@ -1,5 +1,9 @@
 /*
- * moe.h -- C ABI of the B200 (sm_100a) Mixture-of-Experts layer hot path.
+
+ * The token-direction codes (XT_Q, HT_Q, GT_Q, YT_Q, a [C,R] matrix) are stored in
+ * 128 x 128 tiles: the tile of features [128 fb, 128 fb + 128) and tokens [128 tb,
+ * 128 tb + 128) is 16384 contiguous bytes at offset (tb * C/128 + fb) * 16384, row-major
+ * inside (128 feature rows of 128 token bytes); their scales are the UMMA layout of [C,R]. * moe.h -- C ABI of the B200 (sm_100a) Mixture-of-Experts layer hot path.
  *
  * The method is the one described in "Cursor's MoK achieves 2.37x performance boost on
  * NVIDIA GB300 NVL72" (kucoin news flash article): a single MoE layer that routes tokens
@@ -401,10 +405,13 @@ typedef enum {
   MOE_STAGE_BWD_TRANSPOSE = 9,
   MOE_STAGE_BWD_WGRAD = 10,
   MOE_STAGE_BWD_SWIGLU = 11, /* S8: d(router weights) + SwiGLU backward + MX of dg|du   */
-  MOE_NUM_STAGES = 12
+  MOE_STAGE_EP_PULL = 12,   /* expert parallelism: receive layout + pull dispatch         */
+  MOE_STAGE_EP_PUSH = 13,   /* expert parallelism: push of the expert outputs             */
+  MOE_NUM_STAGES = 14
 } moe_stage;
 
-/* When enabled, every stage launched by moe_forward / moe_backward is bracketed by CUDA
+/* When enabled, every stage launched by moe_forward / moe_backward / moe_ep_experts /
+ * moe_ep_combine is bracketed by CUDA
  * events on the launch stream (host-side bookkeeping only; not for use during graph
  * capture).  The events serialise the stages (the gate/up GEMM then starts after the dispatch
  * has finished instead of as its CTAs retire).  moe_profile_collect synchronises on the recorded events, writes the summed

@@ -113,8 +113,14 @@ def test_forward_full_experts(moe, name):
 # ---------------------------------------------------------------------------------------
 def _transposed(codes_buf, canon_scales, C, R, col0, n32):
     """Columns [col0, col0 + n32) of a [C, R] token-direction operand as [n32, C] codes and
-    [n32/32, C] scale bytes (``canon_scales``: the [C, R/32] scales of the whole matrix)."""
-    codes = to_np(codes_buf.view(C, R)[:, col0:col0 + n32]).T
+    [n32/32, C] scale bytes (``canon_scales``: the [C, R/32] scales of the whole matrix).
+    The codes are stored in 128 x 128 tiles (token block major, then feature block; a
+    tile's rows are features of 128 token bytes); col0 starts a 128-token block."""
+    assert col0 % 128 == 0
+    tb0, ntb = col0 // 128, -(-n32 // 128)
+    tiles = codes_buf.view(R // 128, C // 128, 128, 128)[tb0:tb0 + ntb]
+    cr = tiles.permute(1, 2, 0, 3).reshape(C, ntb * 128)     # [features, tokens of the blocks]
+    codes = to_np(cr[:, :n32]).T
     sc = canon_scales[:, col0 // 32:(col0 + n32) // 32].T
     return np.ascontiguousarray(codes), np.ascontiguousarray(sc)
 

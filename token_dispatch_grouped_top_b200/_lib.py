@@ -21,7 +21,8 @@ WS_BUFFERS = {"mtile": 0, "y": 1, "dout_q": 2, "dout_s": 3, "g": 4, "dgu_q": 5, 
               "yt_q": 14, "yt_s": 15, "counts": 16, "y_s": 17, "dxa_s": 19}
 
 STAGES = ["route", "permute", "gateup", "down", "combine", "bwd_dout", "bwd_dgrad_down",
-          "bwd_dgrad_gateup", "bwd_dx", "bwd_transpose", "bwd_wgrad", "bwd_swiglu"]
+          "bwd_dgrad_gateup", "bwd_dx", "bwd_transpose", "bwd_wgrad", "bwd_swiglu", "ep_pull",
+          "ep_push"]
 
 
 class MoeDims(ctypes.Structure):

@@ -1238,7 +1238,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.dst_s = ds_out;
       CUtensorMap tsrc, tdst;
       MOE_TRY(make_tmap(&tsrc, q, R, C, 32, false));  // 32-row boxes
-      MOE_TRY(make_tmap(&tdst, dq_out, C, R, 128, true));
+      MOE_TRY(make_tmap(&tdst, dq_out, R * C / 128, 128, 128, true));  // 128 x 128 tiles
       return cuda_ok(launch_transpose_quant(tsrc, tdst, P, sms, st));
     };
     MOE_TRY(run(TSRC_MX, S->xq, S->xs, d, xt_q, xt_s));         // x^ -> X~^T [d, R]
@@ -1254,8 +1254,8 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     if (D->T == 0) MOE_TRY(cuda_ok(cudaMemsetAsync(S->pad_offsets, 0, 4 * (E + 1), st)));
     const int64_t Kt = std::max<int64_t>(R, 128);
     CUtensorMap ta, tb;
-    MOE_TRY(make_tmap(&ta, xt_q, d, Kt, 128));
-    MOE_TRY(make_tmap(&tb, gt_q, 2 * f, Kt, 256));
+    MOE_TRY(make_tmap(&ta, xt_q, Kt * d / 128, 128, 128));  // tiled (see the requantisation)
+    MOE_TRY(make_tmap(&tb, gt_q, Kt * 2 * f / 128, 128, 256));
     GemmParams P = {};
     P.G = E;
     P.M = d;
@@ -1275,8 +1275,8 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
     MOE_TRY(make_out_tmap(&tg, dWg, static_cast<int64_t>(E) * d, f, true));
     MOE_TRY(make_out_tmap(&tu, dWu, static_cast<int64_t>(E) * d, f, true));
     MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_WGRAD_BF16, ta, tb, tg, tu, P, sms, st)));
-    MOE_TRY(make_tmap(&ta, ht_q, f, Kt, 128));
-    MOE_TRY(make_tmap(&tb, yt_q, d, Kt, 256));
+    MOE_TRY(make_tmap(&ta, ht_q, Kt * f / 128, 128, 128));
+    MOE_TRY(make_tmap(&tb, yt_q, Kt * d / 128, 128, 256));
     P.M = f;
     P.N = d;
     P.sfa = ht_s;
@@ -1467,11 +1467,15 @@ moe_status moe_ep_experts(const moe_dims* D, int32_t rank, int32_t world,
   P.y = at<uint16_t>(ws, L.y);
   P.ys = at<uint8_t>(ws, L.ys);
   P.status = status;
-  MOE_TRY(cuda_ok(launch_ep_layout(P, st)));
-  MOE_TRY(cuda_ok(launch_ep_pull(P, sms, st)));
+  {
+    StageScope sc(MOE_STAGE_EP_PULL, st);
+    MOE_TRY(cuda_ok(launch_ep_layout(P, st)));
+    MOE_TRY(cuda_ok(launch_ep_pull(P, sms, st)));
+  }
   uint8_t* hq = at<uint8_t>(ws, L.hq);
   uint8_t* hs = at<uint8_t>(ws, L.hs);
   {  // gate/up + SwiGLU + MX requantisation of h, over the received rows of E_loc experts
+    StageScope sc(MOE_STAGE_GATEUP, st);
     CUtensorMap ta, tb;
     MOE_TRY(make_tmap(&ta, P.xq, L.R_cap, d, 128));
     MOE_TRY(make_tmap(&tb, W->wgu_q, L.E_loc * 2 * f, d, 256));
@@ -1491,6 +1495,7 @@ moe_status moe_ep_experts(const moe_dims* D, int32_t rank, int32_t world,
     MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_GATEUP_SWIGLU, ta, tb, ta, tb, G, sms, st)));
   }
   {  // down: y as scaled fp16
+    StageScope sc(MOE_STAGE_DOWN, st);
     CUtensorMap ta, tb, ty, ty32;
     MOE_TRY(make_tmap(&ta, hq, L.R_cap, f, 128));
     MOE_TRY(make_tmap(&tb, W->wd_q, L.E_loc * d, f, 256));
@@ -1508,6 +1513,7 @@ moe_status moe_ep_experts(const moe_dims* D, int32_t rank, int32_t world,
     G.out_scales = at<uint8_t>(ws, L.ys);
     MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, ty, ty32, G, sms, st)));
   }
+  StageScope sc(MOE_STAGE_EP_PUSH, st);
   return cuda_ok(launch_ep_push(P, sms, st));
 }
 
@@ -1532,6 +1538,7 @@ moe_status moe_ep_combine(const moe_dims* D, const float* topk_w, const uint16_t
   P.out = out;
   P.status = status;
   P.direct_rows = 1;
+  StageScope sc(MOE_STAGE_COMBINE, static_cast<cudaStream_t>(stream));
   return cuda_ok(launch_combine(P, sms, static_cast<cudaStream_t>(stream)));
 }
 

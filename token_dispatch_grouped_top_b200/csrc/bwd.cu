@@ -9,7 +9,11 @@
 // already holds (x^, h^, dout^ scaled by the row's combine weight, [dg|du]^):
 // blocks of 32 consecutive tokens inside one expert's segment (segments start on 128-row
 // boundaries, so a block never straddles two experts; rows past the segment's count are
-// zeros).  The result is stored transposed ([C, R], K-major for the GEMM).
+// zeros).  The result is stored transposed, K-major for the GEMM, in 128 x 128 tiles: the
+// tile of features [128 fb, +128) and tokens [128 tb, +128) is one contiguous 16 KB block
+// (row = feature, 128 token bytes per row) at block index tb * (C / 128) + fb, so each
+// tile leaves as one sequential 16 KB write and the GEMM loads its 128- and 256-row boxes
+// (one or two adjacent feature blocks of a token block) from contiguous memory.
 //
 // TMA-staged 128 x 128 tiles: see transpose_quant_kernel.  C % 128 == 0 (d, f, 2f all are).
 #include <cuda_fp16.h>
@@ -125,8 +129,8 @@ __device__ __forceinline__ void tq_zero_block(int b, uint8_t* orow, int c, uint8
 // never read by the weight-gradient GEMM).  Thread 0 keeps the next tile's codes (TMA, the
 // 32-row boxes that hold valid rows) and scale chunk (512 B) in flight while all threads
 // work on the current one;
-// the transposed tile and its scale chunk leave through TMA / bulk stores, so global
-// memory sees whole 128-byte lines both ways.  Thread (c, h) handles column c for the
+// the transposed tile (16 contiguous KB) and its scale chunk leave through TMA / bulk
+// stores.  Thread (c, h) handles column c for the
 // 32-row blocks h and h + 2.
 __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(
     const __grid_constant__ CUtensorMap tm_src, const __grid_constant__ CUtensorMap tm_dst,
@@ -219,7 +223,7 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-      tma_store_2d(&tm_dst, smem_u32(S.out[buf]), static_cast<int32_t>(p0), cb * 128);
+      tma_store_2d(&tm_dst, smem_u32(S.out[buf]), 0, (rb * ncb + cb) * 128);  // one 16 KB tile
       bulk_store(P.dst_s + ((static_cast<int64_t>(cb) * kg_dst + rb) << 9), smem_u32(S.sout[buf]),
                  512);
       bulk_commit();

@@ -296,8 +296,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t fb = smem_u32(&S.full[stage]);
           mbar_arrive_expect_tx(fb, ModeCfg<MODE>::kTx);
-          tma_load_2d(smem_u32(S.a[stage]), &tmA, fb, kb * BK, static_cast<int32_t>(ti.a_row0));
-          tma_load_2d(smem_u32(S.b[stage]), &tmB, fb, kb * BK, static_cast<int32_t>(ti.b_row0));
+          if (MODE == GEMM_WGRAD_BF16) {
+            // token-direction operands in 128 x 128 tiles: feature block fb of token block kb
+            // is the 128 rows from (kb * features / 128 + fb) * 128; the B box of 256 rows
+            // spans feature blocks 2j and 2j + 1 of the same token block
+            tma_load_2d(smem_u32(S.a[stage]), &tmA, fb, 0,
+                        static_cast<int32_t>((kb * (P.M >> 7) + (ti.a_row0 >> 7)) * 128));
+            tma_load_2d(smem_u32(S.b[stage]), &tmB, fb, 0,
+                        static_cast<int32_t>((kb * (P.N >> 7) + (ti.b_row0 >> 7)) * 128));
+          } else {
+            tma_load_2d(smem_u32(S.a[stage]), &tmA, fb, kb * BK, static_cast<int32_t>(ti.a_row0));
+            tma_load_2d(smem_u32(S.b[stage]), &tmB, fb, kb * BK, static_cast<int32_t>(ti.b_row0));
+          }
           if (!ModeCfg<MODE>::kBf16) {
             bulk_load(smem_u32(S.sfa[stage]), P.sfa + ((rbA * kgroups + kb) << 9), 512, fb);
             bulk_load(smem_u32(S.sfb[stage]), P.sfb + ((rbB * kgroups + kb) << 9), 512, fb);

@@ -50,14 +50,9 @@ class RankState:
         return e
 
 
-def prepare(dims, x, logits, ws=None, stream=None) -> RankState:
-    """Phase 1 on this rank: route + layout of its T tokens and their MX quantisation;
-    allocates the [T*k, d] receive buffers the owners push into."""
-    from . import Dims, workspace
+def _alloc_state(dims, dev) -> RankState:
     torch = _torch()
-    dev = x.device
     T, d, k, E = dims.T, dims.d, dims.k, dims.E
-    ws = workspace(dims, OP_ROUTE, dev) if ws is None else ws
     i32 = dict(dtype=torch.int32, device=dev)
     st = RankState(T)
     b = st.bufs
@@ -71,6 +66,18 @@ def prepare(dims, x, logits, ws=None, stream=None) -> RankState:
     b["xs"] = torch.empty((max(T, 1), d // 32), dtype=torch.uint8, device=dev)
     b["y"] = torch.empty((max(T * k, 1), d), dtype=torch.float16, device=dev)
     b["ys"] = torch.empty((max(T * k, 1), d // 32), dtype=torch.uint8, device=dev)
+    return st
+
+
+def prepare(dims, x, logits, ws=None, state=None, stream=None) -> RankState:
+    """Phase 1 on this rank: route + layout of its T tokens and their MX quantisation.
+    Allocates the rank's buffers (among them the [T*k, d] receive buffers the owners push
+    into), or refills those of `state`."""
+    from . import workspace
+    dev = x.device
+    ws = workspace(dims, OP_ROUTE, dev) if ws is None else ws
+    st = _alloc_state(dims, dev) if state is None else state
+    b = st.bufs
     check(load().moe_ep_prepare(ctypes.byref(dims.c()), _ptr(x), _ptr(logits),
                                 _ptr(b["topk_idx"]), _ptr(b["topk_w"]), _ptr(b["counts"]),
                                 _ptr(b["offsets"]), _ptr(b["perm"]), _ptr(b["inv_perm"]),
