@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineParams 
       for (int c = 0; c < kCombineChunks; ++c)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[c][i] = 0.f;
+#pragma unroll 2  // two rows' loads in flight
       for (int j = 0; j < k; ++j) {  // j ascending: the sum order is fixed
         const int64_t row = s_row[j];
         const float w = s_w[j];
