@@ -160,7 +160,7 @@ cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream) {
 // (thread i takes 16-byte chunks i, i + 256, ...), so every DRAM access is a long run of a
 // single row rather than k short pieces of different rows.
 constexpr int kCombineThreads = 256;
-constexpr int kCombineChunks = 4;  // 16-byte chunks per thread per column block
+constexpr int kCombineChunks = 2;  // 16-byte chunks per thread per column block (64 registers: 4 CTAs per SM)
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineParams P) {
   __shared__ int s_off[kMaxE + 1];
