@@ -37,6 +37,14 @@ CONFIG_NAME = "dsv3"
 # boxes into a 4 GiB [rows, 4096-byte] matrix (the weight-gradient epilogue's pattern; plain
 # coalesced 16-byte stores reach ~6300 GB/s): the ceiling of an output-dominated kernel.
 WRITE_ONLY_GBS = 5959.0
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels the roofline
+# reports, from ncu captures of the mid configuration (profiles/wgrad_mid_full.md,
+# profiles/grouped_gemm_mid_full.md), as a ratio to the same launches' algorithmic bytes;
+# a full-size launch's traffic is that ratio times its own algorithmic bytes (its operand
+# and output bytes both grow with the shape).  Lines still dirty in L2 when a launch ends
+# are not counted by the capture.
+WGRAD_TRAFFIC_RATIO = (752.110592 + 153.921536 + 349.786368 + 107.617280) / 1428.553728
+GATEUP_TRAFFIC_RATIO = (413.373440 + 168.876032) / 657.063936
 
 
 def _peaks():
@@ -586,7 +594,9 @@ def run_ours(args, case):
     g = stage_info.get("gateup", {"ms_per_launch": float("nan"), "tflops": float("nan")})
     roof_gateup = {"bound": "tensor", "kernel": "grouped_gemm_kernel<GATEUP_SWIGLU>",
                    "achieved": g["tflops"], "peak": mx_peak, "unit": "TFLOP/s",
-                   "frac": g["tflops"] / mx_peak, "traffic": None,
+                   "frac": g["tflops"] / mx_peak,
+                   "traffic": GATEUP_TRAFFIC_RATIO * g["alg_bytes"] if "alg_bytes" in g else None,
+                   "traffic_note": "DRAM bytes per launch, scaled from the mid-shape ncu capture",
                    "peak_note": f"2 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
                                 f"MXFP8:bf16 nominal ratio 2"}
     roofline = roof_gateup
@@ -596,7 +606,10 @@ def run_ours(args, case):
         w = stage_info["bwd_wgrad"]
         roofline = {"bound": "hbm", "kernel": "grouped_gemm_kernel<WGRAD_BF16> (2 launches)",
                     "achieved": w["gbs"], "peak": peaks["hbm"], "unit": "GB/s",
-                    "frac": w["gbs"] / peaks["hbm"], "traffic": None,
+                    "frac": w["gbs"] / peaks["hbm"],
+                    "traffic": WGRAD_TRAFFIC_RATIO * w["alg_bytes"],
+                    "traffic_note": "DRAM bytes of the launch pair, scaled from the mid-shape "
+                                    "ncu capture (ratio to algorithmic bytes 0.954)",
                     "peak_note": f"{peaks['src']} copy bandwidth (read+write); pure-write "
                                  f"streams on this pool measured {WRITE_ONLY_GBS:.0f} GB/s",
                     "frac_of_write_only": w["gbs"] / WRITE_ONLY_GBS}
