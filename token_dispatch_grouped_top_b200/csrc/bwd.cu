@@ -54,11 +54,6 @@ struct TqSmem {
 };
 constexpr size_t kTqSmemBytes = sizeof(TqSmem) + 1024;
 
-__device__ __forceinline__ void bulk_store(void* dst, uint32_t smem_src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_src), "r"(bytes)
-               : "memory");
-}
 
 // Two fp32 products in one packed instruction (each lane rounded to nearest even, as the
 // scalar multiply): (a0, a1) *= (b0, b1).

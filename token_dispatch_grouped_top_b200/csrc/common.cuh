@@ -165,6 +165,14 @@ __device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void* src, ui
       : "memory");
 }
 
+// Untiled bulk copy shared -> global (bulk-group completion; 16-byte aligned, size a
+// multiple of 16).
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_src), "r"(bytes)
+               : "memory");
+}
+
 // TMA tensor store shared -> global (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t smem_src, int32_t x,
                                              int32_t y) {

@@ -263,49 +263,73 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
   return cudaGetLastError();
 }
 
-// S3, second half: the pull gather.  Each expert row (one warp) fetches the MX codes and
-// scales of its token by index from the per-token quantised copy (x quantised once per
-// token, small enough to stay in L2) and writes them to its padded position: codes with
-// 16-byte copies, scales re-laid into the UMMA layout one 4-byte K-group word at a time.
+// S3, second half: the pull gather.  Each expert row fetches the MX codes and scales of its
+// token by index from the per-token quantised copy (x quantised once per token, small
+// enough to stay in L2) and writes them to its padded position: the codes with bulk copies
+// through shared memory (the copy engine moves the bytes; one thread per warp issues
+// them), the scales re-laid into the UMMA layout one 4-byte K-group word at a time.
 // The layer's BF16 variant pulls the bf16 rows of x the same way (no scales).
-constexpr int kGatherChunk = 64;  // rows per CTA step; readiness is published per chunk
+constexpr int kGatherChunk = 64;    // rows per CTA step; readiness is published per chunk
+constexpr int kGatherWarps = 8;
+constexpr int kGatherPiece = 4096;  // bytes per bulk copy; a row is one or more pieces
 
-__global__ void __launch_bounds__(256, 5) gather_rows_kernel(GatherParams P) {
-  __shared__ int s_off[kMaxE + 1];
-  __shared__ int s_mt[kMaxE + 1];
-  __shared__ int s_b[kGatherChunk];  // minibatch of each row of the chunk (-1: none)
+// Per warp two piece buffers: the bulk load of the next piece runs while the current one is
+// stored (a 7 KB MX row is two pieces, a bf16 row of the BF16 variant four).
+struct GatherSmem {
+  uint8_t buf[kGatherWarps][2][kGatherPiece];
+  uint64_t bar[kGatherWarps][2];
+  int64_t rt[kGatherWarps][kGatherChunk / kGatherWarps];  // each row's token (-1: none)
+  int64_t rp[kGatherWarps][kGatherChunk / kGatherWarps];  // and padded position
+  int s_off[kMaxE + 1];
+  int s_mt[kMaxE + 1];
+  int s_b[kGatherChunk];  // minibatch of each row of the chunk (-1: none)
+  int abort_flag;
+};
+constexpr size_t kGatherSmemBytes = sizeof(GatherSmem) + 128;
+
+__global__ void __launch_bounds__(kGatherWarps * 32, 3) gather_rows_kernel(GatherParams P) {
+  extern __shared__ uint8_t g_raw[];
+  GatherSmem& S = *reinterpret_cast<GatherSmem*>(
+      g_raw + ((128u - (smem_u32(g_raw) & 127u)) & 127u));
   // the consumer GEMM (launched as a programmatic dependent) may start now: it waits for
   // each minibatch of rows through the readiness counters, not for this grid to finish
   launch_dependents();
   for (int i = threadIdx.x; i <= P.E; i += blockDim.x) {
-    s_off[i] = P.offsets[i];
-    s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
+    S.s_off[i] = P.offsets[i];
+    S.s_mt[i] = P.mtile_prefix[i] >> P.prefix_shift;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) S.abort_flag = 0;
+  if (lane == 0) {
+    mbar_init(smem_u32(&S.bar[warp][0]), 1);
+    mbar_init(smem_u32(&S.bar[warp][1]), 1);
+    fence_barrier_init();
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t A = P.T * P.k;
-  const int64_t R = static_cast<int64_t>(s_mt[P.E]) * 128;
+  const int64_t R = static_cast<int64_t>(S.s_mt[P.E]) * 128;
   const int d = P.d;
   const int64_t kg = d >> 7;
+  const int64_t rb = P.row_bytes;
   const int64_t nchunks = (A + kGatherChunk - 1) / kGatherChunk;
+  uint32_t ph = 0;  // lane 0: parity of each buffer's next load
   // Chunks of consecutive positions in expert order, one per CTA step, so the rows of the
   // first experts (the ones the GEMM starts with) are published first.
   for (int64_t chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
     // The warp's rows warp, warp + 8, ... of the chunk: lane j < 8 resolves row j's
-    // expert (binary search), token and padded position at once, so the rows' copies
-    // below do not each wait for their own index load first.
+    // expert (binary search), token and padded position at once.
     int64_t my_t = -1, my_p = 0;  // -1: no row (past A, or a failed bounds check)
-    if (lane < kGatherChunk / 8) {
-      const int64_t q = chunk * kGatherChunk + warp + 8 * lane;
+    if (lane < kGatherChunk / kGatherWarps) {
+      const int64_t q = chunk * kGatherChunk + warp + kGatherWarps * lane;
       if (q < A) {
         int lo = 0, hi = P.E;  // s_off[lo] <= q < s_off[hi]
         while (hi - lo > 1) {
           const int mid = (lo + hi) >> 1;
-          if (s_off[mid] <= q) lo = mid; else hi = mid;
+          if (S.s_off[mid] <= q) lo = mid; else hi = mid;
         }
         const int a = P.perm[q];
         const int64_t t = a / P.k;
-        const int64_t p = static_cast<int64_t>(s_mt[lo]) * 128 + (q - s_off[lo]);
+        const int64_t p = static_cast<int64_t>(S.s_mt[lo]) * 128 + (q - S.s_off[lo]);
         if (a < 0 || t >= P.T || p >= R) {
           latch(P.status, MOE_ERR_DEVICE_BOUNDS);
         } else {
@@ -314,44 +338,81 @@ __global__ void __launch_bounds__(256, 5) gather_rows_kernel(GatherParams P) {
         }
       }
     }
+    if (lane < kGatherChunk / kGatherWarps) {
+      S.rt[warp][lane] = my_t;
+      S.rp[warp][lane] = my_p;
+    }
+    __syncwarp();
+    const int64_t* tj = S.rt[warp];
+    const int64_t* pj = S.rp[warp];
+    // scale words (UMMA layout, one 4-byte word per 128-column group) and readiness rows
 #pragma unroll 1
-    for (int j = 0; j < kGatherChunk / 8; ++j) {
-      const int r = warp + 8 * j;
-      const int64_t t = __shfl_sync(kFull, my_t, j), p = __shfl_sync(kFull, my_p, j);
+    for (int j = 0; j < kGatherChunk / kGatherWarps; ++j) {
+      const int64_t t = tj[j], p = pj[j];
       int b = -1;
       if (t >= 0) {
-        const int64_t rb = P.row_bytes;
-        const uint4* src = reinterpret_cast<const uint4*>(P.q_tok + t * rb);
-        uint4* dst = reinterpret_cast<uint4*>(P.q_out + p * rb);
-        const int n16 = static_cast<int>(rb >> 4);
-        // the row's scale words are loaded with its first batch of codes
-        const uint32_t* ssrc =
-            P.s_tok ? reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5)) : nullptr;
-        const uint32_t sw0 = ssrc && lane < kg ? ssrc[lane] : 0u;
-        const uint32_t sw1 = ssrc && lane + 32 < kg ? ssrc[lane + 32] : 0u;
-        // 8 loads per lane in flight (4 KB per warp) before the stores
-        for (int i0 = lane; i0 < n16; i0 += 32 * 8) {
-          uint4 v[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            v[u] = i0 + 32 * u < n16 ? ld_nc_v4(src + i0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (i0 + 32 * u < n16) __stcs(dst + i0 + 32 * u, v[u]);
-        }
-        if (ssrc) {
-          if (lane < kg)
-            *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * lane, kg)) = sw0;
-          if (lane + 32 < kg)
-            *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * (lane + 32), kg)) =
-                sw1;
-          for (int g = lane + 64; g < kg; g += 32)  // rows wider than 8192 columns
+        if (P.s_tok) {
+          const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(P.s_tok + t * (d >> 5));
+          for (int g = lane; g < kg; g += 32)
             *reinterpret_cast<uint32_t*>(P.s_out + umma_scale_offset(p, 4 * g, kg)) = ssrc[g];
         }
         if (P.ready) b = static_cast<int>(p / P.ready_rows);
       }
-      if (P.ready && lane == 0) s_b[r] = b;
+      if (P.ready && lane == 0) S.s_b[warp + kGatherWarps * j] = b;
     }
+    // the codes: lane 0 copies the warp's rows piece by piece with bulk copies, through
+    // shared memory (load of the next piece in flight while the current one is stored)
+    if (lane == 0) {
+      constexpr int NJ = kGatherChunk / kGatherWarps;
+      int lj = 0, sj = 0;
+      int64_t loff = 0, soff = 0;
+      int lb = 0, sbf = 0;
+      while (lj < NJ && tj[lj] < 0) ++lj;
+      sj = lj;
+      uint32_t armed = 0;
+      auto issue_load = [&]() {
+        const uint32_t bytes = static_cast<uint32_t>(rb - loff < kGatherPiece ? rb - loff : kGatherPiece);
+        const uint32_t bar = smem_u32(&S.bar[warp][lb]);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load(smem_u32(S.buf[warp][lb]), P.q_tok + tj[lj] * rb + loff, bytes, bar);
+        armed |= 1u << lb;
+        loff += kGatherPiece;
+        if (loff >= rb) {
+          loff = 0;
+          do ++lj; while (lj < NJ && tj[lj] < 0);
+        }
+        lb ^= 1;
+      };
+      if (lj < NJ) issue_load();
+      while (sj < NJ) {
+        if (lj < NJ) {
+          bulk_wait_read<0>();  // the buffer's previous store has read it
+          issue_load();
+        }
+        if (!mbar_wait(smem_u32(&S.bar[warp][sbf]), (ph >> sbf) & 1u, &S.abort_flag, P.status))
+          break;
+        ph ^= 1u << sbf;
+        armed &= ~(1u << sbf);
+        const uint32_t bytes = static_cast<uint32_t>(rb - soff < kGatherPiece ? rb - soff : kGatherPiece);
+        bulk_store(P.q_out + pj[sj] * rb + soff, smem_u32(S.buf[warp][sbf]), bytes);
+        bulk_commit();
+        soff += kGatherPiece;
+        if (soff >= rb) {
+          soff = 0;
+          do ++sj; while (sj < NJ && tj[sj] < 0);
+        }
+        sbf ^= 1;
+      }
+      // after an abort, let the loads still in flight land before the buffers are reused
+      for (int bq = 0; bq < 2; ++bq)
+        if ((armed >> bq) & 1u) {
+          mbar_drain(smem_u32(&S.bar[warp][bq]), (ph >> bq) & 1u);
+          ph ^= 1u << bq;
+        }
+      bulk_wait_all();            // the rows are in global memory before they are published
+      fence_proxy_async_global();  // (written through the async proxy)
+    }
+    __syncwarp();  // the warp's row table is rewritten by the next chunk
     if (P.ready) {
       // Publish the chunk: every thread's stores are made visible device-wide, then one
       // thread lowers the minibatch counters by the chunk's rows (release; the consumer
@@ -361,7 +422,7 @@ __global__ void __launch_bounds__(256, 5) gather_rows_kernel(GatherParams P) {
       if (threadIdx.x == 0) {
         int cur = -1, n = 0;
         for (int r = 0; r <= kGatherChunk; ++r) {
-          const int b = r < kGatherChunk ? s_b[r] : -1;
+          const int b = r < kGatherChunk ? S.s_b[r] : -1;
           if (b != cur) {
             if (cur >= 0 && cur != P.withhold) red_release_add(P.ready + cur, -n);
             cur = b;
@@ -379,24 +440,28 @@ cudaError_t launch_gather_rows(const GatherParams& P, int num_sms, cudaStream_t 
   const int64_t A = P.T * P.k;
   if (A <= 0) return cudaSuccess;
   const int64_t blocks = (A + kGatherChunk - 1) / kGatherChunk;
-  // All SMs: the whole grid is resident at once (so the consumer GEMM, a programmatic
-  // dependent, launches at once and takes each SM as its dispatch CTAs finish).  Running
-  // the dispatch on a quarter of the SMs beside the GEMM from the start was measured
-  // slower (the GEMM's registers leave room for only ~8 dispatch warps per SM).
-  const int grid = static_cast<int>(blocks < 8LL * num_sms ? blocks : 8LL * num_sms);
-  static bool carveout_set[64] = {false};
+  if (P.row_bytes % 16 || P.row_bytes <= 0) return cudaErrorInvalidValue;  // bulk copies
+  // All SMs, three CTAs each (the piece buffers take 72 KB of shared memory per CTA): the
+  // whole grid is resident at once, so the consumer GEMM, a programmatic dependent,
+  // launches at once and takes each SM as its dispatch CTAs finish.  Running the dispatch
+  // on a quarter of the SMs beside the GEMM from the start was measured slower.
+  const int grid = static_cast<int>(blocks < 3LL * num_sms ? blocks : 3LL * num_sms);
+  static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 64 || !carveout_set[dev]) {
-    // configure the SMs this kernel lands on with the largest shared-memory carveout, so
-    // that a GEMM CTA can join it there without waiting for the SM to drain
-    const cudaError_t e = cudaFuncSetAttribute(gather_rows_kernel,
-                                               cudaFuncAttributePreferredSharedMemoryCarveout,
-                                               static_cast<int>(cudaSharedmemCarveoutMaxShared));
+  if (dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gather_rows_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kGatherSmemBytes));
     if (e != cudaSuccess) return e;
-    if (dev < 64) carveout_set[dev] = true;
+    // the largest shared-memory carveout on the SMs this kernel lands on, so that a GEMM
+    // CTA takes an SM without a reconfiguration once the dispatch CTAs there finish
+    e = cudaFuncSetAttribute(gather_rows_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[dev] = true;
   }
-  gather_rows_kernel<<<grid, 256, 0, stream>>>(P);
+  gather_rows_kernel<<<grid, kGatherWarps * 32, kGatherSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 
