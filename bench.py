@@ -766,6 +766,93 @@ def run_ep(args, case):
     print(json.dumps(line), flush=True)
 
 
+def run_variants(args, case):
+    """The layer's BF16 variant (forward, bf16 operands on tcgen05 kind::f16) beside the
+    MXFP8 forward, and the router GEMM (logits = x . W_r^T, and its backward), timed on one
+    GPU with CUDA events: one JSON line (not the default line)."""
+    import numpy as np
+    import torch
+
+    import synth
+    import token_dispatch_grouped_top_b200 as moe
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dims = moe.Dims(case.T, case.d, case.f, case.E, case.k, case.score_fn)
+    x = torch.from_numpy(synth.make_x(case).view(np.int16)).view(torch.bfloat16).to(dev)
+    lg = torch.from_numpy(synth.make_logits(case)).to(dev)
+    peaks = _peaks()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    def stages(fn):
+        moe.profile_collect()
+        moe.profile_enable(True)
+        for _ in range(args.steps):
+            fn()
+        torch.cuda.synchronize()
+        moe.profile_enable(False)
+        return {n: t / max(c, 1) for n, (t, c) in moe.profile_collect().items()}
+
+    A = case.T * case.k
+    gu_fl, dn_fl = 4.0 * A * case.d * case.f, 2.0 * A * case.d * case.f
+    out = torch.empty((case.T, case.d), dtype=torch.bfloat16, device=dev)
+    # MXFP8 forward (the layer as benchmarked), then the BF16 variant on the same inputs
+    wg, wu, wd = synth.expert_weights_torch(case, dev)
+    pw = moe.prepare_weights(wg, wu, wd, dims)
+    ws = moe.workspace(dims, moe.OP_FORWARD, dev)
+    ms_mx = timed(lambda: moe.forward(x, lg, pw, ws=ws, out=out))
+    del pw, ws
+    pw16 = moe.prepare_weights_bf16(wg, wu, wd, dims)
+    del wg, wu, wd
+    torch.cuda.empty_cache()
+    ws16 = moe.workspace(dims, moe.OP_FORWARD_BF16, dev)
+    f16 = lambda: moe.forward_bf16(x, lg, pw16, ws=ws16, out=out)   # noqa: E731
+    ms_16 = timed(f16)
+    st16 = stages(f16)
+    status = moe.device_status(ws16)
+    del pw16, ws16
+    torch.cuda.empty_cache()
+    bf16 = {"ms_per_step": ms_16, "tokens_per_s": case.T / (ms_16 * 1e-3),
+            "stages_ms": st16, "mxfp8_forward_ms": ms_mx,
+            "bf16_over_mxfp8_time": ms_16 / ms_mx}
+    for name, fl in (("gateup", gu_fl), ("down", dn_fl)):
+        if name in st16:
+            tf = fl / (st16[name] * 1e-3) / 1e12
+            bf16[name + "_tflops"] = tf
+            bf16[name + "_frac_bf16"] = tf / peaks["bf16"]
+    # router GEMM and its backward
+    wr = torch.from_numpy(synth.make_router_weight(case).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    g = torch.from_numpy(synth.make_dlogits(case)).to(dev)
+    wsr = moe.workspace(moe._router_dims(case.T, case.d, case.E), moe.OP_ROUTER, dev)
+    logits = torch.empty((case.T, case.E), dtype=torch.float32, device=dev)
+    ms_rf = timed(lambda: moe.router_logits(x, wr, ws=wsr, out=logits))
+    ms_rb = timed(lambda: moe.router_grads(g, x, wr, ws=wsr))
+    status = max(status, moe.device_status(wsr))
+    rfl = 2.0 * case.T * case.d * case.E
+    router = {"forward_ms": ms_rf, "forward_tflops": rfl / (ms_rf * 1e-3) / 1e12,
+              "backward_ms": ms_rb, "backward_tflops": 2 * rfl / (ms_rb * 1e-3) / 1e12,
+              "note": "backward includes the bf16 copies of G, G^T, W_r^T and x^T"}
+    line = {"metric": "BF16 variant forward and router GEMM, one GPU", "steps": args.steps,
+            "warmup": args.warmup, "bf16_variant": bf16, "router": router,
+            "peak_bf16_tflops": peaks["bf16"], "peak_src": peaks["src"],
+            "device_status": status,
+            "config": {"workload": case.name, "T": case.T, "d": case.d, "f": case.f,
+                       "E": case.E, "k": case.k}}
+    print(json.dumps(line), flush=True)
+
+
 def sweep(args):
     """One JSON line per synthetic configuration and pass (forward, forward+backward).
     Not the default line: a table for the design notes."""
@@ -792,6 +879,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true", help="every synthetic config, one line each")
+    ap.add_argument("--variants", action="store_true",
+                    help="the BF16 layer variant and the router GEMM, one JSON line")
     ap.add_argument("--ep-ranks", type=int, default=0,
                     help="expert-parallel forward with this many ranks emulated on one GPU")
     args = ap.parse_args()
@@ -803,6 +892,9 @@ def main():
         return
     if args.ep_ranks:
         run_ep(args, case)
+        return
+    if args.variants:
+        run_variants(args, case)
         return
     if args.impl == "reference":
         run_reference(args, case)
