@@ -138,11 +138,17 @@ def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, ms: float) ->
     return world * tokens_per_rank * steps / (ms * 1e-3)
 
 
-def algorithmic_bytes(case, bwd: bool) -> dict:
+def algorithmic_bytes(case, bwd: bool, tail_rows=None) -> dict:
     """Bytes each stage must move by the method (the survey's per-unit figures times the
     units of one step): MX bytes include the 1/32 scale overhead, activations count the
     A = T*k assignments (no tile padding), expert outputs and input gradients per
-    assignment are bf16, weights are read once."""
+    assignment are bf16, weights are read once.
+
+    tail_rows (backward): the rows of the experts' partial last tiles.  The dgrad GEMM of
+    the down projection runs the SwiGLU backward in its epilogue for every other row, so G
+    is not stored for them: those rows' SwiGLU bytes (g|u and h^ read, [dg|du]^ written)
+    count in that GEMM's stage, and the SwiGLU stage keeps the tail rows (G written and
+    read) and the per-row partial sums of d(w) (f/128 fp32 each)."""
     T, d, f, E, k = case.T, case.d, case.f, case.E, case.k
     A = T * k
     mx = 1 + 1 / 32
@@ -164,6 +170,11 @@ def algorithmic_bytes(case, bwd: bool) -> dict:
             "bwd_transpose": 2 * A * (2 * d + 3 * f) * mx,
             "bwd_wgrad": 2 * E * 3 * d * f + A * (2 * d + 3 * f) * mx,
         })
+        if tail_rows is not None:
+            full = A - tail_rows
+            by["bwd_dgrad_down"] = (E * f * d * mx + A * d * mx + full * f * (4 + 3 * mx) +
+                                    tail_rows * 2 * f)
+            by["bwd_swiglu"] = tail_rows * f * (2 + 4 + 3 * mx) + A * (f // 128) * 4
     return by
 
 
@@ -172,7 +183,7 @@ def algorithmic_bytes(case, bwd: bool) -> dict:
 F16S = 2 + 1 / 32
 
 
-def implementation_bytes(case, bwd: bool, rows_used: int, rows_out: int) -> dict:
+def implementation_bytes(case, bwd: bool, rows_used: int, rows_out: int, tail_rows=None) -> dict:
     """Bytes the kernels actually move where they differ from the algorithmic count:
     scaled-fp16 expert outputs and input gradients, fp32 G, and the tile-padded rows (``rows_used``:
     rows inside some expert segment; ``rows_out``: rows a GEMM with such an output
@@ -180,13 +191,17 @@ def implementation_bytes(case, bwd: bool, rows_used: int, rows_out: int) -> dict
     T, d, f, k = case.T, case.d, case.f, case.k
     A = T * k
     mx = 1 + 1 / 32
-    alg = algorithmic_bytes(case, bwd)
+    alg = algorithmic_bytes(case, bwd, tail_rows)
     impl = dict(alg)
     impl["down"] = alg["down"] - 2 * A * d + F16S * rows_out * d
     impl["combine"] = F16S * A * d + 2 * T * d
     if bwd:
-        impl["bwd_dgrad_down"] = alg["bwd_dgrad_down"] - 2 * A * f + 4 * rows_out * f
-        impl["bwd_swiglu"] = A * f * (4 + 4 + 3 * mx)
+        if tail_rows is None:
+            impl["bwd_dgrad_down"] = alg["bwd_dgrad_down"] - 2 * A * f + 4 * rows_out * f
+            impl["bwd_swiglu"] = A * f * (4 + 4 + 3 * mx)
+        else:  # G (fp32) stored and read for the tail rows only
+            impl["bwd_dgrad_down"] = alg["bwd_dgrad_down"] + 2 * tail_rows * f
+            impl["bwd_swiglu"] = alg["bwd_swiglu"] + 2 * tail_rows * f
         impl["bwd_dgrad_gateup"] = alg["bwd_dgrad_gateup"] - 2 * A * d + F16S * rows_out * d
         impl["bwd_dx"] = F16S * A * d + 2 * T * d
         impl["bwd_transpose"] = 2 * rows_used * (2 * d + 3 * f) * mx
@@ -206,13 +221,14 @@ def layer_flops(case, bwd: bool) -> dict:
 DATA_MOVEMENT = ("route", "permute", "combine", "bwd_dout", "bwd_dx")
 
 
-def layer_summary(case, stage_ms: dict, ms_step: float, peaks: dict, bwd: bool) -> dict:
+def layer_summary(case, stage_ms: dict, ms_step: float, peaks: dict, bwd: bool,
+                  tail_rows=None) -> dict:
     """Whole-layer roofline of one step: algorithmic FLOPs and HBM bytes
     (:func:`algorithmic_bytes`), t_roof = max(FLOPs / P_mxfp8, bytes / BW_copy), and the
     fraction of each resource the measured step reaches.  Also the aggregate HBM fraction
     (sum of bytes over sum of times) of the data-movement kernels: routing, dispatch and
     combine (forward) and, with the backward, its dispatch and combine twins."""
-    by, fl = algorithmic_bytes(case, bwd), layer_flops(case, bwd)
+    by, fl = algorithmic_bytes(case, bwd, tail_rows), layer_flops(case, bwd)
     flops, nbytes = sum(fl.values()), sum(by.values())
     p_mx, bw = 2.0 * peaks["bf16"] * 1e12, peaks["hbm"] * 1e9
     t_roof = max(flops / p_mx, nbytes / bw)
@@ -232,10 +248,10 @@ def layer_summary(case, stage_ms: dict, ms_step: float, peaks: dict, bwd: bool) 
             "data_movement_hbm_frac": agg(moves), "data_movement_kernels": moves}
 
 
-def _safe_layer_summary(case, stage_info, ms_step, peaks, bwd):
+def _safe_layer_summary(case, stage_info, ms_step, peaks, bwd, tail_rows=None):
     try:
         return layer_summary(case, {n: v["ms_per_launch"] for n, v in stage_info.items()},
-                             ms_step, peaks, bwd)
+                             ms_step, peaks, bwd, tail_rows)
     except Exception as e:  # reporting only: never lose the benchmark line over it
         return {"error": repr(e)}
 
@@ -576,8 +592,9 @@ def run_ours(args, case):
         ws, dims, moe.OP_FORWARD, "counts", 4 * case.E).view(torch.int32)).cpu().numpy()
     r_used = int(((counts_h + 127) // 128 * 128).sum())
     r_out = int((counts_h // 128 * 128 + (counts_h % 128 + 31) // 32 * 32).sum())
-    alg_bytes = algorithmic_bytes(case, bwd)
-    impl_bytes = implementation_bytes(case, bwd, r_used, r_out)
+    tail = int((counts_h % 128).sum())   # rows of the experts' partial last tiles
+    alg_bytes = algorithmic_bytes(case, bwd, tail)
+    impl_bytes = implementation_bytes(case, bwd, r_used, r_out, tail)
     stage_info = {}
     for name, (tot_ms, n) in stages.items():
         s = {"ms_per_launch": tot_ms / max(n, 1), "launches": n}
@@ -643,7 +660,7 @@ def run_ours(args, case):
         "fwd_tokens_per_s": world * case.T / (fwd_ms * 1e-3),
         "bwd_tokens_per_s": world * case.T / (bwd_ms * 1e-3) if bwd else None,
         "layer_tflops": step_flops / (ms_step * 1e-3) / 1e12,
-        "layer_roofline": _safe_layer_summary(case, stage_info, ms_step, peaks, bwd),
+        "layer_roofline": _safe_layer_summary(case, stage_info, ms_step, peaks, bwd, tail),
         "layer_frac_mxfp8": step_flops / (ms_step * 1e-3) / 1e12 / mx_peak,
         "fwd_frac_mxfp8": (fl["gateup"] + fl["down"]) / (fwd_ms * 1e-3) / 1e12 / mx_peak,
         "forward_only": fwd_only,

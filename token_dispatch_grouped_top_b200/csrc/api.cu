@@ -209,7 +209,7 @@ struct WsLayout {
   int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0, ys = 0;
   int64_t tq = 0, ts = 0;  // per-token MX copy of x (forward) or dout (backward)
   // backward
-  int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, dxas = 0, gbuf = 0;
+  int64_t dq = 0, ds = 0, dgu_q = 0, dgu_s = 0, dxa = 0, dxas = 0, gbuf = 0, dwpart = 0;
   int64_t xt_q = 0, xt_s = 0, ht_q = 0, ht_s = 0, gt_q = 0, gt_s = 0, yt_q = 0, yt_s = 0;
   int64_t total = 0;
 };
@@ -272,6 +272,7 @@ WsLayout ws_layout(const moe_dims* D, int op) {
     L.dxa = c.take(2 * R * d);     // scaled fp16
     L.dxas = c.take(R * (d / 32));
     L.gbuf = c.take(4 * R * f);    // fp32: it feeds the MX requantisation of [dg|du]
+    L.dwpart = c.take(4 * R * (f / 128));  // partial sums of <G, h^> per 128 features
     L.xt_q = c.take(d * R);
     L.xt_s = c.take(moe_umma_scale_bytes(d, R));
     L.ht_q = c.take(f * R);
@@ -1146,11 +1147,22 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.tile_ctr = at<uint32_t>(ws, kCtrBwdDgradDown);
       P.ready = ready;
       P.ready_rows = mb;
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_STORE_F32_TMA, ta, tb, tg, tg, P, sms, st, true)));
+      // full tiles: the SwiGLU backward in the epilogue (G never stored); partial tiles: G
+      P.f = f;
+      P.gu = S->gu;
+      P.hq = S->hq;
+      P.hs = S->hs;
+      P.perm = S->perm;
+      P.offsets = S->offsets;
+      P.topk_w = S->topk_w;
+      P.dgu_q = dgu_q;
+      P.dgu_s = dgu_s;
+      P.dw_part = at<float>(ws, L.dwpart);
+      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_DGRAD_SWIGLU, ta, tb, tg, tg, P, sms, st, true)));
     }
     {  // d(router weights), SwiGLU backward, [dg|du] -> MXFP8 along f
       StageScope sc(MOE_STAGE_BWD_SWIGLU, st);
-      SwigluBwdParams P;
+      SwigluBwdParams P = {};
       P.G = gbuf;
       P.gu = S->gu;
       P.h_q = S->hq;
@@ -1165,6 +1177,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.dw_route = dw_route;
       P.dgu_q = dgu_q;
       P.dgu_s = dgu_s;
+      P.dw_part = at<float>(ws, L.dwpart);
       MOE_TRY(cuda_ok(launch_swiglu_bwd(P, sms, st)));
     }
     {  // dXa = [dg|du]^ . [Wg|Wu]'^T

@@ -25,17 +25,6 @@
 
 namespace moe {
 
-__device__ __forceinline__ float e4m3_to_f32_t(uint32_t c) {
-  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
-  const float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20))
-                    : static_cast<float>(m) * 0.001953125f;
-  return (c & 0x80u) ? -v : v;
-}
-
-__device__ __forceinline__ float e8m0_to_f32_t(uint32_t b) {
-  return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
-}
-
 constexpr int kTqThreads = 256;
 constexpr int kTqCtasPerSm = 3;
 constexpr uint32_t kTqTile = 128 * 128;  // bytes of codes per 128 x 128 tile
@@ -197,7 +186,7 @@ __global__ void __launch_bounds__(kTqThreads) transpose_quant_kernel(
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const uint32_t e = (sw >> (8 * q)) & 0xFFu;
-        S.mul[q][tid] = tid < nv ? e8m0_to_f32_t(e) * w : 0.f;
+        S.mul[q][tid] = tid < nv ? e8m0_to_f32(e) * w : 0.f;
       }
     }
     if (__syncthreads_or(!ok)) break;
@@ -251,7 +240,9 @@ cudaError_t launch_transpose_quant(const CUtensorMap& tm_src, const CUtensorMap&
 
 // ---------------------------------------------------------------------------------------
 // SwiGLU backward and d(router weights), one warp per assignment row, after the dgrad GEMM
-// of the down projection has written G = dout^ . Wd'^T (fp32, padded expert order; it is
+// of the down projection.  Rows of full 128-row tiles were done in that GEMM's epilogue
+// (dw_part given): here only their d(w) is summed from its partials.  For the rest (an
+// expert's last, partial tile) the GEMM wrote G = dout^ . Wd'^T (fp32, padded order; it is
 // kept in fp32 because dg, du are requantised from it, where a coarser G would move values
 // across E4M3 rounding boundaries):
 //   dw_route[a] = <G, h^>,  dh = w * G,  dg = dh * u * s * (1 + g (1 - s)),
@@ -261,7 +252,6 @@ cudaError_t launch_transpose_quant(const CUtensorMap& tm_src, const CUtensorMap&
 // ---------------------------------------------------------------------------------------
 constexpr int kSbMaxE = 1024;
 
-__device__ __forceinline__ float sigmoid_fast_b(float x) { return __frcp_rn(1.f + __expf(-x)); }
 
 __device__ __forceinline__ void quant8_store(const float (&v)[8], int lane, uint8_t* q_dst,
                                              uint8_t* s_base, int64_t row, int64_t kb,
@@ -307,6 +297,21 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams P) {
     }
     const int64_t row = s_pad[lo] + (q - s_off[lo]);
     const int a = P.perm[q];
+    if (P.dw_part) {
+      // a row of a full 128-row tile: the dgrad GEMM's epilogue wrote its [dg | du] and the
+      // partial sums of <G, h^> per 128 features; their sum, in block order, is d(w)
+      const int64_t rel = q - s_off[lo], cnt = s_off[lo + 1] - s_off[lo];
+      if ((rel / 128 + 1) * 128 <= cnt) {
+        // all partials loaded at once (lanes), summed by a fixed shuffle tree
+        const float* part = P.dw_part + row * (f >> 7);
+        float acc = 0.f;
+        for (int nb = lane; nb < (f >> 7); nb += 32) acc += part[nb];
+#pragma unroll
+        for (int off = 16; off; off >>= 1) acc += __shfl_down_sync(kFull, acc, off);
+        if (lane == 0) P.dw_route[a] = acc;
+        continue;
+      }
+    }
     const float w = P.topk_w[a];
     const float* Grow = P.G + row * f;
     const uint16_t* grow = P.gu + row * 2 * f;
@@ -329,13 +334,10 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(SwigluBwdParams P) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t code = (hw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-        dwp = fmaf(Gv[i], e4m3_to_f32_t(code) * hsc, dwp);
+        dwp = fmaf(Gv[i], e4m3_to_f32(code) * hsc, dwp);
         const float gb = bf16_bits_to_f32((gw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
         const float ub = bf16_bits_to_f32((uw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
-        const float dh = w * Gv[i];
-        const float sg = sigmoid_fast_b(gb);
-        dg[i] = dh * ub * sg * (1.f + gb * (1.f - sg));
-        du[i] = dh * gb * sg;
+        swiglu_bwd_elem(Gv[i], w, gb, ub, dg[i], du[i]);
       }
       quant8_store(dg, lane, P.dgu_q + row * 2 * f + fi, P.dgu_s, row, fi >> 5, kg2);
       quant8_store(du, lane, P.dgu_q + row * 2 * f + f + fi, P.dgu_s, row, (f + fi) >> 5, kg2);

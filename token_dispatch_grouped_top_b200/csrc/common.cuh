@@ -358,6 +358,32 @@ __device__ __forceinline__ uint32_t mx_quant_block32(const float (&v)[32], uint3
   return static_cast<uint32_t>(s + 127);
 }
 
+// E4M3 code -> its value (exact in fp32); E8M0 byte -> 2^(b - 127) (byte 0: 2^-127).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
+  const float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20))
+                    : static_cast<float>(m) * 0.001953125f;
+  return (c & 0x80u) ? -v : v;
+}
+
+__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
+  return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
+}
+
+// sigmoid(x) = 1 / (1 + e^-x) with the fast exponential and a rounded reciprocal (relative
+// error ~1e-6; large |x|: e^-x -> 0 or inf gives exactly 1 or 0).
+__device__ __forceinline__ float sigmoid_fast(float x) { return __frcp_rn(1.f + __expf(-x)); }
+
+// SwiGLU backward of one element, h = silu(g) * u: with dh = w * G,
+// dg = dh * u * s * (1 + g (1 - s)), du = dh * g * s, s = sigmoid(g).
+__device__ __forceinline__ void swiglu_bwd_elem(float G, float w, float g, float u, float& dg,
+                                                float& du) {
+  const float dh = w * G;
+  const float s = sigmoid_fast(g);
+  dg = dh * u * s * (1.f + g * (1.f - s));
+  du = dh * g * s;
+}
+
 // Byte offset of the scale of (row r, 32-block kb) in the UMMA scale layout of a matrix
 // with `kgroups` = K/128 column groups.
 __host__ __device__ __forceinline__ int64_t umma_scale_offset(int64_t r, int64_t kb,

@@ -61,7 +61,10 @@ struct ModeCfg {
   // operand kind: MXFP8 with block scales, or bf16 (the layer's BF16 variant, kind::f16)
   static constexpr bool kBf16 = MODE == GEMM_GATEUP_BF16 || MODE == GEMM_STORE_F32_BF16;
   static constexpr bool kGateUp = MODE == GEMM_GATEUP_SWIGLU || MODE == GEMM_GATEUP_BF16;
-  static constexpr bool kStoreF32 = MODE == GEMM_STORE_F32_TMA || MODE == GEMM_STORE_F32_BF16;
+  static constexpr bool kStoreF32 = MODE == GEMM_STORE_F32_TMA || MODE == GEMM_STORE_F32_BF16 ||
+                                    MODE == GEMM_DGRAD_SWIGLU;
+  // full tiles of the dgrad of the down projection run the SwiGLU backward in the epilogue
+  static constexpr bool kSwigluBwd = MODE == GEMM_DGRAD_SWIGLU;
   static constexpr uint32_t kTx = kBf16 ? kABytes + kBBytes : kTxBytes;
   static constexpr bool kTmaStore = kStoreF32 || MODE == GEMM_WGRAD_BF16;
   static constexpr int kStages = kTmaStore ? 3 : 4;
@@ -207,11 +210,9 @@ __device__ __forceinline__ void store_swapped_chunk(const float (&v)[32], int tb
   stg_buf ^= 1;
 }
 
-// sigmoid(x) = 1 / (1 + e^-x) with the fast exponential and a rounded reciprocal: the
-// epilogues evaluate it once per output element, and the IEEE exp + division sequence
-// kept the transcendental pipe busy for as long as the MMA main loop of a short-K tile.
-// Relative error ~1e-6 (large |x|: e^-x -> 0 or inf gives exactly 1 or 0).
-__device__ __forceinline__ float sigmoid_fast(float x) { return __frcp_rn(1.f + __expf(-x)); }
+// (sigmoid_fast, common.cuh: the epilogues evaluate it once per output element, and the IEEE
+// exp + division sequence kept the transcendental pipe busy for as long as the MMA main loop
+// of a short-K tile.)
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -572,6 +573,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(taddr + 64 * h + 32, v1);    // gate features 64h+32 .. 64h+63
         tmem_ld32(taddr + 128 + 64 * h, v2);   // up, same features
         tmem_ld32(taddr + 128 + 64 * h + 32, v3);
+      } else if constexpr (ModeCfg<MODE>::kSwigluBwd) {
+        // columns 64..127 first go to this warp's staging buffers (8 KB: [64 columns][32
+        // rows], lane-contiguous), so that only 64 accumulator registers are live at a time;
+        // an earlier (swapped) tile's TMA store may still be reading those buffers
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        float* stash = reinterpret_cast<float*>(S.stg[2 * (warp - 2)]);
+        tmem_ld32(taddr + 128 * h + 64, v2);
+        tmem_ld32(taddr + 128 * h + 96, v3);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          stash[i * 32 + lane] = v2[i];
+          stash[(32 + i) * 32 + lane] = v3[i];
+        }
+        tmem_ld32(taddr + 128 * h, v0);
+        tmem_ld32(taddr + 128 * h + 32, v1);
       } else {
         tmem_ld32(taddr + 128 * h, v0);
         tmem_ld32(taddr + 128 * h + 32, v1);
@@ -585,6 +603,90 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       acc_phase ^= 1u;
 
       const int m = 32 * q + lane;
+      if constexpr (ModeCfg<MODE>::kSwigluBwd) {
+        // A full tile (an expert's partial last tile runs swapped and stores G): for this
+        // row's 128 features, d(combine weight) partial <G, h^>, then dg, du from the saved
+        // g | u, each 32-feature block requantised (MX along 2f) where the SwiGLU-backward
+        // kernel would have stored it.
+        const int64_t row = ti.a_row0 + m;
+        const int f = P.N;
+        const int64_t pos = P.offsets[ti.g] + (row - static_cast<int64_t>(S.prefix[ti.g]) * BM);
+        const float w = P.topk_w[P.perm[pos]];
+        const int nb = ti.j * BN + 128 * h;  // first feature of this thread's 128
+        const uint16_t* grow = P.gu + row * 2 * f;
+        const uint8_t* hrow = P.hq + row * f;
+        const int64_t kgh = f >> 7, kg2 = (2 * f) >> 7;
+        const float* stash = reinterpret_cast<const float*>(S.stg[2 * (warp - 2)]);
+        float dwp = 0.f;
+        uint32_t sbg = 0, sbu = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float G[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            G[i] = c == 0 ? v0[i] : c == 1 ? v1[i] : stash[((c - 2) * 32 + i) * 32 + lane];
+          const int fb = nb + 32 * c;
+          uint4 gq[4], uq[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            gq[i] = __ldg(reinterpret_cast<const uint4*>(grow + fb) + i);
+            uq[i] = __ldg(reinterpret_cast<const uint4*>(grow + f + fb) + i);
+          }
+          const uint4 h0 = __ldg(reinterpret_cast<const uint4*>(hrow + fb));
+          const uint4 h1 = __ldg(reinterpret_cast<const uint4*>(hrow + fb) + 1);
+          const float hsc = e8m0_to_f32(P.hs[umma_scale_offset(row, fb >> 5, kgh)]);
+          const uint32_t gw[16] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y,
+                                   gq[1].z, gq[1].w, gq[2].x, gq[2].y, gq[2].z, gq[2].w,
+                                   gq[3].x, gq[3].y, gq[3].z, gq[3].w};
+          const uint32_t uw[16] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y,
+                                   uq[1].z, uq[1].w, uq[2].x, uq[2].y, uq[2].z, uq[2].w,
+                                   uq[3].x, uq[3].y, uq[3].z, uq[3].w};
+          const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+          // pass 1: <G, h^> and the block maxima of dg and du; pass 2 recomputes dg, du (the
+          // same instructions: the same values) and quantises them four at a time, so no
+          // block array is held in registers
+          float amg = 0.f, amu = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint32_t code = (hw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+            dwp = fmaf(G[i], e4m3_to_f32(code) * hsc, dwp);
+            const float gb = bf16_bits_to_f32((gw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+            const float ub = bf16_bits_to_f32((uw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+            float dg, du;
+            swiglu_bwd_elem(G[i], w, gb, ub, dg, du);
+            amg = fmaxf(amg, fabsf(dg));
+            amu = fmaxf(amu, fabsf(du));
+          }
+          const int sg = mx_scale_exp(amg), su = mx_scale_exp(amu);
+          const float ig = mx_inv_scale(sg), iu = mx_inv_scale(su);
+          sbg |= static_cast<uint32_t>(sg + 127) << (8 * c);
+          sbu |= static_cast<uint32_t>(su + 127) << (8 * c);
+          uint32_t qg[8], qu[8];
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            float dg[4], du[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 4 * i4 + e;
+              const float gb = bf16_bits_to_f32((gw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+              const float ub = bf16_bits_to_f32((uw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+              swiglu_bwd_elem(G[i], w, gb, ub, dg[e], du[e]);
+            }
+            qg[i4] = pack_e4m3x4(dg[0] * ig, dg[1] * ig, dg[2] * ig, dg[3] * ig);
+            qu[i4] = pack_e4m3x4(du[0] * iu, du[1] * iu, du[2] * iu, du[3] * iu);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(P.dgu_q + row * 2 * f + fb);
+          dst[0] = make_uint4(qg[0], qg[1], qg[2], qg[3]);
+          dst[1] = make_uint4(qg[4], qg[5], qg[6], qg[7]);
+          dst = reinterpret_cast<uint4*>(P.dgu_q + row * 2 * f + f + fb);
+          dst[0] = make_uint4(qu[0], qu[1], qu[2], qu[3]);
+          dst[1] = make_uint4(qu[4], qu[5], qu[6], qu[7]);
+        }
+        *reinterpret_cast<uint32_t*>(P.dgu_s + umma_scale_offset(row, nb >> 5, kg2)) = sbg;
+        *reinterpret_cast<uint32_t*>(P.dgu_s + umma_scale_offset(row, (f + nb) >> 5, kg2)) = sbu;
+        P.dw_part[row * (f >> 7) + (nb >> 7)] = dwp;
+        continue;
+      }
       if (ModeCfg<MODE>::kStoreF32) {
         // fp32 rows of 128 columns: four 32-column chunks; whole 32-row boxes are written
         const int32_t x0 = ti.j * BN + 128 * h;
@@ -732,6 +834,8 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& tmA, const CUtensor
       return launch_mode<GEMM_GATEUP_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
     case GEMM_STORE_F32_BF16:
       return launch_mode<GEMM_STORE_F32_BF16>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
+    case GEMM_DGRAD_SWIGLU:
+      return launch_mode<GEMM_DGRAD_SWIGLU>(tmA, tmB, tmC0, tmC1, P, num_sms, stream, pdl);
     default:
       return cudaErrorInvalidValue;
   }

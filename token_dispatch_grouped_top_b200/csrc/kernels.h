@@ -158,6 +158,9 @@ struct SwigluBwdParams {
   float* dw_route;          // [A]
   uint8_t* dgu_q;           // [R, 2f] MX codes of dg | du + UMMA scales
   uint8_t* dgu_s;
+  // nullable: rows of full 128-row tiles were done by the GEMM epilogue (DGRAD_SWIGLU);
+  // their d(combine weight) is the sum of these [R, f/128] partials, in block order
+  const float* dw_part;
 };
 cudaError_t launch_swiglu_bwd(const SwigluBwdParams& P, int num_sms, cudaStream_t stream);
 
@@ -195,6 +198,11 @@ enum GemmMode : int {
   // bytes, 2 per element):
   GEMM_GATEUP_BF16 = 5,    // SwiGLU, h rounded to bf16 [rows, f]
   GEMM_STORE_F32_BF16 = 6, // as STORE_F32_TMA
+  // the dgrad of the down projection with the SwiGLU backward in its epilogue: full
+  // 128-row tiles turn G into [dg | du] (MX along f) and partial sums of <G, h^> without
+  // storing G; an expert's last, partial tile stores G (fp32, as STORE_F32_TMA) for the
+  // SwiGLU-backward kernel
+  GEMM_DGRAD_SWIGLU = 7,
 };
 
 struct GemmParams {
@@ -236,6 +244,15 @@ struct GemmParams {
   // width that is not a multiple of 256 (the router's E experts) run on whole N tiles of
   // a zero-padded B.
   int n_valid;
+  // DGRAD_SWIGLU: the forward's saved g | u (gu), h codes and scales (hq, hs), the layout
+  // (perm, offsets) and routing weights; outputs [dg | du] codes + UMMA scales and, per
+  // row and 128-feature block, the partial sum of G * h^ ([rows, f/128] fp32).
+  const int32_t* perm;
+  const int32_t* offsets;
+  const float* topk_w;
+  uint8_t* dgu_q;
+  uint8_t* dgu_s;
+  float* dw_part;
 };
 // tmC0 / tmC1: output tensor maps of the TMA-store modes (STORE_F32_TMA: fp32 [rows, N],
 // box 32 x 32; WGRAD: bf16 out_a / out_b, box 64 cols x 32 rows); ignored otherwise.
