@@ -253,7 +253,11 @@ moe_status moe_forward_bf16(const moe_dims* dims, const uint16_t* wgu_t, const u
  * dout [T,d] bf16 + saved -> dx [T,d] bf16, dw_route [T,k] fp32 (d loss / d topk_w),
  * dWg, dWu [E,d,f] bf16, dWd [E,f,d] bf16.  Needs the backward weight copies.
  * Every backward GEMM operand is MX-quantised along that GEMM's K (the weight gradients
- * along each expert's tokens); accumulation fp32.  ws: moe_workspace_bytes(BACKWARD). */
+ * along each expert's tokens); accumulation fp32.  For d >= 6144 the SwiGLU backward of
+ * an expert's full 128-row tiles runs in the epilogue of the dgrad GEMM of the down
+ * projection (its K = d is then long enough to hide that work); below that width, and for
+ * every expert's partial last tile, it runs in its own kernel.  The results are the same
+ * either way.  ws: moe_workspace_bytes(BACKWARD). */
 moe_status moe_backward(const moe_dims* dims, const moe_weights* w, const moe_saved* saved,
                         const uint16_t* dout, uint16_t* dx, float* dw_route, uint16_t* dWg,
                         uint16_t* dWu, uint16_t* dWd, void* ws, size_t ws_bytes,

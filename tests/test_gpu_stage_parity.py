@@ -206,14 +206,15 @@ def _backward_stage_parity(moe, case, experts=None, dx_tokens=None):
             print(f"  {what} {nm} stage:")
             assert_close_out(bf16_tensor_f64(grads[nm][e]), ref)
         # 3. dgrad of the down projection, d(combine weight), SwiGLU backward codes
-        # G is stored only for the rows of an expert's partial last tile (the full tiles
-        # run the SwiGLU backward in the GEMM epilogue); the references take the fp64 G
+        # from d = 6144 on G is stored only for the rows of an expert's partial last tile
+        # (the full tiles run the SwiGLU backward in the GEMM epilogue), below it for every
+        # row; the references take the fp64 G
         wdT = _weights_rows(pw, "wdT", wdT_s, E * f, d, e * f + np.arange(f))
         g_ref = mx_values(dq, dsc) @ wdT.T
-        tail = np.arange(n) >= (n // 128) * 128
-        if tail.any():
-            g_gpu = _host_rows(G, R, f, rows[tail]).astype(np.float64)
-            assert_stage_close(g_gpu, g_ref[tail], STAGE_REL, what + " G (partial tile)")
+        stored = np.arange(n) >= (n // 128) * 128 if d >= 6144 else np.ones(n, bool)
+        if stored.any():
+            g_gpu = _host_rows(G, R, f, rows[stored]).astype(np.float64)
+            assert_stage_close(g_gpu, g_ref[stored], STAGE_REL, what + " G")
         assert_stage_close(dw_gpu[asg], np.sum(g_ref * H, axis=1), STAGE_REL,
                            what + " d(combine weight)")
         gu = bf16_tensor_f64(saved.bufs["gu"].view(R, 2 * f).index_select(0, _rows_t(rows)))

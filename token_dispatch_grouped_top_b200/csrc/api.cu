@@ -196,6 +196,7 @@ struct Carve {
 };
 
 // Tile counters of the grouped GEMM launches, in the workspace header (zeroed per call).
+constexpr int kFuseSwigluMinD = 6144;  // d from which the dgrad GEMM runs the SwiGLU backward
 enum : int64_t { kCtrFwdGateUp = 72, kCtrFwdDown = 76, kCtrBwdDgradDown = 72,
                  kCtrBwdDgradGateUp = 76, kCtrBwdWgrad0 = 80, kCtrBwdWgrad1 = 84,
                  kCtrGeneric = 72 };
@@ -1128,6 +1129,10 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
                             at<uint8_t>(ws, L.tq), at<uint8_t>(ws, L.ts), dq, dsc, status, sms,
                             st, ready, mb));
     }
+    // The SwiGLU backward in the dgrad epilogue costs ~30-40K cycles per 128 x 256 tile; it
+    // hides under a tile's MMAs only when K = d is long (measured: 56 K blocks at d = 7168,
+    // -0.15 ms per step; 16 at d = 2048, +0.06 ms), so the fusion is used from this width.
+    const bool fuse_swiglu = d >= kFuseSwigluMinD;
     {  // G = dout^ . Wd'^T (fp32, padded expert order)
       StageScope sc(MOE_STAGE_BWD_DGRAD_DOWN, st);
       CUtensorMap ta, tb, tg;
@@ -1147,7 +1152,8 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.tile_ctr = at<uint32_t>(ws, kCtrBwdDgradDown);
       P.ready = ready;
       P.ready_rows = mb;
-      // full tiles: the SwiGLU backward in the epilogue (G never stored); partial tiles: G
+      // d >= kFuseSwigluMinD: the SwiGLU backward in the epilogue of full tiles (G never
+      // stored for them); partial tiles, and every tile below that width, store G
       P.f = f;
       P.gu = S->gu;
       P.hq = S->hq;
@@ -1158,7 +1164,8 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.dgu_q = dgu_q;
       P.dgu_s = dgu_s;
       P.dw_part = at<float>(ws, L.dwpart);
-      MOE_TRY(cuda_ok(launch_grouped_gemm(GEMM_DGRAD_SWIGLU, ta, tb, tg, tg, P, sms, st, true)));
+      MOE_TRY(cuda_ok(launch_grouped_gemm(fuse_swiglu ? GEMM_DGRAD_SWIGLU : GEMM_STORE_F32_TMA,
+                                          ta, tb, tg, tg, P, sms, st, true)));
     }
     {  // d(router weights), SwiGLU backward, [dg|du] -> MXFP8 along f
       StageScope sc(MOE_STAGE_BWD_SWIGLU, st);
@@ -1177,7 +1184,7 @@ moe_status moe_backward(const moe_dims* D, const moe_weights* W, const moe_saved
       P.dw_route = dw_route;
       P.dgu_q = dgu_q;
       P.dgu_s = dgu_s;
-      P.dw_part = at<float>(ws, L.dwpart);
+      P.dw_part = fuse_swiglu ? at<float>(ws, L.dwpart) : nullptr;
       MOE_TRY(cuda_ok(launch_swiglu_bwd(P, sms, st)));
     }
     {  // dXa = [dg|du]^ . [Wg|Wu]'^T
