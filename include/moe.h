@@ -184,8 +184,8 @@ moe_status moe_route_layout(const moe_dims* dims, const float* logits, int32_t* 
  * nothing is allocated and no workspace is passed.
  *  - The shape rules, pointer checks and device check are those of moe_route_layout.
  *    Problems whose scratch exceeds 8 MiB return MOE_ERR_UNSUPPORTED_SHAPE before any
- *    launch.  The scratch is 256 + 4*nt + 8*nt*E + 4*T*k + 4*(E+1) bytes (each term
- *    rounded up to 256) with nt = ceil(T/64): e.g. E = 256, k = 8 fits T <= 130896.
+ *    launch.  The scratch is 256 + 8*nt*E + 4*T*k + 4*(E+1) bytes (each term rounded up
+ *    to 256) with nt = ceil(T/64): e.g. E = 256, k = 8 fits T <= 131024.
  *  - Every call looks up the array's device address on the current device
  *    (cudaGetSymbolAddress; it allocates nothing), so a device reset is picked up; make
  *    the first call on a device before any stream capture.

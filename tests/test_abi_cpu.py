@@ -76,9 +76,9 @@ def test_dims_rejected_before_any_launch(lib, bad, code):
 
 
 def test_noalloc_scratch_limit_is_host_logic(lib):
-    # E = 256, k = 8: 130896 tokens fill the 8 MiB scratch array exactly; one more token
+    # E = 256, k = 8: 131024 tokens fill the 8 MiB scratch array exactly; one more token
     # is rejected before any CUDA call (so this holds without a GPU)
-    D = _dims(T=130897, d=256, f=256, E=256, k=8, s=1)
+    D = _dims(T=131025, d=256, f=256, E=256, k=8, s=1)
     assert lib.moe_route_layout_noalloc(ctypes.byref(D), 16, 16, 16, 16, 16, 16, 16, None, 16,
                                         None) == 2
     # T > 0 without a status word (checked before the device is touched)

@@ -52,6 +52,21 @@ def test_route_layout_edges(moe, T, E, k, score):
     _route_check(moe, lg, k, score)
 
 
+def test_route_signed_zero_ties(moe):
+    # rows of -0, +0, 1, -1: -0 and +0 tie (lower index first) whichever sign comes first
+    rng = np.random.default_rng(23)
+    lg = rng.choice(np.array([-0.0, 0.0, 1.0, -1.0], np.float32), (700, 64))
+    _route_check(moe, lg, 6, 0)
+
+
+@pytest.mark.parametrize("T,E,k", [(20000, 96, 6), (9000, 256, 8), (17000, 1024, 4)])
+def test_route_many_tiles(moe, T, E, k):
+    # more than 128 tiles of 64 tokens: the lookback runs over several flag windows
+    rng = np.random.default_rng(T + E)
+    lg = (rng.normal(size=(T, E)) + np.linspace(0, 2, E)).astype(np.float32)
+    _route_check(moe, lg, k, 1)
+
+
 def test_route_all_tokens_one_expert_and_empty_batch(moe):
     import torch
     T, E = 500, 16

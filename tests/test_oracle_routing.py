@@ -33,6 +33,17 @@ def test_constructed_ties_lower_index_wins():
     assert idx[2].tolist() == [1, 2, 4]
 
 
+def test_signed_zeros_tie_lower_index_wins():
+    # -0 and +0 are the same value: between them the lower expert index goes first,
+    # whichever of the two carries the minus sign
+    lg = np.full((2, 5), -1.0, np.float32)
+    lg[0, [1, 3]] = [-0.0, 0.0]
+    lg[1, [1, 3]] = [0.0, -0.0]
+    for row in rt.topk_select(lg, 2):
+        assert row.tolist() == [1, 3]
+    assert np.array_equal(rt.topk_select(lg, 4), rt.topk_select_bruteforce(lg, 4))
+
+
 def test_k_equals_E_selects_all_in_logit_order():
     rng = np.random.default_rng(5)
     lg = rng.normal(size=(10, 8)).astype(np.float32)

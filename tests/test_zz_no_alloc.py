@@ -78,13 +78,13 @@ def test_noalloc_matches_workspace_route_and_oracle_twice():
 
 
 def test_noalloc_at_the_scratch_limit():
-    # E = 256, k = 8, T = 130896 needs exactly the 8 MiB of the array; one token more is
+    # E = 256, k = 8, T = 131024 needs exactly the 8 MiB of the array; one token more is
     # rejected before anything is launched
     import torch
 
     import token_dispatch_grouped_top_b200 as moe
     lib = moe.load()
-    case = synth.MoeCase("limit", 130896, 256, 256, 256, 8, 1, "normal0.5", seed=21)
+    case = synth.MoeCase("limit", 131024, 256, 256, 256, 8, 1, "normal0.5", seed=21)
     logits_np = synth.make_logits(case)
     logits = torch.from_numpy(logits_np).cuda()
     dims = moe.Dims(case.T, case.d, case.f, case.E, case.k, case.score_fn).c()

@@ -203,9 +203,9 @@ enum : int64_t { kCtrFwdGateUp = 72, kCtrFwdDown = 76, kCtrBwdDgradDown = 72,
 
 struct WsLayout {
   // header: [0] status word; [64] routing tile counter; [68] routing done counter;
-  // [72, 96) grouped-GEMM tile counters; [128 ...) flags
+  // [72, 96) grouped-GEMM tile counters
   int64_t zero_begin = 64, zero_bytes = 0;
-  int64_t flags = 0, agg = 0, incl = 0, rank = 0, mtile = 0, ready = 0, order = 0;
+  int64_t agg = 0, tstart = 0, rank = 0, mtile = 0, ready = 0, order = 0;
   int64_t idx = 0, w = 0, counts = 0, offsets = 0, perm = 0, inv = 0, pad = 0;
   int64_t xq = 0, xs = 0, hq = 0, hs = 0, y = 0, ys = 0;
   int64_t tq = 0, ts = 0;  // per-token MX copy of x (forward) or dout (backward)
@@ -237,10 +237,9 @@ WsLayout ws_layout(const moe_dims* D, int op) {
   const int64_t nt = route_num_tiles(D->T);
   Carve c;
   c.take(128);  // status word + counters
-  L.flags = c.take(4 * std::max<int64_t>(nt, 1));
-  L.zero_bytes = L.flags + 4 * std::max<int64_t>(nt, 1) - L.zero_begin;
+  L.zero_bytes = 128 - L.zero_begin;
   L.agg = c.take(4 * nt * E);
-  L.incl = c.take(4 * nt * E);
+  L.tstart = c.take(4 * nt * E);
   L.rank = c.take(4 * A);
   L.mtile = c.take(4 * (E + 1));
   L.ready = c.take(4 * (R / 128 + 1));
@@ -425,9 +424,8 @@ moe_status run_route(const moe_dims* D, const float* logits, int32_t* idx, float
   P.pad_offsets = pad;
   P.tile_counter = at<uint32_t>(ws, 64);
   P.done_counter = at<uint32_t>(ws, 68);
-  P.flags = at<uint32_t>(ws, L.flags);
   P.agg = at<int32_t>(ws, L.agg);
-  P.incl = at<int32_t>(ws, L.incl);
+  P.tile_start = at<int32_t>(ws, L.tstart);
   P.status = at<int32_t>(ws, 0);
   return cuda_ok(launch_route_layout(P, perm, inv, num_sms, st));
 }

@@ -21,16 +21,15 @@ struct RouteParams {
   int num_tiles;
   int32_t* topk_idx;
   float* topk_w;
-  int32_t* rank;          // [A] rank of each assignment inside its expert
+  int32_t* rank;          // [A] rank of each assignment among its tile's rows of the expert
   int32_t* counts;        // [E]
   int32_t* offsets;       // [E+1]
   int32_t* mtile_prefix;  // [E+1] 128-row tiles per expert, prefix-summed
   int32_t* pad_offsets;   // [E+1] nullable
   uint32_t* tile_counter;
   uint32_t* done_counter;
-  uint32_t* flags;        // [num_tiles], zeroed before the launch
-  int32_t* agg;           // [num_tiles, E]
-  int32_t* incl;          // [num_tiles, E]
+  int32_t* agg;           // [num_tiles, E] each tile's count per expert
+  int32_t* tile_start;    // [num_tiles, E] each tile's first rank inside each expert
   int32_t* status;
 };
 

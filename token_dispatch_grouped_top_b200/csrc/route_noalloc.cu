@@ -3,8 +3,8 @@
 // Some callers cannot allocate device memory themselves: a plugin whose host framework
 // owns every device allocation, an embedded runtime with a fixed memory budget, or a
 // latency-critical request path where cudaMalloc's implicit device synchronisation is
-// not acceptable.  For them this entry point keeps its scratch (the lookback flags and
-// per-tile count vectors, the per-assignment ranks, the tile counters) in a file-scope
+// not acceptable.  For them this entry point keeps its scratch (the per-tile count
+// vectors and first ranks, the per-assignment ranks, the tile counters) in a file-scope
 // __device__ array of fixed size instead of a workspace.  It runs the same kernels as
 // moe_route_layout.
 //
@@ -18,7 +18,7 @@
 //    down and re-created (cudaDeviceReset) is picked up; make the first call on a device
 //    before any stream capture, since that lookup may load the library's module.
 //  - All calls share the one array.  Each call clears the parts that must start at zero
-//    (counters and lookback flags); calls whose executions overlap on the GPU (different
+//    (the tile counters); calls whose executions overlap on the GPU (different
 //    streams, or different host threads) race on the array and give wrong results.
 //  - The same shape rules and device check as moe_route_layout apply; device-side errors
 //    are latched into the caller's status word, which is therefore required.
@@ -38,19 +38,18 @@ constexpr int64_t kA = 256;
 inline int64_t up(int64_t x) { return (x + kA - 1) / kA * kA; }
 
 struct ScratchLayout {
-  int64_t counters, flags, agg, incl, rank, mtile, total, zero_bytes;
+  int64_t counters, agg, tstart, rank, mtile, total, zero_bytes;
 };
 
-// header: [0, 8) tile + done counters; flags follow, then the count vectors
+// header: [0, 8) tile + done counters, then the count vectors
 ScratchLayout scratch_layout(const moe_dims* D) {
   ScratchLayout L;
   const int64_t nt = moe::route_num_tiles(D->T), E = D->E, A = D->T * D->k;
   L.counters = 0;
-  L.flags = kA;
-  L.zero_bytes = L.flags + 4 * nt;
-  L.agg = up(L.zero_bytes);
-  L.incl = up(L.agg + 4 * nt * E);
-  L.rank = up(L.incl + 4 * nt * E);
+  L.zero_bytes = 8;
+  L.agg = kA;
+  L.tstart = up(L.agg + 4 * nt * E);
+  L.rank = up(L.tstart + 4 * nt * E);
   L.mtile = up(L.rank + 4 * A);
   L.total = up(L.mtile + 4 * (E + 1));
   return L;
@@ -104,7 +103,7 @@ extern "C" moe_status moe_route_layout_noalloc(const moe_dims* D, const float* l
       return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  // counters and lookback flags must start at zero; everything else is written before read
+  // the counters must start at zero; everything else is written before read
   if (cudaMemsetAsync(base, 0, L.zero_bytes, s) != cudaSuccess) return MOE_ERR_CUDA;
   moe::RouteParams P;
   P.logits = logits;
@@ -122,9 +121,8 @@ extern "C" moe_status moe_route_layout_noalloc(const moe_dims* D, const float* l
   P.pad_offsets = pad_offsets;
   P.tile_counter = reinterpret_cast<uint32_t*>(base + L.counters);
   P.done_counter = reinterpret_cast<uint32_t*>(base + L.counters + 4);
-  P.flags = reinterpret_cast<uint32_t*>(base + L.flags);
   P.agg = reinterpret_cast<int32_t*>(base + L.agg);
-  P.incl = reinterpret_cast<int32_t*>(base + L.incl);
+  P.tile_start = reinterpret_cast<int32_t*>(base + L.tstart);
   P.status = status;
   return moe::launch_route_layout(P, perm, inv_perm, sms, s) == cudaSuccess ? MOE_OK
                                                                             : MOE_ERR_CUDA;
