@@ -144,11 +144,12 @@ def algorithmic_bytes(case, bwd: bool, tail_rows=None) -> dict:
     A = T*k assignments (no tile padding), expert outputs and input gradients per
     assignment are bf16, weights are read once.
 
-    tail_rows (backward): the rows of the experts' partial last tiles.  The dgrad GEMM of
-    the down projection runs the SwiGLU backward in its epilogue for every other row, so G
-    is not stored for them: those rows' SwiGLU bytes (g|u and h^ read, [dg|du]^ written)
-    count in that GEMM's stage, and the SwiGLU stage keeps the tail rows (G written and
-    read) and the per-row partial sums of d(w) (f/128 fp32 each)."""
+    tail_rows (backward; given when the library fuses, i.e. for d >= 6144): the rows of
+    the experts' partial last tiles.  The dgrad GEMM of the down projection then runs the
+    SwiGLU backward in its epilogue for every other row, so G is not stored for them:
+    those rows' SwiGLU bytes (g|u and h^ read, [dg|du]^ written) count in that GEMM's
+    stage, and the SwiGLU stage keeps the tail rows (G written and read) and the per-row
+    partial sums of d(w) (f/128 fp32 each).  None: G for every row, as unfused."""
     T, d, f, E, k = case.T, case.d, case.f, case.E, case.k
     A = T * k
     mx = 1 + 1 / 32

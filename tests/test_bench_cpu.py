@@ -94,6 +94,26 @@ def test_layer_summary_closed_form():
     assert rb["bound"] == "hbm"
 
 
+@pytest.mark.parametrize("tail", [0, 1000, 65536])
+def test_fused_swiglu_byte_split(tail):
+    # Fusing the SwiGLU backward into the dgrad epilogue moves the full rows' SwiGLU bytes
+    # into the GEMM's stage and drops exactly their G round trip (2 bytes written and 2
+    # read per element, the survey's bf16 figure) for the d(w) partial sums (4 bytes per
+    # row and 128 features); every other stage keeps its bytes.
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    case = synth.CONFIGS["dsv3_bwd"]
+    A, f = case.T * case.k, case.f
+    plain = bench.algorithmic_bytes(case, True)
+    fused = bench.algorithmic_bytes(case, True, tail_rows=tail)
+    pair = ("bwd_dgrad_down", "bwd_swiglu")
+    saved = sum(plain[s] for s in pair) - sum(fused[s] for s in pair)
+    assert saved == pytest.approx((A - tail) * f * 4 - A * (f // 128) * 4)
+    assert {s: v for s, v in plain.items() if s not in pair} == \
+        {s: v for s, v in fused.items() if s not in pair}
+
+
 @pytest.mark.parametrize("with_bwd", [False, True])
 def test_cpu_baseline_fields(with_bwd):
     sys.path.insert(0, ROOT)
