@@ -139,7 +139,7 @@ def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, ms: float) ->
 
 
 def algorithmic_bytes(case, bwd: bool, tail_rows=None) -> dict:
-    """Bytes each stage must move by the method (the survey's per-unit figures times the
+    """Bytes each stage must move by the method (the per-unit figures of the method times the
     units of one step): MX bytes include the 1/32 scale overhead, activations count the
     A = T*k assignments (no tile padding), expert outputs and input gradients per
     assignment are bf16, weights are read once.

@@ -160,7 +160,7 @@ int64_t moe_min_tokens_for_waves(int32_t num_sms, int32_t waves, int32_t tile_m,
 
 const char* moe_status_string(moe_status s);
 
-/* ---- S1 + S2: routing and layout ------------------------------------------------------
+/* ---- routing and layout ---------------------------------------------------------------
  * Article lead and §01 (router picks experts per token; count tokens per expert, decide
  * placement, keep each expert's tokens contiguous).
  * logits [T,E] fp32 -> topk_idx [T,k] (top-k by logit, ties to the lower expert index,
@@ -217,7 +217,7 @@ moe_status moe_prepare_weights(const moe_dims* dims, const uint16_t* w_gate,
                                int32_t with_backward_copies, const moe_weights* out,
                                void* stream);
 
-/* ---- S1..S7: forward ------------------------------------------------------------------
+/* ---- forward --------------------------------------------------------------------------
  * Article §02/§03: route -> layout -> pull dispatch with fused MXFP8 quantisation ->
  * grouped GEMM gate/up with SwiGLU and MXFP8 requantisation in the epilogue -> grouped
  * GEMM down -> push combine / final weighted merge.
@@ -248,7 +248,7 @@ moe_status moe_forward_bf16(const moe_dims* dims, const uint16_t* wgu_t, const u
                             const uint16_t* x, const float* logits, uint16_t* out, void* ws,
                             size_t ws_bytes, void* stream);
 
-/* ---- S8: backward ---------------------------------------------------------------------
+/* ---- backward -------------------------------------------------------------------------
  * Article §01/§02 (backward = pull reverse-combine + push reverse-dispatch).
  * dout [T,d] bf16 + saved -> dx [T,d] bf16, dw_route [T,k] fp32 (d loss / d topk_w),
  * dWg, dWu [E,d,f] bf16, dWd [E,f,d] bf16.  Needs the backward weight copies.
@@ -307,7 +307,7 @@ moe_status moe_router_grads(const moe_dims* dims, const float* dlogits, const ui
                             const uint16_t* wr, float* dx_r, float* dwr, void* ws,
                             size_t ws_bytes, void* stream);
 
-/* ---- expert parallelism over NVLink (NEXT-2) ---------------------------------------------
+/* ---- expert parallelism over NVLink ------------------------------------------------------
  * Article §01 and §02: G GPUs ("ranks") each own E/G experts (rank r: experts
  * [r*E/G, (r+1)*E/G)) and route their own tokens; the owner of an expert pulls the rows it
  * needs from the tokens' GPUs by source and offset into its own memory (pull dispatch),
@@ -360,7 +360,7 @@ moe_status moe_ep_experts(const moe_dims* dims, int32_t rank, int32_t world,
 moe_status moe_ep_combine(const moe_dims* dims, const float* topk_w, const uint16_t* y,
                           const uint8_t* ys, uint16_t* out, int32_t* status, void* stream);
 
-/* ---- grouped block-scaled GEMM (the engine of S4/S5, exposed for direct use) ----------
+/* ---- grouped block-scaled GEMM (the engine of the expert FFN, exposed for direct use)
  * For each group g and each row r in [128*mtile_prefix[g], 128*mtile_prefix[g+1]):
  *   D[r, n] = sum_k A[r,k] * B[g*N + n, k],  n < N,  fp32 accumulation, fp32 output
  * with A [R,K] / B [G*N,K] MX (UMMA scales).  mtile_prefix [G+1] is device memory
@@ -397,18 +397,18 @@ moe_status moe_grouped_gemm_bf16(int32_t G, int64_t rows_a, int32_t N, int32_t K
 /* ---- per-stage timing (measurement support) ------------------------------------------
  * Stage ids of moe_forward / moe_backward launches. */
 typedef enum {
-  MOE_STAGE_ROUTE = 0,      /* S1+S2: routing, layout, perm/inv scatter                 */
-  MOE_STAGE_PERMUTE = 1,    /* S3: pull dispatch with MXFP8 quantisation                */
-  MOE_STAGE_GATEUP = 2,     /* S4: grouped GEMM gate/up + SwiGLU + requantisation        */
-  MOE_STAGE_DOWN = 3,       /* S5: grouped GEMM down                                    */
-  MOE_STAGE_COMBINE = 4,    /* S6: weighted combine / un-permute                        */
-  MOE_STAGE_BWD_DOUT = 5,   /* S8: dOut quantisation + gather                           */
+  MOE_STAGE_ROUTE = 0,      /* routing, layout, perm/inv scatter                       */
+  MOE_STAGE_PERMUTE = 1,    /* pull dispatch with MXFP8 quantisation                    */
+  MOE_STAGE_GATEUP = 2,     /* grouped GEMM gate/up + SwiGLU + requantisation            */
+  MOE_STAGE_DOWN = 3,       /* grouped GEMM down                                        */
+  MOE_STAGE_COMBINE = 4,    /* weighted combine / un-permute                            */
+  MOE_STAGE_BWD_DOUT = 5,   /* backward: dOut quantisation + gather                     */
   MOE_STAGE_BWD_DGRAD_DOWN = 6,
   MOE_STAGE_BWD_DGRAD_GATEUP = 7,
   MOE_STAGE_BWD_DX = 8,
   MOE_STAGE_BWD_TRANSPOSE = 9,
   MOE_STAGE_BWD_WGRAD = 10,
-  MOE_STAGE_BWD_SWIGLU = 11, /* S8: d(router weights) + SwiGLU backward + MX of dg|du   */
+  MOE_STAGE_BWD_SWIGLU = 11, /* d(router weights) + SwiGLU backward + MX of dg|du       */
   MOE_STAGE_EP_PULL = 12,   /* expert parallelism: receive layout + pull dispatch         */
   MOE_STAGE_EP_PUSH = 13,   /* expert parallelism: push of the expert outputs             */
   MOE_NUM_STAGES = 14

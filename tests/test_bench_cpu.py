@@ -74,7 +74,7 @@ def test_layer_summary_closed_form():
     assert r["bound"] == ("tensor" if t_fl >= t_by else "hbm")
     assert r["tensor_frac"] == pytest.approx(r["flops"] / 4.05e-3 / 2e15)
     assert r["frac_of_roof"] == pytest.approx(r["t_roof_ms"] / 4.05)
-    # the survey's per-unit bytes: logits + idx/w + perm/inv; x + permuted MX rows; bf16
+    # the method's per-unit bytes: logits + idx/w + perm/inv; x + permuted MX rows; bf16
     # expert outputs + out
     mv = (4 * case.T * case.E + 16 * A) + (2 * case.T * case.d + A * case.d * (1 + 1 / 32)) + \
         (2 * A * case.d + 2 * case.T * case.d)
@@ -98,7 +98,7 @@ def test_layer_summary_closed_form():
 def test_fused_swiglu_byte_split(tail):
     # Fusing the SwiGLU backward into the dgrad epilogue moves the full rows' SwiGLU bytes
     # into the GEMM's stage and drops exactly their G round trip (2 bytes written and 2
-    # read per element, the survey's bf16 figure) for the d(w) partial sums (4 bytes per
+    # read per element, counted in bf16) for the d(w) partial sums (4 bytes per
     # row and 128 features); every other stage keeps its bytes.
     sys.path.insert(0, ROOT)
     import bench

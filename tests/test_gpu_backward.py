@@ -1,4 +1,4 @@
-"""GPU parity of the backward pass (S8) against the fp64 oracle, end to end from the raw
+"""GPU parity of the backward pass against the fp64 oracle, end to end from the raw
 inputs.
 
 dX and d(routing weights) must reach relative Frobenius error <= 2e-3 and max-abs <=

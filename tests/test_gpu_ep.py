@@ -1,4 +1,4 @@
-"""Expert parallelism (NEXT-2) through the C ABI, its ranks run on one GPU in phase order:
+"""Expert parallelism through the C ABI, its ranks run on one GPU in phase order:
 each rank's buffers are separate allocations reached through the peer table, and every
 phase is launched only after the previous phase of all ranks (no kernel waits for another).
 

@@ -1,4 +1,4 @@
-"""GPU parity of S1/S2 (routing + layout) and of the MXFP8 quantiser, through the C ABI.
+"""GPU parity of routing + layout and of the MXFP8 quantiser, through the C ABI.
 
 Routing indices, counts, offsets, perm and inv must equal the oracle bit for bit; routing
 weights within 2e-6 (fp32 expf vs fp64 exp); quantised bytes and scales bit-exact.

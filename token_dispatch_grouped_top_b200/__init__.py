@@ -93,7 +93,7 @@ def workspace_view(ws, dims: Dims, op: int, name: str, nbytes: int):
 
 
 def route_layout(logits, k: int, score_fn: int = SCORE_SOFTMAX_TOPK, ws=None, stream=None):
-    """S1 + S2 on the device.  Returns dict of idx, w, counts, offsets, perm, inv, pad_offsets."""
+    """Routing and layout on the device.  Returns dict of idx, w, counts, offsets, perm, inv, pad_offsets."""
     torch = _torch()
     T, E = logits.shape
     dims = Dims(T, 256, 256, E, k, score_fn)

@@ -1,4 +1,4 @@
-// S8 support kernel: token-direction MXFP8 quantisation of the weight-gradient operands.
+// Backward support kernel: token-direction MXFP8 quantisation of the weight-gradient operands.
 //
 // Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72", §01/§02:
 // training adds a backward pass with two reverse communications (pull reverse-combine of

@@ -1,4 +1,4 @@
-// NEXT-2: expert parallelism -- the article's dispatch and combine between GPUs.
+// Expert parallelism: the article's dispatch and combine between GPUs.
 //
 // Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72":
 //   §01 -- the expert owner needs to know how many rows each GPU sends it and where they

@@ -1,5 +1,6 @@
-// S4 / S5 / S7: persistent grouped GEMM on the 5th-generation tensor cores with MXFP8
-// block scaling (tcgen05.mma kind::mxf8f6f4, E8M0 scales, fp32 accumulation in TMEM).
+// Expert FFN and its tile scheduling: persistent grouped GEMM on the 5th-generation tensor
+// cores with MXFP8 block scaling (tcgen05.mma kind::mxf8f6f4, E8M0 scales, fp32
+// accumulation in TMEM).
 //
 // Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72":
 //   §01 -- the grouped GEMM needs each expert's tokens contiguous, else it reorders again;

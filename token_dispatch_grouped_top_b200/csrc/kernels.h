@@ -277,7 +277,7 @@ struct SchedInitParams {
 };
 cudaError_t launch_sched_init(const SchedInitParams& P, cudaStream_t stream);
 
-// Expert parallelism (NEXT-2): the owner rank's receive layout, pull dispatch and push of
+// Expert parallelism: the owner rank's receive layout, pull dispatch and push of
 // the expert outputs, over the peers' buffers (moe_ep_peer table in device memory).
 struct EpParams {
   const moe_ep_peer* peers;  // [world]

@@ -1,4 +1,4 @@
-// MXFP8 quantisation kernels, the pull-dispatch gather (S3) and the push combine (S6).
+// MXFP8 quantisation kernels, the pull-dispatch gather and the push combine.
 //
 // Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72":
 //   §02 -- pull dispatch: the consumer fetches the rows it needs by source and offset and
@@ -153,7 +153,7 @@ cudaError_t launch_quant_cols(const QuantColsParams& P, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// S6: one CTA per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
+// Weighted combine, one CTA per token: out[t] = sum_j w[t,j] * Y[row of assignment (t, j)] (j
 // ascending, fp32; Y read as scaled fp16, each value times its block scale), rounded to
 // bf16.  With unit weights this is the backward's push reverse-dispatch, dX[t] = sum_j
 // dXa[row of (t, j)].  The CTA reads each of the token's k rows as one contiguous stretch
@@ -263,7 +263,7 @@ cudaError_t launch_combine(const CombineParams& P, int num_sms, cudaStream_t str
   return cudaGetLastError();
 }
 
-// S3, second half: the pull gather.  Each expert row fetches the MX codes and scales of its
+// Dispatch, second half: the pull gather.  Each expert row fetches the MX codes and scales of its
 // token by index from the per-token quantised copy (x quantised once per token, small
 // enough to stay in L2) and writes them to its padded position: the codes with bulk copies
 // through shared memory (the copy engine moves the bytes; one thread per warp issues

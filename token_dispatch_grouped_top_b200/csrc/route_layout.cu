@@ -1,4 +1,4 @@
-// S1 + S2: top-k routing and the per-expert layout.
+// Top-k routing and the per-expert layout.
 //
 // Article "Cursor's MoK achieves 2.37x performance boost on NVIDIA GB300 NVL72":
 //   lead / §01 -- the router picks a few experts per token at every step; before the

@@ -1,4 +1,4 @@
-// NEXT-4: the router GEMM in front of the routing step (logits = x . W_r^T, fp32) and its
+// The router GEMM in front of the routing step (logits = x . W_r^T, fp32) and its
 // backward (dx_r = bf16(G) . W_r, dW_r = bf16(G)^T . x), run on the grouped GEMM engine's
 // bf16 mode (tcgen05.mma kind::f16, fp32 accumulation in TMEM) as one-group problems.
 //
