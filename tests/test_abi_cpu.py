@@ -87,6 +87,37 @@ def test_noalloc_scratch_limit_is_host_logic(lib):
                                         None, None) == 1
 
 
+def _noalloc_fits(lib, T, E, k):
+    # With no status word a call that passed the scratch check stops at the null-pointer
+    # check (1) before touching the device; one over the limit stops at the shape check (2)
+    D = _dims(T=T, d=256, f=256, E=E, k=k, s=0)
+    rc = lib.moe_route_layout_noalloc(ctypes.byref(D), 16, 16, 16, 16, 16, 16, 16, None,
+                                      None, None)
+    assert rc in (1, 2), rc
+    return rc == 1
+
+
+@pytest.mark.parametrize("E,k", [(256, 8), (64, 6), (1024, 4), (8, 2), (33, 3)])
+def test_noalloc_scratch_formula(lib, E, k):
+    # the largest T the 8 MiB array takes equals the header's formula:
+    # 256 + 8*nt*E + 4*T*k + 4*(E+1) bytes, each term rounded up to 256, nt = ceil(T/64)
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    def need(T):
+        nt = (T + 63) // 64
+        return 256 + up(4 * nt * E) + up(4 * nt * E) + up(4 * T * k) + up(4 * (E + 1))
+
+    lo, hi = 1, 1 << 24
+    while lo < hi:                      # largest T with need(T) <= 8 MiB
+        mid = (lo + hi + 1) // 2
+        lo, hi = (mid, hi) if need(mid) <= 8 << 20 else (lo, mid - 1)
+    assert _noalloc_fits(lib, lo, E, k)
+    assert not _noalloc_fits(lib, lo + 1, E, k)
+    if (E, k) == (256, 8):
+        assert lo == 131024
+
+
 def test_null_and_workspace_checks(lib):
     D = _dims(T=16, d=256, f=256, E=8, k=2, s=0)
     rc = lib.moe_route_layout(ctypes.byref(D), None, None, None, None, None, None, None, None,
